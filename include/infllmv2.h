@@ -1,0 +1,227 @@
+/*
+ * infllmv2.h -- C ABI of the InfLLM-V2 dense-sparse switchable attention
+ * hot path for NVIDIA B200 (sm_100a).
+ *
+ * The method (InfLLM-V2: Dense-Sparse Switchable Attention for Seamless
+ * Short-to-Long Adaptation; abstract on the cochat.ai paper page) reuses the
+ * dense attention's parameters.  For a long input it works in two steps: it
+ * picks the key blocks that matter for each query, then runs attention over
+ * those blocks alone (reportify digest, Technical Mechanism).  A short input
+ * gets plain dense attention (InfLLM-V2 skill write-up, Architecture
+ * Overview, the dense pathway bullet).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All tensor pointers are DEVICE pointers (cudaMalloc'd or equivalent),
+ *   16-byte aligned, densely packed in the stated row-major layout.
+ * - bf16 = IEEE bfloat16 stored as uint16; fp32 = float.
+ * - Layouts (BSHD):  Q, O  [B, T, Hq,  d] bf16
+ *                    K, V  [B, T, Hkv, d] bf16
+ *                    Kc    [B, n_c, Hkv, 2, d] bf16, n_c = (T-32)/16 + 1 (0 if T < 32):
+ *                          each compressed key as the pair (hi, lo), value hi + lo
+ *                    idx   [B, Hkv, T, topk] int32
+ *                    lse   [B, Hq, T] fp32 (natural log)
+ * - GQA: query head h belongs to KV head g = h / (Hq/Hkv).
+ * - `stream` is a cudaStream_t passed as void*; NULL = legacy default stream.
+ *   Every call only ENQUEUES work on `stream` and returns; nothing
+ *   synchronises except infllmv2_get_status.
+ * - Ownership: the caller allocates and frees every buffer, workspace
+ *   included.  The library allocates no device memory; its only global state
+ *   is one status word per device in a static __device__ variable.  Inputs
+ *   are read-only; outputs are fully overwritten.
+ * - Return value: INFLLMV2_OK or a negative error code.  On a host-side error
+ *   nothing is enqueued.  Device-side conditions (a bounded wait that expired,
+ *   a decode sequence at capacity) set bits in the device status word, read
+ *   with infllmv2_get_status.
+ * - Built and supported: head_dim == 128, block_size == 64, cmp_kernel == 32,
+ *   cmp_stride == 16, causal == 1, Hq/Hkv in {1,2,4,8,16}.  Other values
+ *   return INFLLMV2_ERR_UNSUPPORTED.
+ */
+#ifndef INFLLMV2_H_
+#define INFLLMV2_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define INFLLMV2_OK                    0
+#define INFLLMV2_ERR_INVALID_ARG      -1  /* null pointer, bad shape, topk < forced count */
+#define INFLLMV2_ERR_UNSUPPORTED      -2  /* a value outside the built configuration, misaligned pointer */
+#define INFLLMV2_ERR_CUDA             -3  /* a CUDA runtime/driver call failed (launch, tensor map) */
+#define INFLLMV2_ERR_TIMEOUT          -4  /* a device-side bounded wait expired (reported by get_status) */
+#define INFLLMV2_ERR_WORKSPACE        -5  /* ws_bytes smaller than infllmv2_workspace_bytes() */
+#define INFLLMV2_ERR_DEVICE_CHECK     -6  /* a device-side argument check failed (reported by get_status) */
+
+/* Device status bits (infllmv2_get_status). */
+#define INFLLMV2_STATUS_TIMEOUT        0x1
+#define INFLLMV2_STATUS_SEQ_FULL       0x2  /* decode: seqlens[b] reached the cache capacity */
+
+/* The method's knobs.  Source of each: the sequence-length switch and the
+ * block size (skill write-up, Implementation Steps 2-3); compressed keys that
+ * aggregate tokens hierarchically, here by mean-pooling with window 32 and
+ * stride 16 (skill write-up, Core Concept); blocks kept for local context
+ * (the sliding pattern, ibid.) and the initial block; top-k block selection
+ * (reportify digest, Technical Mechanism). */
+typedef struct infllmv2_params {
+  int32_t B;                /* batch (sequences) */
+  int32_t T;                /* tokens per sequence; for decode: cache capacity Lmax */
+  int32_t Hq;               /* query heads */
+  int32_t Hkv;              /* key/value heads (GQA groups) */
+  int32_t head_dim;         /* d; must be 128 */
+  int32_t block_size;       /* key block size; must be 64 */
+  int32_t cmp_kernel;       /* compression window; must be 32 */
+  int32_t cmp_stride;       /* compression stride; must be 16 */
+  int32_t topk;             /* blocks attended per query row, forced ones included; 1..256 */
+  int32_t n_init;           /* always-kept initial blocks 0..n_init-1 */
+  int32_t n_local;          /* always-kept most recent blocks cur-n_local+1..cur */
+  int32_t switch_threshold; /* forward(): dense iff T <= switch_threshold */
+  float   scale;            /* softmax scale; 0 => 1/sqrt(head_dim) */
+  int32_t causal;           /* must be 1 */
+} infllmv2_params;
+
+/* Operations for infllmv2_workspace_bytes. */
+#define INFLLMV2_OP_SELECT   1
+#define INFLLMV2_OP_FORWARD  2
+#define INFLLMV2_OP_DECODE   3
+
+/* Path reported by infllmv2_forward. */
+#define INFLLMV2_PATH_DENSE  1
+#define INFLLMV2_PATH_SPARSE 2
+
+/*
+ * Compressed keys: Kc[b, j, g, :] = (1/32) * sum_{i=16j}^{16j+31} K[b, i, g, :]
+ * for j < n_c (the compressed pattern's token aggregation, skill write-up,
+ * Core Concept; mean-pooling with window 32, stride 16).  Sums in fp32 in
+ * token order and stores the mean m as two bf16 planes, hi = RNE(m) and
+ * lo = RNE(m - hi) (about 17 significant bits: a single bf16 rounding moves
+ * block scores by up to ~1e-2 relative, more than selection can absorb).
+ *   K  [B, T, Hkv, d] bf16 (in);  Kc [B, n_c, Hkv, 2, d] bf16 (out).
+ */
+int infllmv2_compress_keys(const infllmv2_params* p, const void* K, void* Kc,
+                           void* stream);
+
+/*
+ * Block selection (reportify digest, Technical Mechanism: the first of the
+ * two steps picks the relevant key/value blocks; scores are summed over the
+ * heads of a group, skill write-up, Architecture Overview, Hardware Kernel
+ * bullet).  For every
+ * (b, g, t):
+ *   s[h, j] = scale * Q[b,t,h,:] . Kc[b,j,g,:]   for the visible windows
+ *             j < v(t) = #{j : 16j + 31 <= t},  h in group g;
+ *   p[h, :] = softmax_j s[h, :];   S[j] = sum_{h in g} p[h, j];
+ *   bs[blk] = max { S[j] : window j overlaps block blk's tokens } (-inf if none);
+ *   forced  = {0..n_init-1} U {cur-n_local+1..cur}, cur = t / 64;
+ *   the other topk-|forced| slots take the blocks blk <= cur with the largest
+ *   bs, equal scores to the lower block.
+ *   idx[b, g, t, :] = selected blocks ascending, padded with -1.
+ *   Q  [B, T, Hq, d] bf16 (in);  Kc from infllmv2_compress_keys (in);
+ *   idx [B, Hkv, T, topk] int32 (out);
+ *   ws: device workspace of at least infllmv2_workspace_bytes(p, INFLLMV2_OP_SELECT)
+ *   bytes (block scores of every row; contents on return unspecified).
+ */
+int infllmv2_select_blocks(const infllmv2_params* p, const void* Q, const void* Kc,
+                           int32_t* idx, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Block-sparse causal attention (reportify digest, Technical Mechanism: the
+ * second step attends only to the picked blocks):
+ *   keys(t) = union over blk in idx[b, g, t, :] (blk >= 0) of [64 blk, 64 blk + 63],
+ *             clipped to [0, t];
+ *   O[b,t,h,:] = sum_{i in keys(t)} softmax_i(scale * q.K_i) V_i;
+ *   lse[b,h,t] = log sum_{i in keys(t)} exp(scale * q.K_i).
+ *   idx rows must be ascending with valid entries first (as select_blocks
+ *   writes them); entries > t/64 are ignored.
+ */
+int infllmv2_sparse_attn(const infllmv2_params* p, const void* Q, const void* K,
+                         const void* V, const int32_t* idx, void* O, float* lse,
+                         void* stream);
+
+/*
+ * Exact dense causal attention (skill write-up, Architecture Overview, the
+ * dense pathway bullet): keys(t) = [0, t], same O and lse
+ * definitions as infllmv2_sparse_attn.
+ */
+int infllmv2_dense_attn(const infllmv2_params* p, const void* Q, const void* K,
+                        const void* V, void* O, float* lse, void* stream);
+
+/*
+ * The switchable attention (skill write-up, Implementation Step 3: dense when
+ * seq_len <= threshold, else sparse).  Sparse: compress_keys into Kc_ws, then
+ * select_blocks into idx_ws, then sparse_attn.  Dense: dense_attn; Kc_ws and
+ * idx_ws may be NULL.  *path_used (host pointer, may be NULL) receives
+ * INFLLMV2_PATH_DENSE or INFLLMV2_PATH_SPARSE.
+ *   Kc_ws: [B, n_c, Hkv, 2, d] bf16; idx_ws: [B, Hkv, T, topk] int32 (both out);
+ *   ws: at least infllmv2_workspace_bytes(p, INFLLMV2_OP_FORWARD) bytes.
+ */
+int infllmv2_forward(const infllmv2_params* p, const void* Q, const void* K,
+                     const void* V, void* O, float* lse, void* Kc_ws, int32_t* idx_ws,
+                     int32_t* path_used, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * One decode step for B sequences (reportify digest, Performance Evaluation:
+ * the operator speed-up is reported for both prefill and decode).  p->T is the cache
+ * capacity Lmax in tokens; the compressed-key cache holds n_c(Lmax) rows.
+ * For every sequence b, with pos = seqlens[b] (device int32, pos < Lmax):
+ *   1. K_cache[b,pos] = k_new[b]; V_cache[b,pos] = v_new[b];
+ *   2. if pos >= 31 and (pos-31) % 16 == 0: Kc_cache[b,(pos-31)/16] = mean of
+ *      K_cache[b, pos-31 .. pos]  (incremental compressed-key cache);
+ *   3. the new token attends as query row t = pos exactly as select_blocks +
+ *      sparse_attn define it over the caches;
+ *   4. seqlens[b] = pos + 1.
+ *   q [B, Hq, d], k_new/v_new [B, Hkv, d] bf16 (in);
+ *   K_cache/V_cache [B, Lmax, Hkv, d] bf16, Kc_cache [B, n_c(Lmax), Hkv, 2, d] bf16,
+ *   seqlens [B] int32 (in/out);  O [B, Hq, d] bf16, lse [B, Hq] fp32 (out);
+ *   idx_out [B, Hkv, topk] int32 (out, may be NULL);
+ *   ws: at least infllmv2_workspace_bytes(p, INFLLMV2_OP_DECODE) bytes.
+ * A sequence with seqlens[b] >= Lmax is left untouched, its O/lse rows are
+ * zero and INFLLMV2_STATUS_SEQ_FULL is set.
+ */
+int infllmv2_decode_step(const infllmv2_params* p, const void* q, const void* k_new,
+                         const void* v_new, void* K_cache, void* V_cache, void* Kc_cache,
+                         int32_t* seqlens, void* O, float* lse, int32_t* idx_out,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* Device workspace bytes needed by an operation (0 if none; SIZE_MAX on bad params). */
+size_t infllmv2_workspace_bytes(const infllmv2_params* p, int32_t op);
+
+/* Number of compressed-key rows for T tokens: (T-32)/16 + 1, or 0 if T < 32. */
+int32_t infllmv2_num_compressed(int32_t T);
+
+/*
+ * Synchronises `stream`, returns the current device's status bits in
+ * *status_out (host pointer) and clears them.  Returns INFLLMV2_OK, or
+ * INFLLMV2_ERR_CUDA if the synchronisation itself failed (for example after
+ * an earlier kernel fault).
+ */
+int infllmv2_get_status(void* stream, int32_t* status_out);
+
+/*
+ * Time limit, in nanoseconds, of every device-side bounded wait (mbarrier
+ * polls; default 2e9 = 2 s).  A wait that runs out sets
+ * INFLLMV2_STATUS_TIMEOUT, abandons its loop and the kernel returns after
+ * releasing its tensor memory.  Takes effect for calls enqueued afterwards.
+ */
+void infllmv2_set_wait_limit(int64_t ns);
+
+/*
+ * Self-test of the timeout path: one CTA waits, with the current wait limit,
+ * on an mbarrier that nothing ever arrives on.  The wait expires, the kernel
+ * sets INFLLMV2_STATUS_TIMEOUT and returns; infllmv2_get_status then reports
+ * the bit and the context stays usable.
+ */
+int infllmv2_selftest_timeout(void* stream);
+
+/* Human-readable text of an error code. */
+const char* infllmv2_strerror(int code);
+
+/* Library version, e.g. 100 for 0.1.0. */
+int infllmv2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INFLLMV2_H_ */

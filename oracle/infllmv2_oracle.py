@@ -8,33 +8,35 @@ seeded inputs (bfloat16 bit patterns, widened exactly to float64).
 It is deliberately plain and slow: every query row is computed on its own,
 in float64, in the order the method states its steps:
 
-1. compressed keys: mean of each 32-token key window, windows every 16 tokens
-   ("Compressed Attention (hierarchical token aggregation)", InfLLM-V2 skill
-   write-up, Core Concept; kernel 32 / stride 16 are the method's settings);
+1. compressed keys: the mean of each 32-token key window, one window every
+   16 tokens (the compressed pattern aggregates tokens hierarchically:
+   InfLLM-V2 skill write-up, Core Concept; kernel 32 / stride 16 are the
+   method's settings);
 2. scores of one query token against the compressed keys it may see, a
    softmax per query head, then a sum over the query heads of each GQA group
-   ("LSE approximation fusing head-group summation", skill write-up,
-   Architecture Overview, Hardware Kernel bullet; computed here exactly);
+   (the group summation the skill write-up's Architecture Overview, Hardware
+   Kernel bullet, fuses into its attention loop with an LSE approximation;
+   computed here exactly);
 3. max-pool of the group score onto 64-token key blocks (block size 64,
    skill write-up, Implementation Step 2);
-4. block selection: the initial block and the local (sliding) blocks are
-   always kept, the other slots go to the highest-scoring blocks
-   ("block selection to determine relevant key-value subsets", reportify
-   digest, Technical Mechanism; "Sliding Attention (maintains local
-   context)", skill write-up, Core Concept);
-5. causal attention restricted to the keys of the selected blocks ("sparse
-   attention calculation only on selected subsets", reportify digest,
-   Technical Mechanism), and exact dense causal attention when the sequence
-   is not longer than the switch threshold (skill write-up, Architecture
-   Overview "Dense Pathway" and Implementation Step 3, where ``seq_len <=
-   threshold`` returns the dense result).
+4. block selection: the initial block and the local (sliding-window) blocks
+   are always kept, the other slots go to the highest-scoring blocks (the
+   first of two steps picks the relevant key/value blocks: reportify digest,
+   Technical Mechanism; the sliding pattern keeps local context: skill
+   write-up, Core Concept);
+5. causal attention over the keys of the selected blocks only (the second
+   step: reportify digest, Technical Mechanism), and exact dense causal
+   attention when the sequence is not longer than the switch threshold
+   (skill write-up, Architecture Overview, dense pathway bullet, and
+   Implementation Step 3, whose switch returns the dense result when the
+   length is at most the threshold).
 
 Readings where the pages are silent (each is listed in the design notes):
 
 * A compressed window ``j`` (tokens ``[16j, 16j+31]``) is visible to query
   token ``t`` only when it lies wholly at or before ``t``: ``16j + 31 <= t``
-  (causality: "ensure sliding window respects causality", skill write-up,
-  When NOT to Use).
+  (causality: the skill write-up's When NOT to Use list warns that the
+  sliding window must only look at past tokens).
 * The group sum adds per-head softmax *probabilities* (the pages tie the
   group summation to LSE, i.e. to normalised scores).
 * Block ``b`` pools every visible window that overlaps its tokens
@@ -203,18 +205,22 @@ class RowSelection:
     free_slots: int
 
 
-def select_row(Q: np.ndarray, Kc: np.ndarray, b: int, g: int, t: int,
-               p: Params) -> RowSelection:
-    """Selection for one (batch, kv head, query token)."""
-    Hq, Hkv = Q.shape[2], Kc.shape[2]
-    G = Hq // Hkv
-    q_group = Q[b, t, g * G:(g + 1) * G, :]
-    S = group_scores(q_group, Kc[b, :, g, :], t, p)
+def select_query(q_group: np.ndarray, Kc_g: np.ndarray, t: int, p: Params) -> RowSelection:
+    """Selection for the heads q_group [G, d] of query token t over Kc_g [n, d]."""
+    S = group_scores(q_group, Kc_g, t, p)
     bs = block_scores(S, t, p)
     chosen, ranked = select_from_scores(bs, t, p)
     forced = forced_blocks(t, p)
     return RowSelection(pad_row(chosen, p.topk), bs, ranked, forced,
                         p.topk - len(forced))
+
+
+def select_row(Q: np.ndarray, Kc: np.ndarray, b: int, g: int, t: int,
+               p: Params) -> RowSelection:
+    """Selection for one (batch, kv head, query token)."""
+    Hq, Hkv = Q.shape[2], Kc.shape[2]
+    G = Hq // Hkv
+    return select_query(Q[b, t, g * G:(g + 1) * G, :], Kc[b, :, g, :], t, p)
 
 
 def select_blocks(Q: np.ndarray, K: np.ndarray, p: Params,
@@ -381,10 +387,7 @@ def decode_query(K_seq: np.ndarray, V_seq: np.ndarray, Kc_seq: np.ndarray,
     idx = np.full((Hkv, p.topk), -1, dtype=np.int32)
     for g in range(Hkv):
         qg = q[g * G:(g + 1) * G]
-        S = group_scores(qg, Kc_seq[:, g, :], t, p)
-        bs = block_scores(S, t, p)
-        chosen, _ = select_from_scores(bs, t, p)
-        idx[g] = pad_row(chosen, p.topk)
+        idx[g] = select_query(qg, Kc_seq[:, g, :], t, p).idx
         keys = selected_keys(idx[g], t, p)
         o, lse = attend(qg, K_seq[:, g], V_seq[:, g], keys, p.sm_scale(d))
         O[g * G:(g + 1) * G] = o

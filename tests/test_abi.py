@@ -1,0 +1,102 @@
+"""The C ABI without a GPU: the library loads, exports every symbol the header
+declares, and rejects bad arguments on the host before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from trainable_block_sparse_compressed_b200 import infllmv2 as api
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "infllmv2.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(api._LIB_PATH):
+        from trainable_block_sparse_compressed_b200 import build
+        build.build()
+    return api.load()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(infllmv2_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_symbols() == sorted(api.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    nm = os.popen(f"nm -D --defined-only {api._LIB_PATH}").read()
+    for name in declared_symbols():
+        assert re.search(rf"\bT {name}\b", nm), name
+
+
+def test_host_helpers(lib):
+    assert lib.infllmv2_version() == 100
+    assert api.num_compressed(31) == 0
+    assert api.num_compressed(32) == 1
+    assert api.num_compressed(131072) == 8191
+    for code in [0, -1, -2, -3, -4, -5, -6]:
+        assert lib.infllmv2_strerror(code)
+
+
+def test_workspace_sizes(lib):
+    p = api.make_params(1, 131072, 32, 2, topk=64)
+    # causally packed block scores: sum_t (t//64 + 1) floats per (b, kv head)
+    T = 131072
+    per = sum((t // 64 + 1) for t in range(0, T, 64)) * 64
+    assert api.workspace_bytes(p, api.OP_SELECT) == 2 * per * 4
+    dense = api.make_params(2, 4096, 32, 2, switch_threshold=8192)
+    assert api.workspace_bytes(dense, api.OP_FORWARD) == 0
+    assert api.workspace_bytes(api.make_params(16, 131328, 32, 2), api.OP_DECODE) > 0
+    bad = api.make_params(1, 100, 32, 2, head_dim=64)
+    with pytest.raises(api.InfLLMV2Error):
+        api.workspace_bytes(bad, api.OP_SELECT)
+
+
+FAKE = 0x10000  # never dereferenced: validation fails first
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(head_dim=64), api.ERR_UNSUPPORTED),
+    (dict(block_size=32), api.ERR_UNSUPPORTED),
+    (dict(cmp_kernel=16), api.ERR_UNSUPPORTED),
+    (dict(cmp_stride=32), api.ERR_UNSUPPORTED),
+    (dict(Hq=24), api.ERR_UNSUPPORTED),        # G = 12
+    (dict(Hq=33), api.ERR_INVALID_ARG),        # Hq % Hkv != 0
+    (dict(topk=2), api.ERR_INVALID_ARG),       # < n_init + n_local
+    (dict(topk=257), api.ERR_INVALID_ARG),
+    (dict(n_local=-1), api.ERR_INVALID_ARG),
+    (dict(scale=-1.0), api.ERR_INVALID_ARG),
+])
+def test_bad_params_rejected_on_host(lib, kw, code):
+    base = dict(B=1, T=256, Hq=32, Hkv=2, topk=8)
+    base.update(kw)
+    p = api.make_params(**base)
+    P = ctypes.byref(p)
+    assert lib.infllmv2_select_blocks(P, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == code
+    assert lib.infllmv2_sparse_attn(P, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == code
+
+
+def test_null_and_misaligned_pointers(lib):
+    p = api.make_params(1, 256, 32, 2, topk=8)
+    P = ctypes.byref(p)
+    assert lib.infllmv2_compress_keys(P, None, FAKE, None) == api.ERR_INVALID_ARG
+    assert lib.infllmv2_compress_keys(P, FAKE + 2, FAKE, None) == api.ERR_UNSUPPORTED
+    assert lib.infllmv2_dense_attn(P, FAKE, FAKE, FAKE, None, FAKE, None) == api.ERR_INVALID_ARG
+    assert lib.infllmv2_select_blocks(P, FAKE, FAKE, FAKE, FAKE, 16, None) == api.ERR_WORKSPACE
+    assert lib.infllmv2_get_status(None, None) == api.ERR_INVALID_ARG
+
+
+def test_empty_problems_are_noops(lib):
+    p = api.make_params(0, 256, 32, 2, topk=8)
+    assert lib.infllmv2_compress_keys(ctypes.byref(p), None, None, None) == api.OK
+    p = api.make_params(1, 0, 32, 2, topk=8)
+    assert lib.infllmv2_sparse_attn(ctypes.byref(p), None, None, None, None, None, None, None) == api.OK

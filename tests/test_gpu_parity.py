@@ -1,0 +1,401 @@
+"""GPU parity against the fp64 oracle, through the C ABI.
+
+Small cases are compared element by element on every row; the full-size
+workloads (T = 32768, 131072; decode over a 131072-token cache) on sampled
+rows that the oracle computes one by one.  Attention kernels receive the
+ORACLE's block indices, so their outputs can be compared exactly against the
+oracle; the GPU's own selection is checked with the band rule.
+"""
+import numpy as np
+import pytest
+
+from oracle import infllmv2_oracle as orc
+from trainable_block_sparse_compressed_b200 import workloads as wl
+
+from _helpers import (LSE_ATOL, O_ATOL, check_selection_row, f64, gpu_bf16, sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+
+def _params(api, w, T=None, **kw):
+    T = w.T if T is None else T
+    d = dict(topk=w.topk, n_init=w.n_init, n_local=w.n_local, switch_threshold=w.threshold)
+    d.update(kw)
+    return api.make_params(w.B, T, w.Hq, w.Hkv, **d)
+
+
+def _oparams(w, **kw):
+    d = dict(topk=w.topk, n_init=w.n_init, n_local=w.n_local, threshold=w.threshold)
+    d.update(kw)
+    return orc.Params(**d)
+
+
+# ---------------------------------------------------------------------------
+# compressed keys
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("T,Hkv,B", [(31, 2, 1), (32, 2, 2), (1000, 2, 2), (4111, 1, 1),
+                                     (2048, 4, 1)])
+def test_compress_keys(cuda_lib, T, Hkv, B):
+    import torch
+    api = cuda_lib
+    w = wl.small_workload(B=B, T=T, Hq=Hkv * 4, Hkv=Hkv, needles=0, seed=T)
+    data = wl.make_prefill(w)
+    p = _params(api, w)
+    n_c = api.num_compressed(T)
+    K = gpu_bf16(data["K"])
+    Kc = torch.full((B, max(n_c, 1), Hkv, 2, 128), float("nan"), dtype=torch.bfloat16,
+                    device="cuda")
+    api.compress_keys(p, K, Kc)
+    torch.cuda.synchronize()
+    if n_c == 0:
+        return
+    ref = orc.compress_keys(wl.bf16_to_f64(data["K"]), orc.Params())
+    got = f64(Kc[:, :n_c])
+    hi, lo = got[..., 0, :], got[..., 1, :]
+    # hi is the bf16 rounding of the mean (one ulp at most off, from the fp32 sum)
+    ref_hi = wl.bf16_to_f64(wl.f32_to_bf16_bits(ref.astype(np.float32)))
+    assert np.all(np.abs(hi - ref_hi) <= np.abs(ref_hi) * 2.0 ** -7 + 1e-30)
+    assert np.mean(hi == ref_hi) > 0.999
+    # hi + lo carries ~17 significant bits: |hi + lo - mean| <= 2^-16 |mean| (+ fp32 sum error)
+    err = np.abs(hi + lo - ref)
+    assert np.all(err <= np.abs(ref) * 2.0 ** -16 + 1e-7), (err / (np.abs(ref) + 1e-30)).max()
+
+
+# ---------------------------------------------------------------------------
+# selection
+# ---------------------------------------------------------------------------
+SMALL = [
+    # (B, T, Hq, Hkv, topk, needles, seed)
+    (1, 2048, 8, 2, 8, 4, 1),     # the smallest evaluation workload
+    (2, 1000, 32, 2, 8, 2, 7),    # ragged T, G = 16, two sequences
+    (1, 777, 16, 1, 5, 2, 8),     # G = 16, single kv head
+    (1, 600, 8, 1, 4, 1, 9),      # G = 8
+    (1, 500, 4, 2, 6, 1, 10),     # G = 2
+    (1, 300, 2, 2, 3, 0, 11),     # G = 1, topk == forced count
+    (1, 129, 32, 2, 64, 0, 12),   # topk covers every block
+    (1, 33, 32, 2, 8, 0, 13),     # a single compressed window
+    (1, 20, 32, 2, 8, 0, 14),     # no compressed window at all
+]
+
+
+def _run_select(api, w, data):
+    import torch
+    p = _params(api, w)
+    n_c = api.num_compressed(w.T)
+    Q, K = gpu_bf16(data["Q"]), gpu_bf16(data["K"])
+    Kc = torch.empty((w.B, max(n_c, 1), w.Hkv, 2, 128), dtype=torch.bfloat16, device="cuda")
+    if n_c:
+        api.compress_keys(p, K, Kc)
+    idx = torch.full((w.B, w.Hkv, w.T, w.topk), -7, dtype=torch.int32, device="cuda")
+    ws = api.alloc_workspace(p, api.OP_SELECT)
+    api.select_blocks(p, Q, Kc, idx, ws)
+    torch.cuda.synchronize()
+    assert api.get_status() == 0
+    return idx.cpu().numpy()
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[f"B{c[0]}_T{c[1]}_Hq{c[2]}_Hkv{c[3]}_k{c[4]}" for c in SMALL])
+def test_select_blocks_all_rows(cuda_lib, case):
+    B, T, Hq, Hkv, topk, needles, seed = case
+    w = wl.small_workload(B=B, T=T, Hq=Hq, Hkv=Hkv, topk=topk, needles=needles, seed=seed)
+    data = wl.make_prefill(w)
+    got = _run_select(cuda_lib, w, data)
+    Q, K = wl.bf16_to_f64(data["Q"]), wl.bf16_to_f64(data["K"])
+    _, det = orc.select_blocks(Q, K, _oparams(w))
+    exact = 0
+    for (b, g, t), r in det.items():
+        exact += check_selection_row(r, got[b, g, t], topk)
+    assert exact >= 0.8 * len(det), f"only {exact}/{len(det)} rows exact"
+
+
+# ---------------------------------------------------------------------------
+# attention with the oracle's selection
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("case", SMALL, ids=[f"B{c[0]}_T{c[1]}_Hq{c[2]}_Hkv{c[3]}_k{c[4]}" for c in SMALL])
+def test_sparse_attn_all_rows(cuda_lib, case):
+    import torch
+    api = cuda_lib
+    B, T, Hq, Hkv, topk, needles, seed = case
+    w = wl.small_workload(B=B, T=T, Hq=Hq, Hkv=Hkv, topk=topk, needles=needles, seed=seed)
+    data = wl.make_prefill(w)
+    Q, K, V = (wl.bf16_to_f64(data[x]) for x in "QKV")
+    op = _oparams(w)
+    idx, _ = orc.select_blocks(Q, K, op)
+    O_ref, L_ref = orc.sparse_attention(Q, K, V, idx, op)
+    O = torch.empty((B, T, Hq, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, Hq, T), dtype=torch.float32, device="cuda")
+    api.sparse_attn(_params(api, w), gpu_bf16(data["Q"]), gpu_bf16(data["K"]), gpu_bf16(data["V"]),
+                    torch.from_numpy(idx).cuda(), O, lse)
+    torch.cuda.synchronize()
+    assert api.get_status() == 0
+    assert np.abs(f64(O) - O_ref).max() <= O_ATOL
+    assert np.abs(f64(lse) - L_ref).max() <= LSE_ATOL
+
+
+def test_sparse_attn_unsorted_padding_and_ignored_entries(cuda_lib):
+    """Rows shorter than topk (-1 padded) and entries beyond t//64 (ignored)."""
+    import torch
+    api = cuda_lib
+    w = wl.small_workload(B=1, T=400, Hq=32, Hkv=2, topk=6, needles=0, seed=21)
+    data = wl.make_prefill(w)
+    Q, K, V = (wl.bf16_to_f64(data[x]) for x in "QKV")
+    idx = np.full((1, 2, 400, 6), -1, dtype=np.int32)
+    rng = np.random.default_rng(0)
+    for g in range(2):
+        for t in range(400):
+            cur = t // 64
+            n = int(rng.integers(1, min(6, cur + 1) + 1))
+            blocks = sorted(rng.choice(cur + 1, size=n, replace=False).tolist())
+            row = blocks + ([cur + 1] if cur + 1 <= 6 and n < 6 else [])
+            idx[0, g, t, :len(row)] = row
+    op = orc.Params(topk=6)
+    O_ref, L_ref = orc.sparse_attention(Q, K, V, idx, op)
+    O = torch.empty((1, 400, 32, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((1, 32, 400), dtype=torch.float32, device="cuda")
+    api.sparse_attn(_params(api, w), gpu_bf16(data["Q"]), gpu_bf16(data["K"]), gpu_bf16(data["V"]),
+                    torch.from_numpy(idx).cuda(), O, lse)
+    torch.cuda.synchronize()
+    assert np.abs(f64(O) - O_ref).max() <= O_ATOL
+    assert np.abs(f64(lse) - L_ref).max() <= LSE_ATOL
+
+
+# ---------------------------------------------------------------------------
+# dense path and the switch
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("B,T,Hq,Hkv", [(1, 300, 32, 2), (2, 130, 8, 2), (1, 1, 16, 1)])
+def test_dense_attn_all_rows(cuda_lib, B, T, Hq, Hkv):
+    import torch
+    api = cuda_lib
+    w = wl.small_workload(B=B, T=T, Hq=Hq, Hkv=Hkv, needles=0, seed=T + Hq)
+    data = wl.make_prefill(w)
+    Q, K, V = (wl.bf16_to_f64(data[x]) for x in "QKV")
+    O_ref, L_ref = orc.dense_attention(Q, K, V, orc.Params())
+    O = torch.empty((B, T, Hq, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, Hq, T), dtype=torch.float32, device="cuda")
+    api.dense_attn(_params(api, w), gpu_bf16(data["Q"]), gpu_bf16(data["K"]), gpu_bf16(data["V"]), O, lse)
+    torch.cuda.synchronize()
+    assert np.abs(f64(O) - O_ref).max() <= O_ATOL
+    assert np.abs(f64(lse) - L_ref).max() <= LSE_ATOL
+
+
+def test_dense_switch_workload_sampled(cuda_lib):
+    """B=2, T=4096, Hq=32, Hkv=2 below the 8192 threshold: the switch must
+    take the dense path; sampled rows equal exact causal attention."""
+    api = cuda_lib
+    w = wl.WORKLOADS["dense_switch_B2_T4096_Hq32_Hkv2"]
+    data = wl.make_prefill(w)
+    O, lse, path, _ = api.prefill(gpu_bf16(data["Q"]), gpu_bf16(data["K"]), gpu_bf16(data["V"]),
+                                  topk=w.topk, threshold=w.threshold)
+    assert path == api.PATH_DENSE
+    Q, K, V = (wl.bf16_to_f64(data[x]) for x in "QKV")
+    rows = [(b, g, t) for b in range(2) for g in range(2) for t in sample_rows(w.T, 24, 5)]
+    O_ref, L_ref = orc.dense_attention(Q, K, V, orc.Params(), rows)
+    Og, Lg = f64(O), f64(lse)
+    G = w.Hq // w.Hkv
+    for (b, g, t) in rows:
+        hs = slice(g * G, (g + 1) * G)
+        assert np.abs(Og[b, t, hs] - O_ref[b, t, hs]).max() <= O_ATOL
+        assert np.abs(Lg[b, hs, t] - L_ref[b, hs, t]).max() <= LSE_ATOL
+
+
+def test_switch_takes_sparse_above_threshold(cuda_lib):
+    api = cuda_lib
+    w = wl.small_workload(B=1, T=576, Hq=32, Hkv=2, topk=4, needles=1, seed=3)
+    data = wl.make_prefill(w)
+    *_, path, idx = api.prefill(gpu_bf16(data["Q"]), gpu_bf16(data["K"]), gpu_bf16(data["V"]),
+                                topk=4, threshold=512)
+    assert path == api.PATH_SPARSE and idx is not None
+    *_, path2, idx2 = api.prefill(gpu_bf16(data["Q"]), gpu_bf16(data["K"]), gpu_bf16(data["V"]),
+                                  topk=4, threshold=576)
+    assert path2 == api.PATH_DENSE and idx2 is None
+
+
+# ---------------------------------------------------------------------------
+# full-size prefill workloads, sampled rows
+# ---------------------------------------------------------------------------
+def _full_prefill_check(api, name, n_rows, seed):
+    import torch
+    w = wl.WORKLOADS[name]
+    data = wl.make_prefill(w)
+    Qg, Kg, Vg = gpu_bf16(data["Q"]), gpu_bf16(data["K"]), gpu_bf16(data["V"])
+    O, lse, path, idx = api.prefill(Qg, Kg, Vg, topk=w.topk, threshold=w.threshold)
+    torch.cuda.synchronize()
+    assert path == api.PATH_SPARSE
+    assert api.get_status() == 0
+    Q, K, V = (wl.bf16_to_f64(data[x]) for x in "QKV")
+    op = _oparams(w)
+    needle_rows = [nd.query_block * 64 + 17 for nd in data["needles"][:8]]
+    ts = sample_rows(w.T, n_rows, seed, needle_rows)
+    rows = [(0, g, t) for g in range(w.Hkv) for t in ts]
+    oidx, det = orc.select_blocks(Q, K, op, rows)
+    gidx = idx.cpu().numpy()
+    exact = sum(check_selection_row(det[r], gidx[r], w.topk) for r in rows)
+    assert exact >= 0.5 * len(rows)
+    # attention at full size with the oracle's selection on the sampled rows
+    # (other rows keep the GPU's own selection; they are not compared)
+    full_idx = gidx.copy()
+    for r in rows:
+        full_idx[r] = oidx[r]
+    O2 = torch.empty_like(Qg)
+    lse2 = torch.empty_like(lse)
+    p = api.make_params(w.B, w.T, w.Hq, w.Hkv, topk=w.topk, switch_threshold=w.threshold)
+    api.sparse_attn(p, Qg, Kg, Vg, torch.from_numpy(full_idx).cuda(), O2, lse2)
+    torch.cuda.synchronize()
+    O_ref, L_ref = orc.sparse_attention(Q, K, V, oidx, op, rows)
+    Og, Lg = f64(O2), f64(lse2)
+    Of, Lf = f64(O), f64(lse)
+    G = w.Hq // w.Hkv
+    for (b, g, t) in rows:
+        hs = slice(g * G, (g + 1) * G)
+        assert np.abs(Og[b, t, hs] - O_ref[b, t, hs]).max() <= O_ATOL
+        assert np.abs(Lg[b, hs, t] - L_ref[b, hs, t]).max() <= LSE_ATOL
+        if np.array_equal(gidx[b, g, t], oidx[b, g, t]):   # forward() output too
+            assert np.abs(Of[b, t, hs] - O_ref[b, t, hs]).max() <= O_ATOL
+            assert np.abs(Lf[b, hs, t] - L_ref[b, hs, t]).max() <= LSE_ATOL
+
+
+def test_prefill_32k_sampled(cuda_lib):
+    _full_prefill_check(cuda_lib, "sparse_prefill_T32768_Hq32_Hkv2", 48, 3)
+
+
+def test_prefill_128k_sampled(cuda_lib):
+    _full_prefill_check(cuda_lib, "sparse_prefill_T131072_Hq32_Hkv2", 32, 4)
+
+
+# ---------------------------------------------------------------------------
+# decode
+# ---------------------------------------------------------------------------
+def _decode_setup(api, w, L0, steps, B):
+    import torch
+    data = wl.make_decode(w, L=L0, steps=steps, B=B)
+    Lmax = L0 + steps
+    p = api.make_params(B, Lmax, w.Hq, w.Hkv, topk=w.topk, n_init=w.n_init, n_local=w.n_local)
+    NC = api.num_compressed(Lmax)
+    Kc = torch.zeros((B, Lmax, w.Hkv, 128), dtype=torch.bfloat16, device="cuda")
+    Vc = torch.zeros_like(Kc)
+    Kc[:, :L0] = gpu_bf16(data["K0"])
+    Vc[:, :L0] = gpu_bf16(data["V0"])
+    Kcmp = torch.zeros((B, max(NC, 1), w.Hkv, 2, 128), dtype=torch.bfloat16, device="cuda")
+    p0 = api.make_params(B, L0, w.Hq, w.Hkv)
+    n0 = api.num_compressed(L0)
+    if n0:
+        tmp = torch.empty((B, n0, w.Hkv, 2, 128), dtype=torch.bfloat16, device="cuda")
+        api.compress_keys(p0, gpu_bf16(data["K0"]), tmp)
+        Kcmp[:, :n0] = tmp
+    seqlens = torch.full((B,), L0, dtype=torch.int32, device="cuda")
+    ws = api.alloc_workspace(p, api.OP_DECODE)
+    return data, p, Kc, Vc, Kcmp, seqlens, ws
+
+
+def test_decode_steps_small(cuda_lib):
+    import torch
+    api = cuda_lib
+    w = wl.WORKLOADS["sparse_decode_B16_L131072_Hq32_Hkv2"]
+    B, L0, steps = 3, 990, 40
+    data, p, Kc, Vc, Kcmp, seqlens, ws = _decode_setup(api, w, L0, steps, B)
+    op = orc.Params(topk=w.topk)
+    st = orc.DecodeState.from_prefill(wl.bf16_to_f64(data["K0"]), wl.bf16_to_f64(data["V0"]), op)
+    O = torch.empty((B, w.Hq, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, w.Hq), dtype=torch.float32, device="cuda")
+    idx = torch.empty((B, w.Hkv, w.topk), dtype=torch.int32, device="cuda")
+    for s in range(steps):
+        q = gpu_bf16(data["q"][s])
+        api.decode_step(p, q, gpu_bf16(data["k_new"][s]), gpu_bf16(data["v_new"][s]), Kc, Vc, Kcmp,
+                        seqlens, O, lse, idx, ws)
+        torch.cuda.synchronize()
+        qf = wl.bf16_to_f64(data["q"][s])
+        O_ref, L_ref, i_ref = orc.decode_step(st, qf, wl.bf16_to_f64(data["k_new"][s]),
+                                              wl.bf16_to_f64(data["v_new"][s]), op)
+        gi = idx.cpu().numpy()
+        Og, Lg = f64(O), f64(lse)
+        G = w.Hq // w.Hkv
+        t = L0 + s
+        for b in range(B):
+            for g in range(w.Hkv):
+                r = orc.select_query(qf[b, g * G:(g + 1) * G], st.Kc[b][:, g], t, op)
+                check_selection_row(r, gi[b, g], w.topk)
+                if np.array_equal(gi[b, g], i_ref[b, g]):
+                    hs = slice(g * G, (g + 1) * G)
+                    assert np.abs(Og[b, hs] - O_ref[b, hs]).max() <= O_ATOL
+                    assert np.abs(Lg[b, hs] - L_ref[b, hs]).max() <= LSE_ATOL
+    assert api.get_status() == 0
+    assert seqlens.cpu().tolist() == [L0 + steps] * B
+    # incremental compressed keys == batch compression of the final cache
+    Lf = L0 + steps
+    nf = api.num_compressed(Lf)
+    batch = torch.empty((B, nf, w.Hkv, 2, 128), dtype=torch.bfloat16, device="cuda")
+    api.compress_keys(api.make_params(B, Lf, w.Hq, w.Hkv), Kc[:, :Lf].contiguous(), batch)
+    torch.cuda.synchronize()
+    assert torch.equal(batch, Kcmp[:, :nf])
+
+
+def test_decode_full_cache_sampled(cuda_lib):
+    """B=16 sequences over a 131072-token cache: one step, two sequences
+    checked against the oracle (selection by the band rule, output exact)."""
+    import torch
+    api = cuda_lib
+    w = wl.WORKLOADS["sparse_decode_B16_L131072_Hq32_Hkv2"]
+    B, L0, steps = 16, w.T, 2
+    data, p, Kc, Vc, Kcmp, seqlens, ws = _decode_setup(api, w, L0, steps, B)
+    O = torch.empty((B, w.Hq, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, w.Hq), dtype=torch.float32, device="cuda")
+    idx = torch.empty((B, w.Hkv, w.topk), dtype=torch.int32, device="cuda")
+    api.decode_step(p, gpu_bf16(data["q"][0]), gpu_bf16(data["k_new"][0]), gpu_bf16(data["v_new"][0]),
+                    Kc, Vc, Kcmp, seqlens, O, lse, idx, ws)
+    torch.cuda.synchronize()
+    assert api.get_status() == 0
+    op = orc.Params(topk=w.topk)
+    gi = idx.cpu().numpy()
+    Og, Lg = f64(O), f64(lse)
+    for b in (0, 11):
+        K0 = wl.bf16_to_f64(data["K0"][b])
+        V0 = wl.bf16_to_f64(data["V0"][b])
+        Kseq = np.concatenate([K0, wl.bf16_to_f64(data["k_new"][0][b])[None]], axis=0)
+        Vseq = np.concatenate([V0, wl.bf16_to_f64(data["v_new"][0][b])[None]], axis=0)
+        Kc_seq = orc.compress_keys(Kseq[None], op)[0]
+        qf = wl.bf16_to_f64(data["q"][0][b])
+        t = L0
+        G = w.Hq // w.Hkv
+        O_ref, L_ref, i_ref = orc.decode_query(Kseq, Vseq, Kc_seq, qf, t, op)
+        for g in range(w.Hkv):
+            r = orc.select_query(qf[g * G:(g + 1) * G], Kc_seq[:, g], t, op)
+            check_selection_row(r, gi[b, g], w.topk)
+            if np.array_equal(gi[b, g], i_ref[g]):
+                hs = slice(g * G, (g + 1) * G)
+                assert np.abs(Og[b, hs] - O_ref[hs]).max() <= O_ATOL
+                assert np.abs(Lg[b, hs] - L_ref[hs]).max() <= LSE_ATOL
+
+
+def test_decode_full_sequence_is_reported(cuda_lib):
+    import torch
+    api = cuda_lib
+    w = wl.WORKLOADS["sparse_decode_B16_L131072_Hq32_Hkv2"]
+    B, L0 = 2, 200
+    data, p, Kc, Vc, Kcmp, seqlens, ws = _decode_setup(api, w, L0, 1, B)
+    seqlens[1] = L0 + 1  # == capacity: sequence 1 is full
+    O = torch.full((B, w.Hq, 128), 3.0, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, w.Hq), dtype=torch.float32, device="cuda")
+    api.decode_step(p, gpu_bf16(data["q"][0]), gpu_bf16(data["k_new"][0]), gpu_bf16(data["v_new"][0]),
+                    Kc, Vc, Kcmp, seqlens, O, lse, None, ws)
+    st = api.get_status()
+    assert st & api.STATUS_SEQ_FULL
+    assert seqlens.cpu().tolist() == [L0 + 1, L0 + 1]
+    assert float(O[1].abs().max()) == 0.0
+
+
+# ---------------------------------------------------------------------------
+# bounded waits
+# ---------------------------------------------------------------------------
+def test_timeout_selftest_reports_and_context_survives(cuda_lib):
+    import torch
+    api = cuda_lib
+    assert api.get_status() == 0
+    api.set_wait_limit(1_000_000)  # 1 ms
+    try:
+        api.selftest_timeout()
+        assert api.get_status() & api.STATUS_TIMEOUT
+    finally:
+        api.set_wait_limit(2_000_000_000)
+    assert api.get_status() == 0
+    # the context still runs real work
+    test_compress_keys(cuda_lib, 1000, 2, 2)

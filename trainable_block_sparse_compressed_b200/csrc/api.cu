@@ -1,0 +1,270 @@
+// api.cu -- the C ABI declared in include/infllmv2.h: argument validation,
+// the per-device status word, and the order in which each entry point
+// enqueues its kernels.
+#include <math.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace infllmv2 {
+
+// The library's only global device state: one status word per device (each
+// device that loads the module gets its own copy of this variable).
+__device__ int g_status_word;
+
+namespace {
+
+std::atomic<uint64_t> g_wait_ns{2000000000ull};  // 2 s
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int* g_status_ptr[kMaxDevices] = {};
+int g_sm_count[kMaxDevices] = {};
+
+int current_device() {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess) return -1;
+  return d;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+cudaError_t get_dev_ctx(DevCtx* ctx) {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_status_ptr[d]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_status_word);
+    if (e != cudaSuccess) return e;
+    g_status_ptr[d] = static_cast<int*>(p);
+  }
+  ctx->status = g_status_ptr[d];
+  ctx->wait_ns = g_wait_ns.load();
+  return cudaSuccess;
+}
+
+int sm_count() {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return 148;
+  if (!g_sm_count[d]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d);
+    g_sm_count[d] = n > 0 ? n : 148;
+  }
+  return g_sm_count[d];
+}
+
+namespace {
+
+// Checks the configuration shared by every entry point; fills `g`.
+int validate(const infllmv2_params* p, bool needs_topk, Geometry* g) {
+  if (!p) return INFLLMV2_ERR_INVALID_ARG;
+  if (p->B < 0 || p->T < 0 || p->Hq <= 0 || p->Hkv <= 0) return INFLLMV2_ERR_INVALID_ARG;
+  if (p->Hq % p->Hkv != 0) return INFLLMV2_ERR_INVALID_ARG;
+  if (p->head_dim != kHeadDim || p->block_size != kBlock || p->cmp_kernel != kCmpKernel ||
+      p->cmp_stride != kCmpStride || p->causal != 1)
+    return INFLLMV2_ERR_UNSUPPORTED;
+  const int G = p->Hq / p->Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return INFLLMV2_ERR_UNSUPPORTED;
+  if (!(p->scale >= 0.f) || isinf(p->scale)) return INFLLMV2_ERR_INVALID_ARG;
+  if (needs_topk) {
+    if (p->topk < 1 || p->topk > kMaxTopk || p->n_init < 0 || p->n_local < 0 ||
+        p->n_init + p->n_local > p->topk)
+      return INFLLMV2_ERR_INVALID_ARG;
+  }
+  if (static_cast<int64_t>(p->T) > (1 << 22)) return INFLLMV2_ERR_UNSUPPORTED;
+  g->B = p->B;
+  g->T = p->T;
+  g->Hq = p->Hq;
+  g->Hkv = p->Hkv;
+  g->G = G;
+  g->n_c = num_compressed(p->T);
+  g->topk = p->topk;
+  g->n_init = p->n_init;
+  g->n_local = p->n_local;
+  g->scale = p->scale > 0.f ? p->scale : 1.0f / sqrtf(static_cast<float>(kHeadDim));
+  g->scale_log2 = g->scale * 1.4426950408889634f;
+  return INFLLMV2_OK;
+}
+
+bool empty(const Geometry& g) { return g.B == 0 || g.T == 0; }
+
+// One warp waits on an mbarrier that nothing arrives on; the bounded wait
+// expires, reports INFLLMV2_STATUS_TIMEOUT and the kernel returns.
+__global__ void selftest_wait_kernel(DevCtx ctx) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait(&bar, 0, ctx.wait_ns))
+    report_status(ctx.status, INFLLMV2_STATUS_TIMEOUT);
+}
+
+int check_ptrs(std::initializer_list<const void*> ptrs) {
+  for (const void* q : ptrs) {
+    if (!q) return INFLLMV2_ERR_INVALID_ARG;
+    if (!aligned16(q)) return INFLLMV2_ERR_UNSUPPORTED;
+  }
+  return INFLLMV2_OK;
+}
+
+size_t select_ws_bytes(const Geometry& g) {
+  return static_cast<size_t>(g.B) * g.Hkv * static_cast<size_t>(score_row_offset(g.T)) *
+         sizeof(float);
+}
+
+int ctx_or_error(DevCtx* ctx) {
+  return get_dev_ctx(ctx) == cudaSuccess ? INFLLMV2_OK : INFLLMV2_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace infllmv2
+
+using namespace infllmv2;
+
+extern "C" {
+
+int infllmv2_version(void) { return 100; }
+
+int32_t infllmv2_num_compressed(int32_t T) { return num_compressed(T); }
+
+const char* infllmv2_strerror(int code) {
+  switch (code) {
+    case INFLLMV2_OK: return "ok";
+    case INFLLMV2_ERR_INVALID_ARG: return "invalid argument";
+    case INFLLMV2_ERR_UNSUPPORTED: return "unsupported configuration or misaligned pointer";
+    case INFLLMV2_ERR_CUDA: return "CUDA call failed";
+    case INFLLMV2_ERR_TIMEOUT: return "device wait limit exceeded";
+    case INFLLMV2_ERR_WORKSPACE: return "workspace too small";
+    case INFLLMV2_ERR_DEVICE_CHECK: return "device-side argument check failed";
+    default: return "unknown error";
+  }
+}
+
+void infllmv2_set_wait_limit(int64_t ns) {
+  g_wait_ns.store(ns < 0 ? 0ull : static_cast<uint64_t>(ns));
+}
+
+size_t infllmv2_workspace_bytes(const infllmv2_params* p, int32_t op) {
+  Geometry g;
+  if (validate(p, op != 0, &g) != INFLLMV2_OK) return SIZE_MAX;
+  switch (op) {
+    case INFLLMV2_OP_SELECT: return select_ws_bytes(g);
+    case INFLLMV2_OP_FORWARD: return p->T <= p->switch_threshold ? 0 : select_ws_bytes(g);
+    case INFLLMV2_OP_DECODE: return decode_ws_bytes(g);
+    default: return SIZE_MAX;
+  }
+}
+
+int infllmv2_compress_keys(const infllmv2_params* p, const void* K, void* Kc, void* stream) {
+  Geometry g;
+  if (int e = validate(p, false, &g)) return e;
+  if (empty(g) || g.n_c == 0) return INFLLMV2_OK;
+  if (int e = check_ptrs({K, Kc})) return e;
+  return launch_compress_keys(g, K, Kc, 0, static_cast<cudaStream_t>(stream));
+}
+
+int infllmv2_select_blocks(const infllmv2_params* p, const void* Q, const void* Kc, int32_t* idx,
+                           void* ws, size_t ws_bytes, void* stream) {
+  Geometry g;
+  if (int e = validate(p, true, &g)) return e;
+  if (empty(g)) return INFLLMV2_OK;
+  if (int e = check_ptrs({Q, idx, ws})) return e;
+  if (g.n_c > 0)
+    if (int e = check_ptrs({Kc})) return e;
+  if (ws_bytes < select_ws_bytes(g)) return INFLLMV2_ERR_WORKSPACE;
+  DevCtx ctx;
+  if (int e = ctx_or_error(&ctx)) return e;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* scores = static_cast<float*>(ws);
+  if (int e = launch_score_blocks(g, Q, Kc, scores, ctx, st)) return e;
+  return launch_topk(g, scores, idx, st);
+}
+
+int infllmv2_sparse_attn(const infllmv2_params* p, const void* Q, const void* K, const void* V,
+                         const int32_t* idx, void* O, float* lse, void* stream) {
+  Geometry g;
+  if (int e = validate(p, true, &g)) return e;
+  if (empty(g)) return INFLLMV2_OK;
+  if (int e = check_ptrs({Q, K, V, idx, O, lse})) return e;
+  DevCtx ctx;
+  if (int e = ctx_or_error(&ctx)) return e;
+  return launch_sparse_attn(g, Q, K, V, idx, O, lse, 0, ctx, static_cast<cudaStream_t>(stream));
+}
+
+int infllmv2_dense_attn(const infllmv2_params* p, const void* Q, const void* K, const void* V,
+                        void* O, float* lse, void* stream) {
+  Geometry g;
+  if (int e = validate(p, false, &g)) return e;
+  if (empty(g)) return INFLLMV2_OK;
+  if (int e = check_ptrs({Q, K, V, O, lse})) return e;
+  DevCtx ctx;
+  if (int e = ctx_or_error(&ctx)) return e;
+  return launch_sparse_attn(g, Q, K, V, nullptr, O, lse, 1, ctx,
+                            static_cast<cudaStream_t>(stream));
+}
+
+int infllmv2_forward(const infllmv2_params* p, const void* Q, const void* K, const void* V,
+                     void* O, float* lse, void* Kc_ws, int32_t* idx_ws, int32_t* path_used,
+                     void* ws, size_t ws_bytes, void* stream) {
+  if (!p) return INFLLMV2_ERR_INVALID_ARG;
+  const bool dense = p->T <= p->switch_threshold;
+  if (path_used) *path_used = dense ? INFLLMV2_PATH_DENSE : INFLLMV2_PATH_SPARSE;
+  if (dense) return infllmv2_dense_attn(p, Q, K, V, O, lse, stream);
+  Geometry g;
+  if (int e = validate(p, true, &g)) return e;
+  if (empty(g)) return INFLLMV2_OK;
+  if (g.n_c > 0)
+    if (int e = infllmv2_compress_keys(p, K, Kc_ws, stream)) return e;
+  if (int e = infllmv2_select_blocks(p, Q, Kc_ws, idx_ws, ws, ws_bytes, stream)) return e;
+  return infllmv2_sparse_attn(p, Q, K, V, idx_ws, O, lse, stream);
+}
+
+int infllmv2_decode_step(const infllmv2_params* p, const void* q, const void* k_new,
+                         const void* v_new, void* K_cache, void* V_cache, void* Kc_cache,
+                         int32_t* seqlens, void* O, float* lse, int32_t* idx_out, void* ws,
+                         size_t ws_bytes, void* stream) {
+  Geometry g;
+  if (int e = validate(p, true, &g)) return e;
+  if (g.B == 0) return INFLLMV2_OK;
+  if (g.T < 1) return INFLLMV2_ERR_INVALID_ARG;
+  if (int e = check_ptrs({q, k_new, v_new, K_cache, V_cache, seqlens, O, lse, ws})) return e;
+  if (g.n_c > 0)
+    if (int e = check_ptrs({Kc_cache})) return e;
+  if (idx_out && !aligned16(idx_out)) return INFLLMV2_ERR_UNSUPPORTED;
+  if (ws_bytes < decode_ws_bytes(g)) return INFLLMV2_ERR_WORKSPACE;
+  DevCtx ctx;
+  if (int e = ctx_or_error(&ctx)) return e;
+  return launch_decode_step(g, q, k_new, v_new, K_cache, V_cache, Kc_cache, seqlens, O, lse,
+                            idx_out, ws, ctx, static_cast<cudaStream_t>(stream));
+}
+
+int infllmv2_selftest_timeout(void* stream) {
+  DevCtx ctx;
+  if (int e = ctx_or_error(&ctx)) return e;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(ctx);
+  return cudaGetLastError() == cudaSuccess ? INFLLMV2_OK : INFLLMV2_ERR_CUDA;
+}
+
+int infllmv2_get_status(void* stream, int32_t* status_out) {
+  if (!status_out) return INFLLMV2_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return INFLLMV2_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status_word, sizeof(int)) != cudaSuccess) return INFLLMV2_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_status_word, &zero, sizeof(int)) != cudaSuccess)
+    return INFLLMV2_ERR_CUDA;
+  *status_out = v;
+  return INFLLMV2_OK;
+}
+
+}  // extern "C"

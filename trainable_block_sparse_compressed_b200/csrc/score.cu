@@ -1,0 +1,359 @@
+// score.cu -- block scores for block selection.
+//
+// For every query token t of a (batch, kv head g) the method needs
+//   p[h, j] = softmax_j(scale * q[t,h] . Kc[j])   over the visible windows j < v(t),
+//   S[j]    = sum over the query heads h of group g of p[h, j],
+//   bs[blk] = max of S over the windows overlapping block blk
+// (InfLLM-V2 skill write-up, Architecture Overview, Hardware Kernel bullet:
+// scores are summed over the heads of a group; block size 64, Implementation
+// Step 2; windows of 32 tokens every 16, Core Concept).  The softmax needs
+// each head's log-sum-exp over all visible windows before any probability can
+// be summed, so the kernel makes two passes over the compressed keys.
+//
+// One CTA owns a 128-row query tile: 128/G consecutive tokens x the G heads
+// of one group, rows ordered (token, head) -- exactly the box a single TMA
+// load of the BSHD query tensor produces.  Compressed-key tiles of 128 rows
+// stream through a 2-stage TMA ring.  Both passes run the same tcgen05.mma
+// (M = N = 128, bf16 in, fp32 accumulate in tensor memory) over K = 2 x 128:
+// each compressed key is the bf16 pair hi + lo, so q . Kc = q . hi + q . lo
+// is accumulated in one tile (a single bf16 rounding of the keys would move
+// block scores by up to ~1e-2 relative):
+//
+//   pass 1  D = Q  x Kc^T : a TMEM lane is a query row; each thread keeps the
+//           running max / sum of its row -> per-row LSE, no cross-lane work;
+//   pass 2  D = Kc x Q^T  : operands swapped, a TMEM lane is a compressed key
+//           j and the thread holds all (token, head) scores of that key, so
+//           the group sum over heads is a register sum, and the max-pool over
+//           windows 4b-1 .. 4b+3 is two xor-shuffles plus one shuffle-up
+//           across neighbouring lanes (neighbouring windows).
+//
+// Warp roles: warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs, warps
+// 2-5 (128 threads = 128 TMEM lanes) run the softmax / pooling epilogue.  The
+// accumulator is double-buffered in TMEM (2 x 128 columns) so the MMA of tile
+// i+1 overlaps the epilogue of tile i.  Block scores go to a causally packed
+// fp32 workspace (row t holds t/64 + 1 scores) for the top-k kernel.
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace infllmv2 {
+namespace {
+
+constexpr int kRows = 128;                 // query rows per tile (M of pass 1)
+constexpr int kKcTile = 128;               // compressed keys per tile
+constexpr int kStages = 2;
+constexpr int kHalfBytes = kRows * 64 * 2; // one 64-channel half of a 128-row tile
+constexpr int kTileBytes = 2 * kHalfBytes; // 32 KB: the query tile
+constexpr int kKcBytes = 4 * kHalfBytes;   // 64 KB: hi and lo planes of 128 compressed keys
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 256;
+
+struct ScoreSmem {
+  uint64_t q_full;
+  uint64_t kc_full[kStages];
+  uint64_t kc_empty[kStages];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  float lse2[kRows];                 // per query row: log2-domain LSE
+  float carry[3][4][kRows];          // S of the window just before each 32-lane quadrant
+};
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, const DevCtx& ctx,
+                                              volatile int* abort_flag) {
+  if (*abort_flag) return false;
+  if (mbar_wait(bar, parity, ctx.wait_ns)) return true;
+  report_status(ctx.status, INFLLMV2_STATUS_TIMEOUT);
+  *abort_flag = 1;
+  return false;
+}
+
+template <int G>
+__global__ void __launch_bounds__(kThreads, 1)
+    score_blocks_kernel(const __grid_constant__ CUtensorMap tmQ,
+                        const __grid_constant__ CUtensorMap tmKc, float* __restrict__ scores,
+                        int B, int T, int Hkv, int n_c, float scale_log2, DevCtx ctx) {
+  constexpr int TPT = kRows / G;  // tokens per tile
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* sQ = base;
+  uint8_t* sKc = base + kTileBytes;
+  ScoreSmem& sm = *reinterpret_cast<ScoreSmem*>(base + kTileBytes + kKcBytes * kStages);
+
+  // heaviest (latest) query tiles first
+  const int n_qt = (T + TPT - 1) / TPT;
+  const int bg = blockIdx.x % (B * Hkv);
+  const int qt = n_qt - 1 - static_cast<int>(blockIdx.x / (B * Hkv));
+  const int b = bg / Hkv, g = bg % Hkv;
+  const int t0 = qt * TPT;
+  const int t_last = min(t0 + TPT - 1, T - 1);
+  const int v_max = min(n_c, visible_windows(t_last));
+  const int n_t = (v_max + kKcTile - 1) / kKcTile;
+  const int n_it = 2 * n_t;
+
+  const int warp = warp_id(), lane = lane_id();
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.kc_full[s], 1);
+      mbar_init(&sm.kc_empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&sm.acc_full[a], 1);
+      mbar_init(&sm.acc_empty[a], 128);
+    }
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  if (threadIdx.x >= 64) {
+    const int r = threadIdx.x - 64;
+    for (int k = 0; k < 3 * 4; ++k) (&sm.carry[0][0][0])[k * kRows + r] = -INFINITY;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort_flag = &sm.abort_flag;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0 && n_t > 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmKc);
+      mbar_arrive_expect_tx(&sm.q_full, kTileBytes);
+      tma_load_4d(sQ, &tmQ, &sm.q_full, 0, g * G, t0, b);
+      tma_load_4d(sQ + kHalfBytes, &tmQ, &sm.q_full, 64, g * G, t0, b);
+      int issued = 0;
+      for (int it = 0; it < n_it; ++it) {
+        const int s = it % kStages;
+        const int i = it < n_t ? it : it - n_t;
+        if (it >= kStages &&
+            !wait_or_abort(&sm.kc_empty[s], ((it / kStages) & 1) ^ 1, ctx, abort_flag))
+          break;
+        uint8_t* dst = sKc + s * kKcBytes;
+        mbar_arrive_expect_tx(&sm.kc_full[s], kKcBytes);
+#pragma unroll
+        for (int x = 0; x < 4; ++x)  // hi d[0:64], hi d[64:128], lo d[0:64], lo d[64:128]
+          tma_load_4d(dst + x * kHalfBytes, &tmKc, &sm.kc_full[s], 64 * x, g, i * kKcTile, b);
+        ++issued;
+      }
+      // drain: never leave with copies of this CTA in flight (matters only
+      // when a wait above gave up; otherwise these phases completed long ago)
+      mbar_wait(&sm.q_full, 0, ctx.wait_ns);
+      for (int s = 0; s < kStages && s < issued; ++s) {
+        const int fills = (issued - 1 - s) / kStages + 1;  // fills of stage s
+        mbar_wait(&sm.kc_full[s], (fills - 1) & 1, ctx.wait_ns);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0 && n_t > 0) {
+      constexpr uint32_t idesc = instr_desc_bf16(128, 128, 0, 0);
+      bool ok = wait_or_abort(&sm.q_full, 0, ctx, abort_flag);
+      const uint32_t q_addr = smem_u32(sQ);
+      for (int it = 0; ok && it < n_it; ++it) {
+        const int s = it % kStages, a = it & 1;
+        if (!wait_or_abort(&sm.kc_full[s], (it / kStages) & 1, ctx, abort_flag)) break;
+        if (it >= 2 && !wait_or_abort(&sm.acc_empty[a], ((it >> 1) & 1) ^ 1, ctx, abort_flag))
+          break;
+        tc_fence_after();
+        const uint32_t kc_addr = smem_u32(sKc + s * kKcBytes);
+        const bool pass1 = it < n_t;
+        // q . Kc = q . hi + q . lo: K = 2 x 128, the query tile used twice
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const uint32_t off = ((k >> 2) & 1) * kHalfBytes + (k & 3) * 32;
+          const uint64_t qd = smem_desc(q_addr + off, 16, 1024, 2);
+          const uint64_t kd = smem_desc(kc_addr + (k >> 3) * kTileBytes + off, 16, 1024, 2);
+          umma_bf16(tmem + a * 128, pass1 ? qd : kd, pass1 ? kd : qd, idesc, k > 0 ? 1u : 0u);
+        }
+        umma_commit(&sm.kc_empty[s]);
+        umma_commit(&sm.acc_full[a]);
+      }
+      // drain: all MMAs of this CTA complete before TMEM is released
+      umma_commit(&sm.drain);
+      mbar_wait(&sm.drain, 0, ctx.wait_ns);
+    }
+  } else {
+    // ---------------- epilogue: 4 warps, thread <-> TMEM lane ----------------
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;  // TMEM lane this thread reads
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const int64_t slab = score_row_offset(T);
+    float* srow_base = scores + (static_cast<int64_t>(b) * Hkv + g) * slab;
+
+    // pass-1 row identity
+    const int my_tok = r / G;
+    const int my_t = t0 + my_tok;
+    const int my_v = my_t < T ? min(n_c, visible_windows(my_t)) : 0;
+    float m_run = -INFINITY, l_run = 0.f;
+
+    for (int it = 0; it < n_it; ++it) {
+      const int a = it & 1;
+      // all 128 threads take the same decision, so the named barriers below
+      // are always reached by the whole group
+      const bool ok = !*abort_flag && mbar_wait(&sm.acc_full[a], (it >> 1) & 1, ctx.wait_ns);
+      if (named_bar_or(2, 128, !ok)) {
+        if (!ok) report_status(ctx.status, INFLLMV2_STATUS_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      float x[kRows];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float* xc = x + 32 * c;
+        tmem_ld32(lane_addr + a * 128 + 32 * c, *reinterpret_cast<float(*)[32]>(xc));
+      }
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&sm.acc_empty[a]);
+
+      if (it < n_t) {
+        // ---- pass 1: running max / sum of row r over its visible windows ----
+        const int j0 = it * kKcTile;
+        const int nv = min(kKcTile, my_v - j0);  // valid columns (may be <= 0)
+        float tmax = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < kKcTile; ++c)
+          if (c < nv) tmax = fmaxf(tmax, x[c]);
+        const float m_new = fmaxf(m_run, tmax);
+        if (m_new > -INFINITY) {
+          const float mb = m_new * scale_log2;
+          float acc = 0.f;
+#pragma unroll
+          for (int c = 0; c < kKcTile; ++c)
+            if (c < nv) acc += fast_exp2(fmaf(x[c], scale_log2, -mb));
+          l_run = l_run * fast_exp2((m_run - m_new) * scale_log2) + acc;
+          m_run = m_new;
+        }
+        if (it == n_t - 1) {
+          sm.lse2[r] = my_v > 0 ? m_run * scale_log2 + __log2f(l_run) : INFINITY;
+          named_bar_sync(1, 128);
+        }
+      } else {
+        // ---- pass 2: lane r is compressed key j; columns are (token, head) rows ----
+        const int i = it - n_t;
+        const int j = i * kKcTile + r;
+        float S[TPT];
+#pragma unroll
+        for (int tok = 0; tok < TPT; ++tok) {
+          const int t = t0 + tok;
+          const int v = t < T ? min(n_c, visible_windows(t)) : 0;
+          float acc = 0.f;
+#pragma unroll
+          for (int h = 0; h < G; ++h)
+            acc += fast_exp2(fmaf(x[tok * G + h], scale_log2, -sm.lse2[tok * G + h]));
+          S[tok] = j < v ? acc : -INFINITY;
+        }
+        const int cb = i % 3;
+        if (lane == 31) {
+#pragma unroll
+          for (int tok = 0; tok < TPT; ++tok) {
+            if (quad < 3)
+              sm.carry[cb][quad + 1][tok] = S[tok];
+            else
+              sm.carry[(i + 1) % 3][0][tok] = S[tok];
+          }
+        }
+        named_bar_sync(1, 128);
+        const int blk = i * (kKcTile / 4) + quad * 8 + (lane >> 2);
+#pragma unroll
+        for (int tok = 0; tok < TPT; ++tok) {
+          float m4 = fmaxf(S[tok], __shfl_xor_sync(0xffffffffu, S[tok], 1));
+          m4 = fmaxf(m4, __shfl_xor_sync(0xffffffffu, m4, 2));
+          float prev = __shfl_up_sync(0xffffffffu, S[tok], 1);
+          if (lane == 0) prev = sm.carry[cb][quad][tok];
+          const int t = t0 + tok;
+          if ((lane & 3) == 0 && t < T && blk <= t / kBlock)
+            srow_base[score_row_offset(t) + blk] = fmaxf(m4, prev);
+        }
+      }
+    }
+    // blocks past the last compressed-key tile: at most block 32*n_t, whose
+    // only visible window can be the last one of the final tile.
+    if (!*abort_flag) {
+      for (int tok = r; tok < TPT; tok += 128) {
+        const int t = t0 + tok;
+        if (t >= T) continue;
+        const int cur = t / kBlock;
+        for (int blk = n_t * (kKcTile / 4); blk <= cur; ++blk)
+          srow_base[score_row_offset(t) + blk] =
+              blk == n_t * (kKcTile / 4) ? sm.carry[n_t % 3][0][tok] : -INFINITY;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int G>
+int launch_score_g(const Geometry& g, const CUtensorMap& tq, const CUtensorMap& tk, float* scores,
+                   const DevCtx& ctx, cudaStream_t st) {
+  constexpr int TPT = kRows / G;
+  const size_t smem = 1024 + kTileBytes + kKcBytes * kStages + sizeof(ScoreSmem);
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(score_blocks_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return INFLLMV2_ERR_CUDA;
+    configured = true;
+  }
+  const int n_qt = (g.T + TPT - 1) / TPT;
+  const unsigned grid = static_cast<unsigned>(n_qt) * g.B * g.Hkv;
+  score_blocks_kernel<G><<<grid, kThreads, smem, st>>>(tq, tk, scores, g.B, g.T, g.Hkv, g.n_c,
+                                                       g.scale_log2, ctx);
+  return cudaGetLastError() == cudaSuccess ? INFLLMV2_OK : INFLLMV2_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_score_blocks(const Geometry& g, const void* Q, const void* Kc, float* scores,
+                        const DevCtx& ctx, cudaStream_t st) {
+  if (g.B == 0 || g.T == 0) return INFLLMV2_OK;
+  const int TPT = kRows / g.G;
+  CUtensorMap tq, tk;
+  {
+    const uint64_t dims[4] = {static_cast<uint64_t>(kHeadDim), static_cast<uint64_t>(g.Hq),
+                              static_cast<uint64_t>(g.T), static_cast<uint64_t>(g.B)};
+    const uint64_t strides[3] = {static_cast<uint64_t>(kHeadDim) * 2,
+                                 static_cast<uint64_t>(g.Hq) * kHeadDim * 2,
+                                 static_cast<uint64_t>(g.T) * g.Hq * kHeadDim * 2};
+    const uint32_t box[4] = {64u, static_cast<uint32_t>(g.G), static_cast<uint32_t>(TPT), 1u};
+    if (int e = make_tmap_bf16_4d(&tq, Q, dims, strides, box)) return e;
+  }
+  {
+    // n_c may be 0: give the map one row so that it stays encodable; no
+    // tile is loaded in that case.
+    const uint64_t rows = g.n_c > 0 ? static_cast<uint64_t>(g.n_c) : 1u;
+    const uint64_t dims[4] = {static_cast<uint64_t>(kKcRow), static_cast<uint64_t>(g.Hkv), rows,
+                              static_cast<uint64_t>(g.B)};
+    const uint64_t strides[3] = {static_cast<uint64_t>(kKcRow) * 2,
+                                 static_cast<uint64_t>(g.Hkv) * kKcRow * 2,
+                                 rows * g.Hkv * kKcRow * 2};
+    const uint32_t box[4] = {64u, 1u, static_cast<uint32_t>(kKcTile), 1u};
+    if (int e = make_tmap_bf16_4d(&tk, g.n_c > 0 ? Kc : Q, dims, strides, box)) return e;
+  }
+  switch (g.G) {
+    case 1: return launch_score_g<1>(g, tq, tk, scores, ctx, st);
+    case 2: return launch_score_g<2>(g, tq, tk, scores, ctx, st);
+    case 4: return launch_score_g<4>(g, tq, tk, scores, ctx, st);
+    case 8: return launch_score_g<8>(g, tq, tk, scores, ctx, st);
+    case 16: return launch_score_g<16>(g, tq, tk, scores, ctx, st);
+    default: return INFLLMV2_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace infllmv2

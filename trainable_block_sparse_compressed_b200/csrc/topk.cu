@@ -1,0 +1,45 @@
+// topk.cu -- prefill block selection: one warp per (batch, kv head, token)
+// row of the causally packed block-score workspace (see topk.cuh for the
+// selection rule).
+#include "common.cuh"
+#include "topk.cuh"
+
+namespace infllmv2 {
+namespace {
+
+template <int VPL>
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ scores,
+                                                    int32_t* __restrict__ idx, int B, int Hkv,
+                                                    int T, int topk, int n_init, int n_local) {
+  const int64_t row = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t n_rows = static_cast<int64_t>(B) * Hkv * T;
+  if (row >= n_rows) return;
+  const int t = static_cast<int>(row % T);
+  const int64_t bg = row / T;
+  const float* srow = scores + bg * score_row_offset(T) + score_row_offset(t);
+  warp_select_row<VPL>(srow, t / kBlock, topk, n_init, n_local, idx + row * topk);
+}
+
+}  // namespace
+
+int launch_topk(const Geometry& g, const float* scores, int32_t* idx, cudaStream_t st) {
+  if (g.B == 0 || g.T == 0) return INFLLMV2_OK;
+  const int nb_max = (g.T - 1) / kBlock + 1;
+  const int64_t rows = static_cast<int64_t>(g.B) * g.Hkv * g.T;
+  const unsigned blocks = static_cast<unsigned>((rows + 7) / 8);
+  const int vpl = topk_vpl(nb_max);
+#define INFLLMV2_TOPK(V)                                                             \
+  topk_kernel<V><<<blocks, 256, 0, st>>>(scores, idx, g.B, g.Hkv, g.T, g.topk, g.n_init, \
+                                         g.n_local)
+  switch (vpl) {
+    case 4: INFLLMV2_TOPK(4); break;
+    case 16: INFLLMV2_TOPK(16); break;
+    case 64: INFLLMV2_TOPK(64); break;
+    case 128: INFLLMV2_TOPK(128); break;
+    default: return INFLLMV2_ERR_UNSUPPORTED;
+  }
+#undef INFLLMV2_TOPK
+  return cudaGetLastError() == cudaSuccess ? INFLLMV2_OK : INFLLMV2_ERR_CUDA;
+}
+
+}  // namespace infllmv2

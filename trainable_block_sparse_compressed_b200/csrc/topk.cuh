@@ -1,0 +1,97 @@
+// topk.cuh -- warp-collective block selection for one query row.
+//
+// For query token t (cur = t / 64) the selection keeps the forced blocks --
+// the initial blocks 0 .. n_init-1 and the n_local most recent blocks
+// cur-n_local+1 .. cur (InfLLM-V2 skill write-up, Core Concept: the sliding
+// pattern keeps local context) -- and fills the remaining topk - |forced|
+// slots with the highest-scoring other blocks b <= cur (reportify digest,
+// Technical Mechanism: block selection).  Equal scores go to the lower block
+// index; -inf (no visible compressed window) ranks below every finite score.
+// The output row lists the kept blocks in ascending order, padded with -1.
+//
+// Scores become order-preserving 32-bit keys (non-candidates get key 0), each
+// lane holds VPL keys in registers (block i at lane i % 32, slot i / 32), and
+// the warp finds the exact free-th largest key tau by a most-significant-bit-
+// first search: 32 rounds of "count keys >= candidate".  Blocks with key > tau
+// are kept; among keys == tau the lowest indices fill the remaining slots,
+// ranked with ballots in index order.
+#pragma once
+
+#include "common.cuh"
+
+namespace infllmv2 {
+
+__device__ __forceinline__ uint32_t order_key(float s) {
+  const uint32_t u = __float_as_uint(s);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// srow: the nb = cur + 1 block scores of the row (global or shared memory).
+// orow: topk output entries.  All 32 lanes of the warp must call.
+template <int VPL>
+__device__ __forceinline__ void warp_select_row(const float* srow, int cur, int topk, int n_init,
+                                                int n_local, int32_t* orow) {
+  const int lane = threadIdx.x & 31;
+  const int nb = cur + 1;
+  auto forced = [&](int i) { return i < n_init || i > cur - n_local; };
+  const int a = min(n_init, nb);
+  const int lo = max(0, cur - n_local + 1);
+  const int n_forced = a + (nb - lo) - max(0, a - lo);
+  const int free_slots = topk - n_forced;
+  const int n_cand = nb - n_forced;
+
+  uint32_t key[VPL];
+#pragma unroll
+  for (int s = 0; s < VPL; ++s) {
+    const int i = s * 32 + lane;
+    key[s] = (i < nb && !forced(i)) ? order_key(srow[i]) : 0u;
+  }
+
+  uint32_t tau = 0;
+  int need_eq = 0;
+  const bool take_all = free_slots >= n_cand;
+  if (!take_all) {
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t c = tau | (1u << bit);
+      int cnt = 0;
+#pragma unroll
+      for (int s = 0; s < VPL; ++s) cnt += key[s] >= c ? 1 : 0;
+      cnt = __reduce_add_sync(0xffffffffu, cnt);
+      if (cnt >= free_slots) tau = c;
+    }
+    int gt = 0;
+#pragma unroll
+    for (int s = 0; s < VPL; ++s) gt += key[s] > tau ? 1 : 0;
+    gt = __reduce_add_sync(0xffffffffu, gt);
+    need_eq = free_slots - gt;
+  }
+
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int written = 0, eq_seen = 0;
+#pragma unroll
+  for (int s = 0; s < VPL; ++s) {
+    const int i = s * 32 + lane;
+    const bool valid = i < nb;
+    const bool is_forced = valid && forced(i);
+    bool keep = is_forced || (valid && (take_all || key[s] > tau));
+    const bool eq = valid && !is_forced && !take_all && key[s] == tau;
+    const uint32_t eq_ballot = __ballot_sync(0xffffffffu, eq);
+    if (eq) keep = (eq_seen + __popc(eq_ballot & lt_mask)) < need_eq;
+    eq_seen += __popc(eq_ballot);
+    const uint32_t kb = __ballot_sync(0xffffffffu, keep);
+    if (keep) orow[written + __popc(kb & lt_mask)] = i;
+    written += __popc(kb);
+  }
+  for (int k = written + lane; k < topk; k += 32) orow[k] = -1;
+}
+
+// Values per lane needed for rows of up to nb_max blocks (0 if too many).
+inline int topk_vpl(int nb_max) {
+  if (nb_max <= 32 * 4) return 4;
+  if (nb_max <= 32 * 16) return 16;
+  if (nb_max <= 32 * 64) return 64;
+  if (nb_max <= 32 * 128) return 128;
+  return 0;
+}
+
+}  // namespace infllmv2
