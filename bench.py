@@ -1,0 +1,484 @@
+"""Benchmark of the InfLLM-V2 sparse attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the whole prefill path (length switch -> compressed
+keys -> block scoring + top-k selection -> block-sparse attention) over the
+T = 131072 sparse-prefill workload (B=1, Hq=32, Hkv=2, d=128, top-64 with
+1 init + 2 local blocks), seeded synthetic bf16 inputs already resident in
+HBM.  The L2 cache is flushed (256 MB write) between timed steps, outside the
+per-step CUDA events.  Extra keys report the T = 32768 prefill and the decode
+workload (B=16 sequences over a 131072-token cache, 256 steps in a CUDA
+graph).  With N > 1 (torchrun) every rank runs an independent replica: the
+path has no exchange step; value = all ranks' tokens / max-over-ranks time.
+
+--impl reference times the fp64 CPU oracle (the only other implementation of
+the method this project has) on a bounded sample of query rows of the same
+workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse-attn prefill tokens/s + TFLOP/s at 32k/128k; decode tok/s, HBM GB/s"
+MAIN = "sparse_prefill_T131072_Hq32_Hkv2"
+SIDE = "sparse_prefill_T32768_Hq32_Hkv2"
+DECODE = "sparse_decode_B16_L131072_Hq32_Hkv2"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas; barrier + max over ranks only)
+# ---------------------------------------------------------------------------
+class Dist:
+    def __init__(self, n_gpus: int):
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch
+            import torch.distributed as dist
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        import torch
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 9]
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4)
+                          if r[5 + i].strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def kernel_source_hash(name: str) -> str:
+    path = os.path.join(ROOT, "trainable_block_sparse_compressed_b200", "csrc", name)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(kernel_file: str, workload: str):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken
+    on the current source of the kernel; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel_file, {}).get(workload)
+    if not e or e.get("source_sha") != kernel_source_hash(kernel_file):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def attended_keys(idx_np, T):
+    """Keys each (b, g, t) row attends: selected blocks clipped to [0, t]."""
+    import numpy as np
+    t = np.arange(T)[None, None, :, None]
+    valid = (idx_np >= 0) & (idx_np <= (t // 64))
+    start = idx_np.astype(np.int64) * 64
+    n = np.minimum(start + 63, t) - start + 1
+    return np.where(valid, n, 0).sum(axis=-1)  # [B, Hkv, T]
+
+
+# ---------------------------------------------------------------------------
+# our implementation
+# ---------------------------------------------------------------------------
+def run_prefill(api, wl, w, steps, warmup, dist, flush, time_e2e=True, clocks=None):
+    import numpy as np
+    import torch
+    data = wl.make_prefill(w)
+    Qh, Kh, Vh = (wl.to_torch_bf16(data[x]) for x in "QKV")
+    Q, K, V = Qh.cuda(), Kh.cuda(), Vh.cuda()
+    B, T, Hq, Hkv = w.B, w.T, w.Hq, w.Hkv
+    G = Hq // Hkv
+    p = api.make_params(B, T, Hq, Hkv, topk=w.topk, n_init=w.n_init, n_local=w.n_local,
+                        switch_threshold=w.threshold)
+    assert T > w.threshold
+    n_c = api.num_compressed(T)
+    Kc = torch.empty((B, n_c, Hkv, 2, 128), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((B, Hkv, T, w.topk), dtype=torch.int32, device="cuda")
+    ws = api.alloc_workspace(p, api.OP_FORWARD)
+    O = torch.empty_like(Q)
+    lse = torch.empty((B, Hq, T), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(evs=None):
+        # the length switch (T > threshold -> sparse), then the three stages
+        if evs: evs[0].record(stream)
+        api.compress_keys(p, K, Kc)
+        if evs: evs[1].record(stream)
+        api.select_blocks(p, Q, Kc, idx, ws)
+        if evs: evs[2].record(stream)
+        api.sparse_attn(p, Q, K, V, idx, O, lse)
+        if evs: evs[3].record(stream)
+
+    for _ in range(warmup):
+        flush()
+        step()
+    torch.cuda.synchronize()
+    assert api.get_status() == 0
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    dist.barrier()
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+    for s in range(steps):
+        flush()
+        step(evs[s])
+    torch.cuda.synchronize()
+    dist.barrier()
+    clk = clocks.stop() if clocks else None
+    per = [[e[i].elapsed_time(e[i + 1]) for i in range(3)] for e in evs]
+    step_ms = [sum(x) for x in per]
+    ms = sum(step_ms) / steps
+    kern = {name: sum(x[i] for x in per) / steps
+            for i, name in enumerate(["compress_keys", "select_blocks", "sparse_attn"])}
+    assert api.get_status() == 0
+    # useful work of this selection
+    nkeys = attended_keys(idx.cpu().numpy(), T)  # noqa: E501
+    useful_attn_flops = float(4 * 128 * G * nkeys.sum())
+    v = np.array([0 if t < 31 else (t - 31) // 16 + 1 for t in range(T)], dtype=np.int64)
+    useful_score_flops = float(2 * 128 * Hq * B * v.sum())
+    executed_score_flops = 0.0
+    tpt = 128 // G
+    for t0 in range(0, T, tpt):
+        tl = min(t0 + tpt - 1, T - 1)
+        vt = 0 if tl < 31 else min(n_c, (tl - 31) // 16 + 1)
+        nt = (vt + 127) // 128
+        executed_score_flops += 2 * 2 * (2 * 128 * 128 * 256) * nt  # 2 passes, hi+lo
+    executed_score_flops *= B * Hkv
+    idx_np = idx.cpu().numpy()
+    cur = (np.arange(T) // 64)[None, None, :, None]
+    n_valid = ((idx_np >= 0) & (idx_np <= cur)).sum(axis=-1)
+    pairs = int(((n_valid + 1) // 2).sum())
+    # per gathered pair: S^T (128 keys x 16 heads x 128) and P V, 2 FLOP per MAC
+    executed_attn_flops = float(pairs) * 2 * (2 * 128 * 16 * 128)
+    out = dict(ms=ms, step_ms=step_ms, kernels=kern, tokens=B * T,
+               useful_attn_flops=useful_attn_flops, useful_score_flops=useful_score_flops,
+               executed_score_flops=executed_score_flops, executed_attn_flops=executed_attn_flops,
+               clocks=clk, launches_per_step=4)
+    if time_e2e:
+        # end to end through the C ABI from pinned host buffers
+        Qp, Kp, Vp = Qh.pin_memory(), Kh.pin_memory(), Vh.pin_memory()
+        Op = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+        Lp = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+        def e2e_step():
+            Q.copy_(Qp, non_blocking=True)
+            K.copy_(Kp, non_blocking=True)
+            V.copy_(Vp, non_blocking=True)
+            api.forward(p, Q, K, V, O, lse, Kc, idx, ws)
+            Op.copy_(O, non_blocking=True)
+            Lp.copy_(lse, non_blocking=True)
+        e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dist.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out["e2e_ms"] = e0.elapsed_time(e1) / steps
+        out["h2d"] = sum(x.numel() * x.element_size() for x in (Qp, Kp, Vp))
+        out["d2h"] = Op.numel() * Op.element_size() + Lp.numel() * Lp.element_size()
+    del Q, K, V, Kc, idx, ws, O, lse
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_decode(api, wl, w, steps, warmup, flush):
+    """256 decode steps over B=16 caches of 131072 tokens, captured in a CUDA graph."""
+    import torch
+    B, L0, Hq, Hkv = w.B, w.T, w.Hq, w.Hkv
+    total = warmup + steps
+    data = wl.make_decode(w, L=L0, steps=total, B=B)
+    Lmax = L0 + total
+    p = api.make_params(B, Lmax, Hq, Hkv, topk=w.topk, n_init=w.n_init, n_local=w.n_local)
+    Kc = torch.zeros((B, Lmax, Hkv, 128), dtype=torch.bfloat16, device="cuda")
+    Vc = torch.zeros_like(Kc)
+    Kc[:, :L0] = wl.to_torch_bf16(data["K0"]).cuda()
+    Vc[:, :L0] = wl.to_torch_bf16(data["V0"]).cuda()
+    NC = api.num_compressed(Lmax)
+    Kcmp = torch.zeros((B, NC, Hkv, 2, 128), dtype=torch.bfloat16, device="cuda")
+    n0 = api.num_compressed(L0)
+    tmp = torch.empty((B, n0, Hkv, 2, 128), dtype=torch.bfloat16, device="cuda")
+    api.compress_keys(api.make_params(B, L0, Hq, Hkv), Kc[:, :L0].contiguous(), tmp)
+    Kcmp[:, :n0] = tmp
+    del tmp
+    seqlens = torch.full((B,), L0, dtype=torch.int32, device="cuda")
+    q = wl.to_torch_bf16(data["q"]).cuda()
+    kn = wl.to_torch_bf16(data["k_new"]).cuda()
+    vn = wl.to_torch_bf16(data["v_new"]).cuda()
+    O = torch.empty((B, Hq, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
+    ws = api.alloc_workspace(p, api.OP_DECODE)
+    for s in range(warmup):
+        api.decode_step(p, q[s], kn[s], vn[s], Kc, Vc, Kcmp, seqlens, O, lse, None, ws)
+    torch.cuda.synchronize()
+    # capture the timed steps in one graph (inputs of each step are distinct slices)
+    g = torch.cuda.CUDAGraph()
+    st = torch.cuda.Stream()
+    seq_start = seqlens.clone()
+    with torch.cuda.stream(st):
+        with torch.cuda.graph(g, stream=st):
+            for s in range(warmup, total):
+                api.decode_step(p, q[s], kn[s], vn[s], Kc, Vc, Kcmp, seqlens, O, lse, None, ws)
+    torch.cuda.synchronize()
+    seqlens.copy_(seq_start)
+    flush()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    assert api.get_status() == 0
+    assert int(seqlens[0]) == L0 + total
+    per_step = ms / steps
+    # algorithmic HBM bytes per step: every visible compressed key (hi+lo) of
+    # every sequence and kv head, the K and V rows of the selected blocks, the
+    # appended K/V rows, q and the outputs
+    nc_vis = (L0 + warmup + steps // 2 - 31) // 16 + 1
+    kc_bytes = B * Hkv * nc_vis * 2 * 128 * 2
+    kv_bytes = B * Hkv * w.topk * 64 * 128 * 2 * 2
+    small = B * (Hq * 128 * 2 * 2 + Hkv * 128 * 2 * 2 + Hq * 4)
+    bytes_step = kc_bytes + kv_bytes + small
+    del g
+    return dict(ms_per_step=per_step, tokens_per_s=B / (per_step / 1e3),
+                hbm_gbs=bytes_step / (per_step / 1e3) / 1e9, bytes_per_step=bytes_step,
+                steps=steps, launches_per_step=6)
+
+
+def cpu_oracle_sample(w, seconds=15.0):
+    """Times the fp64 oracle on query rows of the workload until `seconds`
+    pass; returns tokens/s (a token = its Hkv query groups) and the sample."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+    from oracle import infllmv2_oracle as orc
+    from trainable_block_sparse_compressed_b200 import workloads as wl
+    data = wl.make_prefill(w)
+    Q, K, V = (wl.bf16_to_f64(data[x]) for x in "QKV")
+    p = orc.Params(topk=w.topk, n_init=w.n_init, n_local=w.n_local, threshold=w.threshold)
+    rng = np.random.default_rng(0)
+    with threadpool_limits(limits=1):
+        t0 = time.perf_counter()
+        Kc = orc.compress_keys(K, p)
+        t_cmp = time.perf_counter() - t0
+        G = w.Hq // w.Hkv
+        rows = 0
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < seconds:
+            t = int(rng.integers(0, w.T))
+            for g in range(w.Hkv):
+                r = orc.select_row(Q, Kc, 0, g, t, p)
+                keys = orc.selected_keys(r.idx, t, p)
+                orc.attend(Q[0, t, g * G:(g + 1) * G], K[0, :, g], V[0, :, g], keys, p.sm_scale(128))
+            rows += 1
+        el = time.perf_counter() - t0
+    per_token = el / rows
+    total_s = t_cmp + per_token * w.T * w.B
+    return dict(value=w.T * w.B / total_s, unit="tokens/s", cores=1, kind="oracle",
+                sample=f"{rows} random query tokens x {w.Hkv} kv groups of {w.name} "
+                       f"(selection + attention, fp64 numpy, 1 thread) in {el:.1f} s, "
+                       f"plus full compressed keys ({t_cmp:.1f} s); extrapolated to all "
+                       f"{w.T} tokens")
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extras", action="store_true", help="skip the 32k and decode extras")
+    ap.add_argument("--baseline-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    from trainable_block_sparse_compressed_b200 import workloads as wl
+    w = wl.WORKLOADS[MAIN]
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return
+        t0 = time.perf_counter()
+        vals = []
+        for _ in range(args.warmup + args.steps):
+            vals.append(cpu_oracle_sample(w, seconds=max(2.0, args.baseline_seconds / 4)))
+        res = vals[-1]
+        value = statistics.mean(v["value"] for v in vals[args.warmup:])
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 0,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1e3 * w.T / value, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "impl": "reference",
+                "config": {"workload": MAIN, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv,
+                           "d": 128, "topk": w.topk, "n_init": w.n_init, "n_local": w.n_local},
+                "cpu_baseline": dict(res, value=value),
+                "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0},
+                "wall_s": time.perf_counter() - t0}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    from trainable_block_sparse_compressed_b200 import infllmv2 as api
+    dist = Dist(args.gpus)
+    torch.cuda.set_device(dist.local)
+    api.load()
+    peaks, peak_src = load_peaks()
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def flush():
+        flush_buf.zero_()
+
+    clocks = ClockSampler(dist.local)
+    main_r = run_prefill(api, wl, w, args.steps, args.warmup, dist, flush, True, clocks)
+    ms = dist.max(main_r["ms"])
+    e2e_ms = dist.max(main_r["e2e_ms"])
+    tokens_all = main_r["tokens"] * dist.world
+    value = tokens_all / (ms / 1e3)
+
+    extras = {}
+    if not args.no_extras:
+        side = run_prefill(api, wl, wl.WORKLOADS[SIDE], args.steps, args.warmup, dist, flush,
+                           False, None)
+        sms = dist.max(side["ms"])
+        extras["prefill_T32768"] = {
+            "tokens_per_s": side["tokens"] * dist.world / (sms / 1e3), "ms_per_step": sms,
+            "useful_tflops": (side["useful_attn_flops"] + side["useful_score_flops"]) / (sms / 1e3) / 1e12,
+            "kernels_ms": side["kernels"]}
+        wd = wl.WORKLOADS[DECODE]
+        dec = run_decode(api, wl, wd, 256, 8, flush)
+        dms = dist.max(dec["ms_per_step"])
+        extras["decode_B16_L131072"] = {
+            "tokens_per_s": wd.B * dist.world / (dms / 1e3), "ms_per_step": dms,
+            "hbm_gbs": dec["bytes_per_step"] / (dms / 1e3) / 1e9,
+            "hbm_frac_of_measured": dec["bytes_per_step"] / (dms / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "algorithmic_bytes_per_step": dec["bytes_per_step"], "steps": 256,
+            "timing": "256 steps in one CUDA graph, L2 flushed before the replay"}
+
+    # roofline of the dominant kernel (the block-sparse attention)
+    kern = main_r["kernels"]
+    dom = max(kern, key=kern.get)
+    sustained = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    if dom == "sparse_attn":
+        achieved = main_r["useful_attn_flops"] / (kern[dom] / 1e3) / 1e12
+        kfile = "sparse_attn.cu"
+    else:
+        achieved = main_r["useful_score_flops"] / (kern[dom] / 1e3) / 1e12
+        kfile = "score.cu"
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": sustained,
+                "unit": "TFLOP/s", "frac": achieved / sustained,
+                "peak_source": f"{peak_src} bf16 sustained",
+                "traffic": profiled_traffic(kfile, MAIN)}
+    useful = main_r["useful_attn_flops"] + main_r["useful_score_flops"]
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": MAIN, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "d": 128,
+                   "topk": w.topk, "n_init": w.n_init, "n_local": w.n_local,
+                   "switch_threshold": w.threshold, "needles": w.needles,
+                   "parallelism": f"replicas x{dist.world}",
+                   "l2": "flushed between timed steps (256 MB write, outside the events)"},
+        "useful_tflops": useful * dist.world / (ms / 1e3) / 1e12,
+        "executed_tflops": (main_r["executed_attn_flops"] + main_r["executed_score_flops"])
+        * dist.world / (ms / 1e3) / 1e12,
+        "kernels_ms": kern,
+        "roofline": roofline,
+        "e2e": {"value": tokens_all / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": main_r["h2d"], "d2h_bytes_per_step": main_r["d2h"]},
+        "gpu_launches": main_r["launches_per_step"] * args.steps,
+        "clocks": main_r["clocks"],
+    }
+    line.update(extras)
+    if dist.rank == 0:
+        line["cpu_baseline"] = cpu_oracle_sample(w, args.baseline_seconds)
+        print(json.dumps(line), flush=True)
+    dist.close()
+
+
+if __name__ == "__main__":
+    main()
