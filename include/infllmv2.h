@@ -184,6 +184,39 @@ int infllmv2_decode_step(const infllmv2_params* p, const void* q, const void* k_
                          int32_t* seqlens, void* O, float* lse, int32_t* idx_out,
                          void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * infllmv2_decode_step without a workspace argument: nothing is allocated,
+ * by the caller or by the library.  The paper has no counterpart; this entry
+ * point exists for callers that cannot allocate device memory.  A host
+ * runtime that embeds the library often hands it only the step's inputs and
+ * outputs: its own allocator already owns the rest of the GPU's memory (a
+ * pool reserved up front), its plugin interface has no way to pass scratch
+ * space, and a cudaMalloc of its own from inside the decode loop would fail
+ * or fragment that pool.
+ *
+ * Arguments and results are those of infllmv2_decode_step.  The scratch is
+ * one file-scope static __device__ array of INFLLMV2_NOALLOC_SCRATCH_BYTES
+ * bytes inside the library, so every GPU that loads the library holds that
+ * memory until the process exits.
+ * - If infllmv2_workspace_bytes(p, INFLLMV2_OP_DECODE) exceeds the array, the
+ *   call returns INFLLMV2_ERR_WORKSPACE and enqueues nothing.  (The B=16,
+ *   131072-token, Hq=32, Hkv=2 decode needs about 19 MiB.)
+ * - The first call on a device looks up the array's device address with
+ *   that device current (cudaGetSymbolAddress); make this first call before
+ *   any stream capture on that device.
+ * - All calls share the one array, which keeps the last call's contents.
+ *   Calls whose kernels can overlap on the GPU (different streams with no
+ *   ordering between them) race on it and corrupt each other's results;
+ *   calls issued on one stream are ordered and safe.  Nothing in the array
+ *   needs clearing between calls: every kernel of a step writes the scratch
+ *   it reads later in the same step.
+ */
+#define INFLLMV2_NOALLOC_SCRATCH_BYTES (32u << 20)
+int infllmv2_decode_step_noalloc(const infllmv2_params* p, const void* q, const void* k_new,
+                                 const void* v_new, void* K_cache, void* V_cache,
+                                 void* Kc_cache, int32_t* seqlens, void* O, float* lse,
+                                 int32_t* idx_out, void* stream);
+
 /* Device workspace bytes needed by an operation (0 if none; SIZE_MAX on bad params). */
 size_t infllmv2_workspace_bytes(const infllmv2_params* p, int32_t op);
 

@@ -247,6 +247,60 @@ int infllmv2_decode_step(const infllmv2_params* p, const void* q, const void* k_
                             idx_out, ws, ctx, static_cast<cudaStream_t>(stream));
 }
 
+}  // extern "C"
+
+namespace infllmv2 {
+namespace {
+
+// Scratch of infllmv2_decode_step_noalloc: a fixed array in every device's
+// copy of this module, so neither the caller nor the library allocates.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[INFLLMV2_NOALLOC_SCRATCH_BYTES];
+
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the array on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address must be looked
+// up, once per device, with that device current.
+int noalloc_scratch(void** out) {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return INFLLMV2_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_noalloc_ptr[d]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr)
+      return INFLLMV2_ERR_CUDA;
+    g_noalloc_ptr[d] = ptr;
+  }
+  *out = g_noalloc_ptr[d];
+  return INFLLMV2_OK;
+}
+
+}  // namespace
+}  // namespace infllmv2
+
+extern "C" {
+
+int infllmv2_decode_step_noalloc(const infllmv2_params* p, const void* q, const void* k_new,
+                                 const void* v_new, void* K_cache, void* V_cache,
+                                 void* Kc_cache, int32_t* seqlens, void* O, float* lse,
+                                 int32_t* idx_out, void* stream) {
+  Geometry g;
+  if (int e = validate(p, true, &g)) return e;
+  if (g.B == 0) return INFLLMV2_OK;
+  if (g.T < 1) return INFLLMV2_ERR_INVALID_ARG;
+  if (int e = check_ptrs({q, k_new, v_new, K_cache, V_cache, seqlens, O, lse})) return e;
+  if (g.n_c > 0)
+    if (int e = check_ptrs({Kc_cache})) return e;
+  if (idx_out && !aligned16(idx_out)) return INFLLMV2_ERR_UNSUPPORTED;
+  if (decode_ws_bytes(g) > INFLLMV2_NOALLOC_SCRATCH_BYTES) return INFLLMV2_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (int e = noalloc_scratch(&scratch)) return e;
+  DevCtx ctx;
+  if (int e = ctx_or_error(&ctx)) return e;
+  return launch_decode_step(g, q, k_new, v_new, K_cache, V_cache, Kc_cache, seqlens, O, lse,
+                            idx_out, scratch, ctx, static_cast<cudaStream_t>(stream));
+}
+
 int infllmv2_selftest_timeout(void* stream) {
   DevCtx ctx;
   if (int e = ctx_or_error(&ctx)) return e;

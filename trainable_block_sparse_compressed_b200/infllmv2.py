@@ -35,8 +35,9 @@ EXPORTS = (
     "infllmv2_dense_attn", "infllmv2_forward", "infllmv2_decode_step",
     "infllmv2_workspace_bytes", "infllmv2_num_compressed", "infllmv2_get_status",
     "infllmv2_set_wait_limit", "infllmv2_selftest_timeout", "infllmv2_strerror",
-    "infllmv2_version",
+    "infllmv2_version", "infllmv2_decode_step_noalloc",
 )
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class InfLLMV2Error(RuntimeError):
@@ -84,6 +85,8 @@ def load(path: Optional[str] = None):
         "infllmv2_forward": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "infllmv2_decode_step": (ctypes.c_int,
                                  [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "infllmv2_decode_step_noalloc": (ctypes.c_int,
+                                         [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "infllmv2_workspace_bytes": (sz, [P, i32]),
         "infllmv2_num_compressed": (i32, [i32]),
         "infllmv2_get_status": (ctypes.c_int, [vp, ctypes.POINTER(i32)]),
@@ -190,6 +193,17 @@ def decode_step(p: Params, q, k_new, v_new, K_cache, V_cache, Kc_cache, seqlens,
                                        _ptr(K_cache), _ptr(V_cache), _ptr(Kc_cache),
                                        _ptr(seqlens), _ptr(O), _ptr(lse), _ptr(idx_out), _ptr(ws),
                                        nbytes, _stream(stream)))
+
+
+def decode_step_noalloc(p: Params, q, k_new, v_new, K_cache, V_cache, Kc_cache, seqlens, O,
+                        lse, idx_out=None, stream=None):
+    """decode_step with the library's fixed scratch array instead of a
+    workspace (for callers that cannot allocate device memory)."""
+    _check("infllmv2_decode_step_noalloc",
+           load().infllmv2_decode_step_noalloc(ctypes.byref(p), _ptr(q), _ptr(k_new), _ptr(v_new),
+                                               _ptr(K_cache), _ptr(V_cache), _ptr(Kc_cache),
+                                               _ptr(seqlens), _ptr(O), _ptr(lse), _ptr(idx_out),
+                                               _stream(stream)))
 
 
 # --------------------------------------------------------------------------
