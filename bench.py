@@ -44,18 +44,25 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # distributed plumbing (replicas; barrier + max over ranks only)
 # ---------------------------------------------------------------------------
 class Dist:
-    def __init__(self, n_gpus: int):
+    """One process per GPU under torchrun.  The step has no exchange, so the
+    only collectives are the barrier around the timed region and the max of
+    the per-rank times (gloo when CUDA is absent, or when asked for)."""
+
+    def __init__(self, n_gpus: int, backend: str | None = None):
         self.rank = int(os.environ.get("RANK", "0"))
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = None
+        self.device = "cpu"
         if self.world > 1:
             import datetime
             import torch
             import torch.distributed as dist
-            backend = "nccl" if torch.cuda.is_available() else "gloo"
+            if backend is None:
+                backend = "nccl" if torch.cuda.is_available() else "gloo"
             if backend == "nccl":
                 torch.cuda.set_device(self.local)
+                self.device = "cuda"
             dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
             self.pg = dist
 
@@ -67,14 +74,18 @@ class Dist:
         if not self.pg:
             return x
         import torch
-        dev = "cuda" if torch.cuda.is_available() else "cpu"
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
     def close(self):
         if self.pg:
             self.pg.destroy_process_group()
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Units all ranks processed per second, timed by the slowest rank."""
+    return units_per_rank * world / (ms_max / 1e3)
 
 
 # ---------------------------------------------------------------------------
@@ -175,6 +186,7 @@ def run_prefill(api, wl, w, steps, warmup, dist, flush, time_e2e=True, clocks=No
     idx = torch.empty((B, Hkv, T, w.topk), dtype=torch.int32, device="cuda")
     ws = api.alloc_workspace(p, api.OP_FORWARD)
     O = torch.empty_like(Q)
+    aws = api.alloc_workspace(p, api.OP_ATTN)
     lse = torch.empty((B, Hq, T), dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
 
@@ -185,7 +197,7 @@ def run_prefill(api, wl, w, steps, warmup, dist, flush, time_e2e=True, clocks=No
         if evs: evs[1].record(stream)
         api.select_blocks(p, Q, Kc, idx, ws)
         if evs: evs[2].record(stream)
-        api.sparse_attn(p, Q, K, V, idx, O, lse)
+        api.sparse_attn(p, Q, K, V, idx, O, lse, aws)
         if evs: evs[3].record(stream)
 
     for _ in range(warmup):
@@ -232,7 +244,7 @@ def run_prefill(api, wl, w, steps, warmup, dist, flush, time_e2e=True, clocks=No
     out = dict(ms=ms, step_ms=step_ms, kernels=kern, tokens=B * T,
                useful_attn_flops=useful_attn_flops, useful_score_flops=useful_score_flops,
                executed_score_flops=executed_score_flops, executed_attn_flops=executed_attn_flops,
-               clocks=clk, launches_per_step=4)
+               clocks=clk, launches_per_step=5)
     if time_e2e:
         # end to end through the C ABI from pinned host buffers
         Qp, Kp, Vp = Qh.pin_memory(), Kh.pin_memory(), Vh.pin_memory()
@@ -416,8 +428,7 @@ def main():
     main_r = run_prefill(api, wl, w, args.steps, args.warmup, dist, flush, True, clocks)
     ms = dist.max(main_r["ms"])
     e2e_ms = dist.max(main_r["e2e_ms"])
-    tokens_all = main_r["tokens"] * dist.world
-    value = tokens_all / (ms / 1e3)
+    value = whole_job_rate(main_r["tokens"], dist.world, ms)
 
     extras = {}
     if not args.no_extras:
@@ -425,14 +436,14 @@ def main():
                            False, None)
         sms = dist.max(side["ms"])
         extras["prefill_T32768"] = {
-            "tokens_per_s": side["tokens"] * dist.world / (sms / 1e3), "ms_per_step": sms,
+            "tokens_per_s": whole_job_rate(side["tokens"], dist.world, sms), "ms_per_step": sms,
             "useful_tflops": (side["useful_attn_flops"] + side["useful_score_flops"]) / (sms / 1e3) / 1e12,
             "kernels_ms": side["kernels"]}
         wd = wl.WORKLOADS[DECODE]
         dec = run_decode(api, wl, wd, 256, 8, flush)
         dms = dist.max(dec["ms_per_step"])
         extras["decode_B16_L131072"] = {
-            "tokens_per_s": wd.B * dist.world / (dms / 1e3), "ms_per_step": dms,
+            "tokens_per_s": whole_job_rate(wd.B, dist.world, dms), "ms_per_step": dms,
             "hbm_gbs": dec["bytes_per_step"] / (dms / 1e3) / 1e9,
             "hbm_frac_of_measured": dec["bytes_per_step"] / (dms / 1e3) / 1e9 / peaks["hbm_gbs"],
             "algorithmic_bytes_per_step": dec["bytes_per_step"], "steps": 256,
@@ -463,12 +474,12 @@ def main():
                    "switch_threshold": w.threshold, "needles": w.needles,
                    "parallelism": f"replicas x{dist.world}",
                    "l2": "flushed between timed steps (256 MB write, outside the events)"},
-        "useful_tflops": useful * dist.world / (ms / 1e3) / 1e12,
-        "executed_tflops": (main_r["executed_attn_flops"] + main_r["executed_score_flops"])
-        * dist.world / (ms / 1e3) / 1e12,
+        "useful_tflops": whole_job_rate(useful, dist.world, ms) / 1e12,
+        "executed_tflops": whole_job_rate(
+            main_r["executed_attn_flops"] + main_r["executed_score_flops"], dist.world, ms) / 1e12,
         "kernels_ms": kern,
         "roofline": roofline,
-        "e2e": {"value": tokens_all / (e2e_ms / 1e3), "unit": "tokens/s",
+        "e2e": {"value": whole_job_rate(main_r["tokens"], dist.world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": main_r["h2d"], "d2h_bytes_per_step": main_r["d2h"]},
         "gpu_launches": main_r["launches_per_step"] * args.steps,
         "clocks": main_r["clocks"],

@@ -86,6 +86,7 @@ typedef struct infllmv2_params {
 #define INFLLMV2_OP_SELECT   1
 #define INFLLMV2_OP_FORWARD  2
 #define INFLLMV2_OP_DECODE   3
+#define INFLLMV2_OP_ATTN     4  /* sparse_attn / dense_attn: packed K and V */
 
 /* Path reported by infllmv2_forward. */
 #define INFLLMV2_PATH_DENSE  1
@@ -134,18 +135,25 @@ int infllmv2_select_blocks(const infllmv2_params* p, const void* Q, const void* 
  *   lse[b,h,t] = log sum_{i in keys(t)} exp(scale * q.K_i).
  *   idx rows must be ascending with valid entries first (as select_blocks
  *   writes them); entries > t/64 are ignored.
+ *   ws: optional device workspace of infllmv2_workspace_bytes(p,
+ *   INFLLMV2_OP_ATTN) bytes.  With it, K and V are first repacked into
+ *   block-contiguous tiles (one 16 KB chunk per 64-key block and kv head) so
+ *   that every selected block is gathered by one bulk copy; with ws == NULL
+ *   (or ws_bytes too small for it) blocks are gathered from K and V directly
+ *   by tensor-map copies, which is slower.  Results are identical.
  */
 int infllmv2_sparse_attn(const infllmv2_params* p, const void* Q, const void* K,
-                         const void* V, const int32_t* idx, void* O, float* lse,
-                         void* stream);
+                         const void* V, const int32_t* idx, void* O, float* lse, void* ws,
+                         size_t ws_bytes, void* stream);
 
 /*
  * Exact dense causal attention (skill write-up, Architecture Overview, the
  * dense pathway bullet): keys(t) = [0, t], same O and lse
- * definitions as infllmv2_sparse_attn.
+ * definitions as infllmv2_sparse_attn; ws as for infllmv2_sparse_attn.
  */
 int infllmv2_dense_attn(const infllmv2_params* p, const void* Q, const void* K,
-                        const void* V, void* O, float* lse, void* stream);
+                        const void* V, void* O, float* lse, void* ws, size_t ws_bytes,
+                        void* stream);
 
 /*
  * The switchable attention (skill write-up, Implementation Step 3: dense when

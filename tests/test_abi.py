@@ -54,7 +54,12 @@ def test_workspace_sizes(lib):
     per = sum((t // 64 + 1) for t in range(0, T, 64)) * 64
     assert api.workspace_bytes(p, api.OP_SELECT) == 2 * per * 4
     dense = api.make_params(2, 4096, 32, 2, switch_threshold=8192)
-    assert api.workspace_bytes(dense, api.OP_FORWARD) == 0
+    # dense forward: only the packed K/V tiles (2 tensors x B x Hkv x blocks x 16 KB)
+    assert api.workspace_bytes(dense, api.OP_FORWARD) == 2 * 2 * 2 * 64 * 16384
+    assert api.workspace_bytes(dense, api.OP_ATTN) == 2 * 2 * 2 * 64 * 16384
+    # sparse forward: block scores (256-byte aligned) then the tiles
+    assert api.workspace_bytes(p, api.OP_FORWARD) == \
+        (-(-api.workspace_bytes(p, api.OP_SELECT) // 256) * 256) + api.workspace_bytes(p, api.OP_ATTN)
     assert api.workspace_bytes(api.make_params(16, 131328, 32, 2), api.OP_DECODE) > 0
     bad = api.make_params(1, 100, 32, 2, head_dim=64)
     with pytest.raises(api.InfLLMV2Error):
@@ -82,7 +87,7 @@ def test_bad_params_rejected_on_host(lib, kw, code):
     p = api.make_params(**base)
     P = ctypes.byref(p)
     assert lib.infllmv2_select_blocks(P, FAKE, FAKE, FAKE, FAKE, 1 << 30, None) == code
-    assert lib.infllmv2_sparse_attn(P, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None) == code
+    assert lib.infllmv2_sparse_attn(P, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0, None) == code
 
 
 def test_null_and_misaligned_pointers(lib):
@@ -90,7 +95,7 @@ def test_null_and_misaligned_pointers(lib):
     P = ctypes.byref(p)
     assert lib.infllmv2_compress_keys(P, None, FAKE, None) == api.ERR_INVALID_ARG
     assert lib.infllmv2_compress_keys(P, FAKE + 2, FAKE, None) == api.ERR_UNSUPPORTED
-    assert lib.infllmv2_dense_attn(P, FAKE, FAKE, FAKE, None, FAKE, None) == api.ERR_INVALID_ARG
+    assert lib.infllmv2_dense_attn(P, FAKE, FAKE, FAKE, None, FAKE, None, 0, None) == api.ERR_INVALID_ARG
     assert lib.infllmv2_select_blocks(P, FAKE, FAKE, FAKE, FAKE, 16, None) == api.ERR_WORKSPACE
     assert lib.infllmv2_get_status(None, None) == api.ERR_INVALID_ARG
 
@@ -99,4 +104,5 @@ def test_empty_problems_are_noops(lib):
     p = api.make_params(0, 256, 32, 2, topk=8)
     assert lib.infllmv2_compress_keys(ctypes.byref(p), None, None, None) == api.OK
     p = api.make_params(1, 0, 32, 2, topk=8)
-    assert lib.infllmv2_sparse_attn(ctypes.byref(p), None, None, None, None, None, None, None) == api.OK
+    assert lib.infllmv2_sparse_attn(ctypes.byref(p), None, None, None, None, None, None, None, 0,
+                                    None) == api.OK

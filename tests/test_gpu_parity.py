@@ -111,8 +111,9 @@ def test_select_blocks_all_rows(cuda_lib, case):
 # ---------------------------------------------------------------------------
 # attention with the oracle's selection
 # ---------------------------------------------------------------------------
+@pytest.mark.parametrize("packed", [True, False], ids=["packed_kv", "tensor_map_gather"])
 @pytest.mark.parametrize("case", SMALL, ids=[f"B{c[0]}_T{c[1]}_Hq{c[2]}_Hkv{c[3]}_k{c[4]}" for c in SMALL])
-def test_sparse_attn_all_rows(cuda_lib, case):
+def test_sparse_attn_all_rows(cuda_lib, case, packed):
     import torch
     api = cuda_lib
     B, T, Hq, Hkv, topk, needles, seed = case
@@ -124,8 +125,10 @@ def test_sparse_attn_all_rows(cuda_lib, case):
     O_ref, L_ref = orc.sparse_attention(Q, K, V, idx, op)
     O = torch.empty((B, T, Hq, 128), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((B, Hq, T), dtype=torch.float32, device="cuda")
-    api.sparse_attn(_params(api, w), gpu_bf16(data["Q"]), gpu_bf16(data["K"]), gpu_bf16(data["V"]),
-                    torch.from_numpy(idx).cuda(), O, lse)
+    p = _params(api, w)
+    ws = api.alloc_workspace(p, api.OP_ATTN) if packed else None
+    api.sparse_attn(p, gpu_bf16(data["Q"]), gpu_bf16(data["K"]), gpu_bf16(data["V"]),
+                    torch.from_numpy(idx).cuda(), O, lse, ws)
     torch.cuda.synchronize()
     assert api.get_status() == 0
     assert np.abs(f64(O) - O_ref).max() <= O_ATOL
@@ -152,8 +155,9 @@ def test_sparse_attn_unsorted_padding_and_ignored_entries(cuda_lib):
     O_ref, L_ref = orc.sparse_attention(Q, K, V, idx, op)
     O = torch.empty((1, 400, 32, 128), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((1, 32, 400), dtype=torch.float32, device="cuda")
-    api.sparse_attn(_params(api, w), gpu_bf16(data["Q"]), gpu_bf16(data["K"]), gpu_bf16(data["V"]),
-                    torch.from_numpy(idx).cuda(), O, lse)
+    p = _params(api, w)
+    api.sparse_attn(p, gpu_bf16(data["Q"]), gpu_bf16(data["K"]), gpu_bf16(data["V"]),
+                    torch.from_numpy(idx).cuda(), O, lse, api.alloc_workspace(p, api.OP_ATTN))
     torch.cuda.synchronize()
     assert np.abs(f64(O) - O_ref).max() <= O_ATOL
     assert np.abs(f64(lse) - L_ref).max() <= LSE_ATOL
@@ -162,8 +166,9 @@ def test_sparse_attn_unsorted_padding_and_ignored_entries(cuda_lib):
 # ---------------------------------------------------------------------------
 # dense path and the switch
 # ---------------------------------------------------------------------------
+@pytest.mark.parametrize("packed", [True, False], ids=["packed_kv", "tensor_map_gather"])
 @pytest.mark.parametrize("B,T,Hq,Hkv", [(1, 300, 32, 2), (2, 130, 8, 2), (1, 1, 16, 1)])
-def test_dense_attn_all_rows(cuda_lib, B, T, Hq, Hkv):
+def test_dense_attn_all_rows(cuda_lib, B, T, Hq, Hkv, packed):
     import torch
     api = cuda_lib
     w = wl.small_workload(B=B, T=T, Hq=Hq, Hkv=Hkv, needles=0, seed=T + Hq)
@@ -172,7 +177,9 @@ def test_dense_attn_all_rows(cuda_lib, B, T, Hq, Hkv):
     O_ref, L_ref = orc.dense_attention(Q, K, V, orc.Params())
     O = torch.empty((B, T, Hq, 128), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((B, Hq, T), dtype=torch.float32, device="cuda")
-    api.dense_attn(_params(api, w), gpu_bf16(data["Q"]), gpu_bf16(data["K"]), gpu_bf16(data["V"]), O, lse)
+    p = _params(api, w)
+    ws = api.alloc_workspace(p, api.OP_ATTN) if packed else None
+    api.dense_attn(p, gpu_bf16(data["Q"]), gpu_bf16(data["K"]), gpu_bf16(data["V"]), O, lse, ws)
     torch.cuda.synchronize()
     assert np.abs(f64(O) - O_ref).max() <= O_ATOL
     assert np.abs(f64(lse) - L_ref).max() <= LSE_ATOL
@@ -239,7 +246,8 @@ def _full_prefill_check(api, name, n_rows, seed):
     O2 = torch.empty_like(Qg)
     lse2 = torch.empty_like(lse)
     p = api.make_params(w.B, w.T, w.Hq, w.Hkv, topk=w.topk, switch_threshold=w.threshold)
-    api.sparse_attn(p, Qg, Kg, Vg, torch.from_numpy(full_idx).cuda(), O2, lse2)
+    api.sparse_attn(p, Qg, Kg, Vg, torch.from_numpy(full_idx).cuda(), O2, lse2,
+                    api.alloc_workspace(p, api.OP_ATTN))
     torch.cuda.synchronize()
     O_ref, L_ref = orc.sparse_attention(Q, K, V, oidx, op, rows)
     Og, Lg = f64(O2), f64(lse2)

@@ -116,6 +116,8 @@ int check_ptrs(std::initializer_list<const void*> ptrs) {
   return INFLLMV2_OK;
 }
 
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
 size_t select_ws_bytes(const Geometry& g) {
   return static_cast<size_t>(g.B) * g.Hkv * static_cast<size_t>(score_row_offset(g.T)) *
          sizeof(float);
@@ -158,8 +160,11 @@ size_t infllmv2_workspace_bytes(const infllmv2_params* p, int32_t op) {
   if (validate(p, op != 0, &g) != INFLLMV2_OK) return SIZE_MAX;
   switch (op) {
     case INFLLMV2_OP_SELECT: return select_ws_bytes(g);
-    case INFLLMV2_OP_FORWARD: return p->T <= p->switch_threshold ? 0 : select_ws_bytes(g);
+    case INFLLMV2_OP_FORWARD:
+      return p->T <= p->switch_threshold ? packed_kv_bytes(g)
+                                         : align256(select_ws_bytes(g)) + packed_kv_bytes(g);
     case INFLLMV2_OP_DECODE: return decode_ws_bytes(g);
+    case INFLLMV2_OP_ATTN: return packed_kv_bytes(g);
     default: return SIZE_MAX;
   }
 }
@@ -190,26 +195,36 @@ int infllmv2_select_blocks(const infllmv2_params* p, const void* Q, const void* 
 }
 
 int infllmv2_sparse_attn(const infllmv2_params* p, const void* Q, const void* K, const void* V,
-                         const int32_t* idx, void* O, float* lse, void* stream) {
+                         const int32_t* idx, void* O, float* lse, void* ws, size_t ws_bytes,
+                         void* stream) {
   Geometry g;
   if (int e = validate(p, true, &g)) return e;
   if (empty(g)) return INFLLMV2_OK;
   if (int e = check_ptrs({Q, K, V, idx, O, lse})) return e;
+  if (ws && !aligned16(ws)) return INFLLMV2_ERR_UNSUPPORTED;
   DevCtx ctx;
   if (int e = ctx_or_error(&ctx)) return e;
-  return launch_sparse_attn(g, Q, K, V, idx, O, lse, 0, ctx, static_cast<cudaStream_t>(stream));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool pack = ws && ws_bytes >= packed_kv_bytes(g);
+  if (pack)
+    if (int e = launch_pack_kv(g, K, V, ws, st)) return e;
+  return launch_sparse_attn(g, Q, K, V, idx, O, lse, 0, pack ? ws : nullptr, ctx, st);
 }
 
 int infllmv2_dense_attn(const infllmv2_params* p, const void* Q, const void* K, const void* V,
-                        void* O, float* lse, void* stream) {
+                        void* O, float* lse, void* ws, size_t ws_bytes, void* stream) {
   Geometry g;
   if (int e = validate(p, false, &g)) return e;
   if (empty(g)) return INFLLMV2_OK;
   if (int e = check_ptrs({Q, K, V, O, lse})) return e;
+  if (ws && !aligned16(ws)) return INFLLMV2_ERR_UNSUPPORTED;
   DevCtx ctx;
   if (int e = ctx_or_error(&ctx)) return e;
-  return launch_sparse_attn(g, Q, K, V, nullptr, O, lse, 1, ctx,
-                            static_cast<cudaStream_t>(stream));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool pack = ws && ws_bytes >= packed_kv_bytes(g);
+  if (pack)
+    if (int e = launch_pack_kv(g, K, V, ws, st)) return e;
+  return launch_sparse_attn(g, Q, K, V, nullptr, O, lse, 1, pack ? ws : nullptr, ctx, st);
 }
 
 int infllmv2_forward(const infllmv2_params* p, const void* Q, const void* K, const void* V,
@@ -218,14 +233,18 @@ int infllmv2_forward(const infllmv2_params* p, const void* Q, const void* K, con
   if (!p) return INFLLMV2_ERR_INVALID_ARG;
   const bool dense = p->T <= p->switch_threshold;
   if (path_used) *path_used = dense ? INFLLMV2_PATH_DENSE : INFLLMV2_PATH_SPARSE;
-  if (dense) return infllmv2_dense_attn(p, Q, K, V, O, lse, stream);
+  if (dense) return infllmv2_dense_attn(p, Q, K, V, O, lse, ws, ws_bytes, stream);
   Geometry g;
   if (int e = validate(p, true, &g)) return e;
   if (empty(g)) return INFLLMV2_OK;
+  // workspace: block scores of the selection, then the packed K/V tiles
+  const size_t sel = align256(select_ws_bytes(g));
+  if (ws_bytes < sel) return INFLLMV2_ERR_WORKSPACE;
   if (g.n_c > 0)
     if (int e = infllmv2_compress_keys(p, K, Kc_ws, stream)) return e;
   if (int e = infllmv2_select_blocks(p, Q, Kc_ws, idx_ws, ws, ws_bytes, stream)) return e;
-  return infllmv2_sparse_attn(p, Q, K, V, idx_ws, O, lse, stream);
+  return infllmv2_sparse_attn(p, Q, K, V, idx_ws, O, lse, static_cast<uint8_t*>(ws) + sel,
+                              ws_bytes - sel, stream);
 }
 
 int infllmv2_decode_step(const infllmv2_params* p, const void* q, const void* k_new,

@@ -91,10 +91,15 @@ int launch_compress_keys(const Geometry& g, const void* K, void* Kc, int kv_rows
 int launch_score_blocks(const Geometry& g, const void* Q, const void* Kc, float* scores,
                         const DevCtx& ctx, cudaStream_t st);
 int launch_topk(const Geometry& g, const float* scores, int32_t* idx, cudaStream_t st);
+// K/V block tiles (pack.cu): bytes for both tensors, and the repacking launch.
+size_t packed_kv_bytes(const Geometry& g);
+int launch_pack_kv(const Geometry& g, const void* K, const void* V, void* packed,
+                   cudaStream_t st);
 // Sparse attention over selected blocks; dense == 1 attends to every block <= t/64.
+// packed: K/V tiles from launch_pack_kv, or null to gather from K and V.
 int launch_sparse_attn(const Geometry& g, const void* Q, const void* K, const void* V,
-                       const int32_t* idx, void* O, float* lse, int dense, const DevCtx& ctx,
-                       cudaStream_t st);
+                       const int32_t* idx, void* O, float* lse, int dense, const void* packed,
+                       const DevCtx& ctx, cudaStream_t st);
 // Decode (decode.cu); g.T is the cache capacity.
 size_t decode_ws_bytes(const Geometry& g);
 int launch_decode_step(const Geometry& g, const void* q, const void* k_new, const void* v_new,

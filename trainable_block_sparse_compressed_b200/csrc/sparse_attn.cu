@@ -10,19 +10,31 @@
 // work by the union size; the kernel therefore runs each token on its own and
 // swaps the operands so that the 128-row side of tcgen05.mma is keys:
 //
-//   S^T[128 keys x 16 heads]  = K_pair (A, K-major) x Q^T (B, K-major)
-//   O^T[128 d    x 16 heads] += V_pair^T (A, MN-major) x P^T (B, K-major)
+//   S^T[128 keys x 16 heads]  = K_pair (A, K-major)   x Q^T (B, K-major)
+//   O^T[128 d    x 16 heads]  = V_pair^T (A, MN-major) x P^T (B, MN-major)
 //
 // A "pair" is two selected 64-key blocks gathered by TMA into one 128-row
-// operand (K and V: 4 x 8 KB boxes each).  Heads beyond G are padding.
-// Persistent CTAs (one per SM) stream pairs of consecutive items through a
-// 3-stage ring without draining between items.
+// operand (K and V: 2 x 2 boxes of 64 rows x 128 B).  Heads beyond G are
+// padding.  Persistent CTAs (one per SM) stream the pairs of their items
+// without draining between items.
 //
-// Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer / TMEM owner, warps
-// 2-5 = softmax (thread = TMEM lane = key row for S^T, = channel d for O^T).
-// Each pair's P V product lands in a fresh TMEM buffer and is folded into an
-// fp32 register accumulator with the usual online-softmax rescale, so the
-// accumulator never has to be rescaled inside tensor memory.
+// What bounds this kernel is the gather: every pair moves 64 KB from L2 into
+// shared memory through the SM's copy engine, which serves requests in issue
+// order, and S of a pair cannot start before its K has landed.  K and V travel
+// in separate rings (3 x 32 KB each), each filled by its own producer warp:
+// K is released as soon as its S product completes, V after its P V product,
+// so a wait for a V stage never holds back a K request.  The MMA warp runs a
+// non-blocking event loop that issues each P V the moment its P is written.
+// The softmax is split over two warpgroups by heads (heads 0-7 and 8-15 of
+// the same key rows), halving each thread's dependent chain.
+//
+// Softmax (thread = TMEM lane = key row of S^T, = channel d of O^T, for eight
+// heads): each head keeps a reference maximum m that only moves when a score
+// exceeds it by more than 8 (log2 units), so the common pair needs a single
+// barrier-OR and no cross-lane reduction; P = exp2(s - m) <= 256 stays exact
+// enough in bf16.  Each pair's P V lands in a fresh TMEM buffer and is folded
+// into an fp32 register accumulator with the rescale of its own reference, so
+// the accumulator is never rescaled inside tensor memory.
 //
 // Decode mode: one query token per sequence at t = seqlens[b]; the selected
 // blocks of each (sequence, kv head) are split into chunks so that enough
@@ -34,18 +46,24 @@
 namespace infllmv2 {
 namespace {
 
-constexpr int kStages = 3;
-constexpr int kSlotBytes = 64 * 128;                 // 64 rows x 128 B (one box)
+constexpr int kKStages = 3;
+constexpr int kVStages = 3;
+constexpr int kHalves = 2;                           // softmax warpgroups, 8 heads each
+constexpr int kHH = 8;                               // heads per warpgroup
+constexpr int kSlotBytes = 64 * 128;                 // 64 rows x 128 B (one TMA box)
 constexpr int kHalf = 2 * kSlotBytes;                // 128 rows x 64 channels
-constexpr int kStageBytes = 4 * kHalf;               // K (2 halves) + V (2 halves) = 64 KB
+constexpr int kPairBytes = 2 * kHalf;                // K or V of one pair: 32 KB
 constexpr int kQBytes = 16 * 256;                    // 16 rows x 128 channels
 constexpr int kPBytes = 16 * 256;                    // 16 heads x 128 keys
-constexpr int kThreads = 192;
+constexpr int kSoftmaxThreads = 128 * kHalves;
+constexpr int kThreads = 96 + kSoftmaxThreads;    // producers K/Q, MMA, producer V, softmax
 constexpr uint32_t kTmemCols = 64;                   // S^T x2, PV x2 (16 columns each)
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleSlack = 8.0f;                // log2 units
 
 struct AttnSmem {
-  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t q_full[2], q_empty[2];
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full[2];
@@ -53,11 +71,15 @@ struct AttnSmem {
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
-  float red[2][4][16];   // per-warp partial head maxima, double-buffered by pair
-  float lsum[4][16];     // per-warp partial row sums at item end
+  float red[kHalves][4][kHH];   // per-warp head maxima (rescale path)
+  float lsum[kHalves][4][kHH];  // per-warp row sums at item end
+  int blocks[kMaxTopk];
 };
 
 struct AttnArgs {
+  const uint8_t* Kp;        // packed K / V tiles (pack.cu), or null: tensor-map gather
+  const uint8_t* Vp;
+  int nb;                   // blocks per (batch, kv head) of the packed tiles
   const int32_t* idx;       // selected blocks (null when dense)
   __nv_bfloat16* O;         // final output (prefill / dense)
   float* lse;
@@ -89,8 +111,21 @@ __device__ __forceinline__ int count_valid(const int32_t* __restrict__ row, int 
   return n;
 }
 
-// Resolves work item `it` (warp-collective: every lane gets the same answer).
-__device__ __forceinline__ Item resolve_item(int64_t it, const AttnArgs& a, int lane) {
+// The same count by one thread alone.
+__device__ __forceinline__ int count_valid_1(const int32_t* __restrict__ row, int topk, int cur) {
+  int n = 0;
+  while (n < topk) {
+    const int v = __ldg(row + n);
+    if (v < 0 || v > cur) break;
+    ++n;
+  }
+  return n;
+}
+
+// Resolves work item `it`.  collective: called by a whole warp (every lane
+// gets the same answer); otherwise by a single thread.
+__device__ __forceinline__ Item resolve_item(int64_t it, const AttnArgs& a, int lane,
+                                             bool collective) {
   Item r;
   if (a.mode == 2) {
     const int c = static_cast<int>(it % a.n_chunks);
@@ -101,7 +136,10 @@ __device__ __forceinline__ Item resolve_item(int64_t it, const AttnArgs& a, int 
     r.qtok = 0;
     r.cur = r.t / kBlock;
     r.row = a.idx + bg * a.topk;
-    const int nv = (r.t >= 0 && r.t < a.T) ? count_valid(r.row, a.topk, r.cur, lane) : 0;
+    int nv = 0;
+    if (r.t >= 0 && r.t < a.T)
+      nv = collective ? count_valid(r.row, a.topk, r.cur, lane)
+                      : count_valid_1(r.row, a.topk, r.cur);
     r.e0 = c * a.chunk_blocks;
     r.n = max(0, min(a.chunk_blocks, nv - r.e0));
   } else {
@@ -118,14 +156,27 @@ __device__ __forceinline__ Item resolve_item(int64_t it, const AttnArgs& a, int 
       r.n = r.cur + 1;
     } else {
       r.row = a.idx + ((static_cast<int64_t>(r.b) * a.Hkv + r.g) * a.T + r.t) * a.topk;
-      r.n = count_valid(r.row, a.topk, r.cur, lane);
+      r.n = collective ? count_valid(r.row, a.topk, r.cur, lane)
+                       : count_valid_1(r.row, a.topk, r.cur);
     }
   }
   r.n_pairs = (r.n + 1) >> 1;
   return r;
 }
 
-// Block of entry e (0 <= e < n) of an item.
+// The k-th item of this CTA (>= n_items when there is none).  Items are dealt
+// in chunks of consecutive ones, chunk j to CTA j % gridDim.x: tokens that
+// CTAs process at the same time are then far apart, so they do not all fetch
+// the same local blocks from the same L2 lines at once, as they would if
+// consecutive tokens went to consecutive CTAs.
+constexpr int kChunkItems = 16;
+__device__ __forceinline__ int64_t item_of(int64_t k, int64_t n_items) {
+  const int64_t chunk = k / kChunkItems;
+  const int64_t it = (chunk * gridDim.x + blockIdx.x) * kChunkItems + k % kChunkItems;
+  return it < n_items ? it : n_items;
+}
+
+// Block of entry e (0 <= e < n) of an item, from global memory.
 __device__ __forceinline__ int item_block(const Item& it, int e) {
   return it.row ? __ldg(it.row + it.e0 + e) : it.e0 + e;
 }
@@ -147,8 +198,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t* sKV = base;                                   // kStages x 64 KB
-  uint8_t* sQ = sKV + kStages * kStageBytes;             // 2 x 4 KB
+  uint8_t* sK = base;                                    // kKStages x 32 KB
+  uint8_t* sV = sK + kKStages * kPairBytes;              // kVStages x 32 KB
+  uint8_t* sQ = sV + kVStages * kPairBytes;              // 2 x 4 KB
   uint8_t* sP = sQ + 2 * kQBytes;                        // 2 x 4 KB
   AttnSmem& sm = *reinterpret_cast<AttnSmem*>(sP + 2 * kPBytes);
 
@@ -162,23 +214,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   // second slot stale, and stale data must be finite (it is multiplied by 0)
   {
     uint4* p = reinterpret_cast<uint4*>(base);
-    const int n16 = (kStages * kStageBytes + 2 * kQBytes + 2 * kPBytes) / 16;
+    const int n16 = ((kKStages + kVStages) * kPairBytes + 2 * kQBytes + 2 * kPBytes) / 16;
     for (int i = threadIdx.x; i < n16; i += blockDim.x) p[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
   }
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sm.kv_full[s], 1);
-      mbar_init(&sm.kv_empty[s], 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.v_empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&sm.q_full[a], 1);
       mbar_init(&sm.q_empty[a], 1);
       mbar_init(&sm.s_full[a], 1);
-      mbar_init(&sm.s_empty[a], 128);
-      mbar_init(&sm.p_full[a], 128);
+      mbar_init(&sm.s_empty[a], kSoftmaxThreads);
+      mbar_init(&sm.p_full[a], kSoftmaxThreads);
       mbar_init(&sm.pv_full[a], 1);
-      mbar_init(&sm.pv_empty[a], 128);
+      mbar_init(&sm.pv_empty[a], kSoftmaxThreads);
     }
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
@@ -194,207 +250,305 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort_flag = &sm.abort_flag;
 
-  if (warp == 0) {
-    // ------------------------------ producer ------------------------------
+  if (warp == 0 || warp == 2) {
+    // ------------------------------ producers ------------------------------
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
     }
-    int64_t gp = 0;  // global pair counter of this CTA
-    int qk = 0;      // items with at least one pair
-    int q_issued = 0;
-    int64_t kv_issued = 0;
+    struct PairLoad {
+      int64_t gp;
+      int b, g, blk0, blk1;
+      bool two;
+    };
+    // packed tiles: one 16 KB bulk copy per block, block b of the pair at
+    // slot offset 16 KB; otherwise two 64-channel tensor-map boxes per block,
+    // 128-byte swizzled, halves 16 KB apart
+    auto issue = [&](const PairLoad& pl, bool is_v) -> bool {
+      const int nst = is_v ? kVStages : kKStages;
+      const int s = static_cast<int>(pl.gp % nst);
+      uint64_t* full = is_v ? &sm.v_full[s] : &sm.k_full[s];
+      uint64_t* empty = is_v ? &sm.v_empty[s] : &sm.k_empty[s];
+      if (pl.gp >= nst && !wait_or_abort(empty, ((pl.gp / nst) & 1) ^ 1, ctx, abort_flag))
+        return false;
+      uint8_t* st = (is_v ? sV : sK) + s * kPairBytes;
+      const uint8_t* packed = is_v ? args.Vp : args.Kp;
+      const CUtensorMap* tm = is_v ? &tmV : &tmK;
+      const int64_t tile0 = (static_cast<int64_t>(pl.b) * args.Hkv + pl.g) * args.nb;
+      mbar_arrive_expect_tx(full, (pl.two ? 4 : 2) * kSlotBytes);
+      for (int slot = 0; slot < (pl.two ? 2 : 1); ++slot) {
+        const int blk = slot ? pl.blk1 : pl.blk0;
+        if (packed) {
+          bulk_load(st + slot * kHalf, packed + (tile0 + blk) * kHalf, kHalf, full);
+        } else {
+          tma_load_4d(st + slot * kSlotBytes, tm, full, 0, pl.g, blk * kBlock, pl.b);
+          tma_load_4d(st + kHalf + slot * kSlotBytes, tm, full, 64, pl.g, blk * kBlock, pl.b);
+        }
+      }
+      return true;
+    };
+    // warp 0 issues Q and K, warp 2 issues V: a wait for a free V stage (which
+    // frees only after a softmax and a P V product) never holds back the K
+    // that the next S product needs, and the reverse
+    const bool is_v = warp == 2;
+    int64_t gp = 0;       // pairs issued by this warp
+    int qk = 0;           // Q loads issued
     bool ok = true;
-    for (int64_t it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
-      const Item item = resolve_item(it, args, lane);
+    for (int64_t k = 0, it; ok && (it = item_of(k, n_items)) < n_items; ++k) {
+      const Item item = resolve_item(it, args, lane, true);
       if (item.n_pairs == 0) continue;
-      const int qb = qk & 1;
-      if (lane == 0) {
+      if (!is_v && lane == 0) {
+        const int qb = qk & 1;
         if (qk >= 2) ok = wait_or_abort(&sm.q_empty[qb], ((qk >> 1) & 1) ^ 1, ctx, abort_flag);
         if (ok) {
           uint8_t* qdst = sQ + qb * kQBytes;
           mbar_arrive_expect_tx(&sm.q_full[qb], G * 256);
           tma_load_4d(qdst, &tmQ, &sm.q_full[qb], 0, item.g * G, item.qtok, item.b);
           tma_load_4d(qdst + 2048, &tmQ, &sm.q_full[qb], 64, item.g * G, item.qtok, item.b);
-          ++q_issued;
+          ++qk;
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      ++qk;
-      for (int p = 0; ok && p < item.n_pairs; ++p, ++gp) {
-        const int blk0 = item_block(item, 2 * p);
-        const bool two = 2 * p + 1 < item.n;
-        const int blk1 = two ? item_block(item, 2 * p + 1) : 0;
-        if (lane == 0) {
-          const int s = static_cast<int>(gp % kStages);
-          if (gp >= kStages)
-            ok = wait_or_abort(&sm.kv_empty[s], ((gp / kStages) & 1) ^ 1, ctx, abort_flag);
-          if (ok) {
-            uint8_t* st = sKV + s * kStageBytes;
-            mbar_arrive_expect_tx(&sm.kv_full[s], (two ? 8 : 4) * kSlotBytes);
-            for (int slot = 0; slot < (two ? 2 : 1); ++slot) {
-              const int r0 = (slot ? blk1 : blk0) * kBlock;
-              uint8_t* d = st + slot * kSlotBytes;
-              tma_load_4d(d, &tmK, &sm.kv_full[s], 0, item.g, r0, item.b);
-              tma_load_4d(d + kHalf, &tmK, &sm.kv_full[s], 64, item.g, r0, item.b);
-              tma_load_4d(d + 2 * kHalf, &tmV, &sm.kv_full[s], 0, item.g, r0, item.b);
-              tma_load_4d(d + 3 * kHalf, &tmV, &sm.kv_full[s], 64, item.g, r0, item.b);
-            }
-            ++kv_issued;
-          }
-        }
+      for (int p = 0; ok && p < item.n_pairs; ++p) {
+        PairLoad pl;
+        pl.gp = gp;
+        pl.b = item.b;
+        pl.g = item.g;
+        pl.blk0 = item_block(item, 2 * p);
+        pl.two = 2 * p + 1 < item.n;
+        pl.blk1 = pl.two ? item_block(item, 2 * p + 1) : 0;
+        if (lane == 0) ok = issue(pl, is_v);
         ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (ok) ++gp;
       }
     }
     // drain: never leave with copies of this CTA in flight (matters only when
     // a wait above gave up; otherwise these phases completed long ago)
     if (lane == 0) {
-      for (int x = 0; x < 2 && x < q_issued; ++x)
-        mbar_wait(&sm.q_full[x], ((q_issued - 1 - x) / 2) & 1, ctx.wait_ns);
-      for (int x = 0; x < kStages && x < kv_issued; ++x)
-        mbar_wait(&sm.kv_full[x], ((kv_issued - 1 - x) / kStages) & 1, ctx.wait_ns);
+      if (!is_v) {
+        for (int x = 0; x < 2 && x < qk; ++x)
+          mbar_wait(&sm.q_full[x], ((qk - 1 - x) >> 1) & 1, ctx.wait_ns);
+        for (int x = 0; x < kKStages && x < gp; ++x)
+          mbar_wait(&sm.k_full[x], ((gp - 1 - x) / kKStages) & 1, ctx.wait_ns);
+      } else {
+        for (int x = 0; x < kVStages && x < gp; ++x)
+          mbar_wait(&sm.v_full[x], ((gp - 1 - x) / kVStages) & 1, ctx.wait_ns);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer ------------------------------
-    // The whole warp walks the items (the index scan is warp-collective);
-    // lane 0 waits on barriers and issues the tensor-core work.
-    constexpr uint32_t idesc_s = instr_desc_bf16(128, 16, 0, 0);
-    constexpr uint32_t idesc_pv = instr_desc_bf16(128, 16, 1, 0);
-    int64_t gp = 0;
-    int qk = 0;
-    bool ok = true;
-    bool pv_pending = false;  // P V of pair gp-1 not yet issued
-    auto issue_pv = [&](int64_t q) -> bool {
-      const int a = static_cast<int>(q & 1);
-      const int s = static_cast<int>(q % kStages);
-      if (!wait_or_abort(&sm.p_full[a], (q >> 1) & 1, ctx, abort_flag)) return false;
-      if (q >= 2 && !wait_or_abort(&sm.pv_empty[a], ((q >> 1) & 1) ^ 1, ctx, abort_flag))
+    // Lane 0 alone runs a non-blocking event loop: it issues every P V whose
+    // P, V stage and TMEM buffer are ready (in pair order), and the next S^T
+    // when its K stage, Q and S buffer are ready.  It gives up when nothing
+    // has been issued for the wait limit.
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = instr_desc_bf16(128, 16, 0, 0);
+      constexpr uint32_t idesc_pv = instr_desc_bf16(128, 16, 1, 1);
+      int64_t k_item = 0;
+      Item item;
+      item.n_pairs = 0;
+      int p = 0;
+      auto next_item = [&]() {
+        for (int64_t it; (it = item_of(k_item, n_items)) < n_items;) {
+          ++k_item;
+          item = resolve_item(it, args, 0, false);
+          if (item.n_pairs > 0) {
+            p = 0;
+            return true;
+          }
+        }
         return false;
-      tc_fence_after();
-      const uint32_t v_addr = smem_u32(sKV + s * kStageBytes + 2 * kHalf);
-      const uint32_t p_addr = smem_u32(sP + a * kPBytes);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint64_t ad = smem_desc(v_addr + k * 2048, kHalf, 1024, 2);
-        const uint64_t bd = smem_desc(p_addr + (k >> 2) * 2048 + (k & 3) * 32, 16, 1024, 2);
-        umma_bf16(tmem + 32 + a * 16, ad, bd, idesc_pv, k > 0 ? 1u : 0u);
-      }
-      umma_commit(&sm.pv_full[a]);
-      umma_commit(&sm.kv_empty[s]);
-      return true;
-    };
-    for (int64_t it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
-      const Item item = resolve_item(it, args, lane);
-      if (item.n_pairs == 0) continue;
-      const int qb = qk & 1;
-      if (lane == 0) {
-        ok = wait_or_abort(&sm.q_full[qb], (qk >> 1) & 1, ctx, abort_flag);
-        const uint32_t q_addr = smem_u32(sQ + qb * kQBytes);
-        for (int p = 0; ok && p < item.n_pairs; ++p, ++gp) {
-          const int s = static_cast<int>(gp % kStages);
-          const int a = static_cast<int>(gp & 1);
-          if (!wait_or_abort(&sm.kv_full[s], (gp / kStages) & 1, ctx, abort_flag) ||
-              (gp >= 2 && !wait_or_abort(&sm.s_empty[a], ((gp >> 1) & 1) ^ 1, ctx, abort_flag))) {
-            ok = false;
-            break;
-          }
+      };
+      bool have = next_item();
+      int64_t gp_s = 0;   // S products issued
+      int64_t gp_pv = 0;  // P V products issued
+      int qk = 0;         // items whose Q has been consumed
+      uint64_t t_progress = global_timer_ns();
+      while (true) {
+        bool did = false;
+        // P V products, in order, as soon as P, V and the TMEM buffer are ready
+        while (gp_pv < gp_s) {
+          const int a = static_cast<int>(gp_pv & 1);
+          const int vs = static_cast<int>(gp_pv % kVStages);
+          if (!mbar_test(&sm.p_full[a], (gp_pv >> 1) & 1)) break;
+          if (gp_pv >= 2 && !mbar_test(&sm.pv_empty[a], ((gp_pv >> 1) & 1) ^ 1)) break;
+          if (!mbar_test(&sm.v_full[vs], (gp_pv / kVStages) & 1)) break;
           tc_fence_after();
-          const uint32_t k_addr = smem_u32(sKV + s * kStageBytes);
+          const uint32_t v_addr = smem_u32(sV + vs * kPairBytes);
+          const uint32_t p_addr = smem_u32(sP + a * kPBytes);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint32_t off = (k >> 2) * kHalf + (k & 3) * 32;
-            const uint64_t ad = smem_desc(k_addr + off, 16, 1024, 2);
-            const uint64_t bd = smem_desc(q_addr + (k >> 2) * 2048 + (k & 3) * 32, 16, 1024, 2);
-            umma_bf16(tmem + a * 16, ad, bd, idesc_s, k > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk) {
+            // A: V^T, MN-major 128-byte swizzle: 16 keys = two 8-row groups (2 KB)
+            // (packed tiles: MN-major, no swizzle, channel groups 128 B apart
+            // (SBO), 8-key groups 2 KB apart (LBO), 16 keys = 4 KB)
+            const uint64_t ad = args.Vp ? smem_desc(v_addr + kk * 4096, 2048, 128, 0)
+                                        : smem_desc(v_addr + kk * 2048, kHalf, 1024, 2);
+            // B: P^T, MN-major, no swizzle: 8x8 core matrices of 128 B, heads
+            // 0-7 / 8-15 128 B apart (SBO), 8-key groups 256 B apart (LBO)
+            const uint64_t bd = smem_desc(p_addr + kk * 512, 256, 128, 0);
+            umma_bf16(tmem + 32 + a * 16, ad, bd, idesc_pv, kk > 0 ? 1u : 0u);
           }
-          umma_commit(&sm.s_full[a]);
-          if (p == item.n_pairs - 1) umma_commit(&sm.q_empty[qb]);
-          if (pv_pending && !issue_pv(gp - 1)) {
-            ok = false;
-            break;
+          umma_commit(&sm.pv_full[a]);
+          umma_commit(&sm.v_empty[vs]);
+          ++gp_pv;
+          did = true;
+        }
+        // the next S^T product
+        if (have) {
+          const int qb = qk & 1;
+          const int ks = static_cast<int>(gp_s % kKStages);
+          const int a = static_cast<int>(gp_s & 1);
+          bool ready = gp_s - gp_pv < 2;
+          if (ready && p == 0) ready = mbar_test(&sm.q_full[qb], (qk >> 1) & 1);
+          if (ready) ready = mbar_test(&sm.k_full[ks], (gp_s / kKStages) & 1);
+          if (ready && gp_s >= 2) ready = mbar_test(&sm.s_empty[a], ((gp_s >> 1) & 1) ^ 1);
+          if (ready) {
+            tc_fence_after();
+            const uint32_t k_addr = smem_u32(sK + ks * kPairBytes);
+            const uint32_t q_addr = smem_u32(sQ + qb * kQBytes);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              // packed tiles: K-major, no swizzle, 16 channels = two 128 B
+              // core-matrix columns (LBO), 8-row groups 2 KB apart (SBO);
+              // boxes: K-major 128-byte swizzle, 64-channel halves 16 KB apart
+              const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+              const uint64_t ad = args.Kp ? smem_desc(k_addr + kk * 256, 128, 2048, 0)
+                                          : smem_desc(k_addr + off, 16, 1024, 2);
+              const uint64_t bd =
+                  smem_desc(q_addr + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024, 2);
+              umma_bf16(tmem + a * 16, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&sm.s_full[a]);
+            umma_commit(&sm.k_empty[ks]);
+            ++gp_s;
+            if (++p == item.n_pairs) {
+              umma_commit(&sm.q_empty[qb]);
+              ++qk;
+              have = next_item();
+            }
+            did = true;
           }
-          pv_pending = true;
+        } else if (gp_pv == gp_s) {
+          break;
+        }
+        if (did) {
+          t_progress = global_timer_ns();
+        } else if (!*abort_flag && global_timer_ns() - t_progress <= ctx.wait_ns) {
+          // idle: back off so that polling does not contend with the copy
+          // engine's and the other warps' updates of the same barriers
+          __nanosleep(64);
+        } else {
+          if (!*abort_flag) report_status(ctx.status, INFLLMV2_STATUS_TIMEOUT);
+          *abort_flag = 1;
+          break;
         }
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      gp = __shfl_sync(0xffffffffu, gp, 0);
-      ++qk;
-    }
-    if (lane == 0) {
-      if (ok && pv_pending) issue_pv(gp - 1);
       // drain: all MMAs of this CTA complete before TMEM is released
       umma_commit(&sm.drain);
       mbar_wait(&sm.drain, 0, ctx.wait_ns);
     }
   } else {
     // ------------------------------ softmax ------------------------------
-    const int quad = warp & 3;
+    // two warpgroups on the same items: warpgroup hf owns heads 8hf .. 8hf+7
+    const int hf = (warp - 3) >> 2;
+    const int quad = warp & 3;       // TMEM lane quadrant of this warp
     const int r = quad * 32 + lane;  // key row of S^T and channel d of O^T
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const int gt = threadIdx.x - 96; // index among all softmax threads
+    // this thread's TMEM lane, at the first of its warpgroup's eight columns
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + hf * kHH;
+    // Every named barrier spans all 256 softmax threads: a decision taken
+    // there (rescale, abort) is the same for both warpgroups, so neither can
+    // leave the loop while the other waits at a later barrier.
+    constexpr uint32_t bar_sync_id = 1, bar_or_id = 2;
     const int slot = r >> 6;         // which block of the pair this key row belongs to
     const int krow = r & 63;
+    // P^T (MN-major, no swizzle): key r's heads 8hf..8hf+7 form one 16-byte
+    // row of core matrix (r / 8, hf) at (r / 8) * 256 + hf * 128 + (r % 8) * 16
+    const uint32_t p_off = (r >> 3) * 256 + hf * 128 + (r & 7) * 16;
     int64_t gp = 0;
     bool ok = true;
-    // P^T operand byte offset of this thread's key column (K-major, 128-byte swizzle)
-    const uint32_t p_col = (r >> 6) * 2048 + (krow & 7) * 2;
-    for (int64_t it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
-      const Item item = resolve_item(it, args, lane);
-      float m[16], l[16], o[16], alpha_prev[16];
+    for (int64_t k = 0, it; ok && (it = item_of(k, n_items)) < n_items; ++k) {
+      const Item item = resolve_item(it, args, lane, true);
+      // the item's blocks, staged once in shared memory by all 256 threads
+      if (item.row)
+        for (int e = gt; e < item.n; e += kSoftmaxThreads)
+          sm.blocks[e] = __ldg(item.row + item.e0 + e);
+      named_bar_sync(bar_sync_id, kSoftmaxThreads);
+      float m[kHH], l[kHH], o[kHH], alpha_prev[kHH];
 #pragma unroll
-      for (int h = 0; h < 16; ++h) {
+      for (int h = 0; h < kHH; ++h) {
         m[h] = -INFINITY;
         l[h] = 0.f;
         o[h] = 0.f;
         alpha_prev[h] = 0.f;
       }
       for (int p = 0; p <= item.n_pairs; ++p) {
-        float alpha[16];
+        float alpha[kHH];
         if (p < item.n_pairs) {
           const int a = static_cast<int>(gp & 1);
-          const bool w = !*abort_flag && mbar_wait(&sm.s_full[a], (gp >> 1) & 1, ctx.wait_ns);
-          if (named_bar_or(2, 128, !w)) {
-            if (!w) report_status(ctx.status, INFLLMV2_STATUS_TIMEOUT);
+          if (!*abort_flag && !mbar_wait(&sm.s_full[a], (gp >> 1) & 1, ctx.wait_ns)) {
+            report_status(ctx.status, INFLLMV2_STATUS_TIMEOUT);
             *abort_flag = 1;
-            ok = false;
-            break;
           }
           tc_fence_after();
-          float x[16];
-          tmem_ld16(lane_addr + a * 16, x);
+          float x[kHH];
+          tmem_ld8(lane_addr + a * 16, x);
           tmem_ld_wait();
           tc_fence_before();
           mbar_arrive(&sm.s_empty[a]);
           const int e = 2 * p + slot;
-          const int blk = e < item.n ? item_block(item, e) : -1;
+          const int blk = e < item.n ? (item.row ? sm.blocks[e] : item.e0 + e) : -1;
           const bool valid = blk >= 0 && blk * kBlock + krow <= item.t;
-          float s[16];
+          float s[kHH];
+          bool exceed = false;
 #pragma unroll
-          for (int h = 0; h < 16; ++h) {
+          for (int h = 0; h < kHH; ++h) {
             s[h] = valid ? x[h] * scale_log2 : -INFINITY;
-            const float wm = warp_max(s[h]);
-            if (lane == 0) sm.red[a][quad][h] = wm;
+            exceed |= s[h] > m[h] + kRescaleSlack;
           }
-          named_bar_sync(1, 128);
+          // one barrier decides for the warpgroup: move the references (first
+          // pair, or a score far above them) or abort after a timeout.
+          // Decisions use barrier-ORed snapshots of the CTA-wide abort flag,
+          // which other threads may set at any moment, so that the group's
+          // threads never split at a later named barrier.
+          const bool ab = *abort_flag != 0;
+          if (named_bar_or(bar_or_id, kSoftmaxThreads, exceed || ab)) {
+            if (named_bar_or(bar_or_id, kSoftmaxThreads, ab)) {
+              ok = false;
+              break;
+            }
 #pragma unroll
-          for (int h = 0; h < 16; ++h) {
-            const float tm = fmaxf(fmaxf(sm.red[a][0][h], sm.red[a][1][h]),
-                                   fmaxf(sm.red[a][2][h], sm.red[a][3][h]));
-            const float mn = fmaxf(m[h], tm);
-            alpha[h] = fast_exp2(m[h] - mn);
-            m[h] = mn;
-            const float pr = fast_exp2(s[h] - mn);
-            l[h] = l[h] * alpha[h] + pr;
-            s[h] = pr;
-          }
-          // P^T (bf16) into this pair's P buffer: row = head, column = key
-          uint8_t* pb = sP + a * kPBytes;
+            for (int h = 0; h < kHH; ++h) {
+              float wm;
+              asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(wm) : "f"(s[h]));
+              if (lane == 0) sm.red[hf][quad][h] = wm;
+            }
+            named_bar_sync(bar_sync_id, kSoftmaxThreads);
 #pragma unroll
-          for (int h = 0; h < 16; ++h) {
-            const uint32_t off =
-                p_col + (h >> 3) * 1024 + (h & 7) * 128 + (((krow >> 3) ^ (h & 7)) << 4);
-            *reinterpret_cast<__nv_bfloat16*>(pb + off) = __float2bfloat16_rn(s[h]);
+            for (int h = 0; h < kHH; ++h) {
+              const float tm = fmaxf(fmaxf(sm.red[hf][0][h], sm.red[hf][1][h]),
+                                     fmaxf(sm.red[hf][2][h], sm.red[hf][3][h]));
+              const float mn = fmaxf(m[h], tm);
+              alpha[h] = fast_exp2(m[h] - mn);
+              m[h] = mn;
+            }
+            named_bar_sync(bar_sync_id, kSoftmaxThreads);  // red[] is rewritten later
+          } else {
+#pragma unroll
+            for (int h = 0; h < kHH; ++h) alpha[h] = 1.f;
           }
+          uint32_t pk[4];
+#pragma unroll
+          for (int h = 0; h < kHH; h += 2) {
+            const float p0 = fast_exp2(s[h] - m[h]);
+            const float p1 = fast_exp2(s[h + 1] - m[h + 1]);
+            l[h] = l[h] * alpha[h] + p0;
+            l[h + 1] = l[h + 1] * alpha[h + 1] + p1;
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+            pk[h >> 1] = *reinterpret_cast<uint32_t*>(&b2);
+          }
+          *reinterpret_cast<uint4*>(sP + a * kPBytes + p_off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           fence_proxy_async_smem();
           mbar_arrive(&sm.p_full[a]);
         }
@@ -402,69 +556,79 @@ __global__ void __launch_bounds__(kThreads, 1)
           // fold in P V of the previous pair
           const int64_t q = gp - 1;
           const int a = static_cast<int>(q & 1);
-          const bool w = !*abort_flag && mbar_wait(&sm.pv_full[a], (q >> 1) & 1, ctx.wait_ns);
-          if (named_bar_or(2, 128, !w)) {
-            if (!w) report_status(ctx.status, INFLLMV2_STATUS_TIMEOUT);
+          if (!*abort_flag && !mbar_wait(&sm.pv_full[a], (q >> 1) & 1, ctx.wait_ns)) {
+            report_status(ctx.status, INFLLMV2_STATUS_TIMEOUT);
             *abort_flag = 1;
-            ok = false;
-            break;
           }
           tc_fence_after();
-          float pv[16];
-          tmem_ld16(lane_addr + 32 + a * 16, pv);
+          float pv[kHH];
+          tmem_ld8(lane_addr + 32 + a * 16, pv);
           tmem_ld_wait();
           tc_fence_before();
           mbar_arrive(&sm.pv_empty[a]);
 #pragma unroll
-          for (int h = 0; h < 16; ++h) o[h] = o[h] * alpha_prev[h] + pv[h];
+          for (int h = 0; h < kHH; ++h) o[h] = o[h] * alpha_prev[h] + pv[h];
         }
         if (p < item.n_pairs) {
 #pragma unroll
-          for (int h = 0; h < 16; ++h) alpha_prev[h] = alpha[h];
+          for (int h = 0; h < kHH; ++h) alpha_prev[h] = alpha[h];
           ++gp;
         }
       }
       if (!ok) break;
       // ---- item epilogue: row sums, then final output or decode partial ----
 #pragma unroll
-      for (int h = 0; h < 16; ++h) {
+      for (int h = 0; h < kHH; ++h) {
         const float ws = warp_sum(l[h]);
-        if (lane == 0) sm.lsum[quad][h] = ws;
+        if (lane == 0) sm.lsum[hf][quad][h] = ws;
       }
-      named_bar_sync(1, 128);
+      if (named_bar_or(bar_or_id, kSoftmaxThreads, *abort_flag)) {
+        ok = false;
+        break;
+      }
+      // heads of this warpgroup that exist (G < 16 leaves padding heads)
+      const int h_begin = hf * kHH;
       if (args.mode == 2) {
         float* po = args.part + it * (G * kHeadDim);
         float* pml = args.part + n_items * (G * kHeadDim) + it * (2 * G);
 #pragma unroll
-        for (int h = 0; h < G; ++h) po[h * kHeadDim + r] = item.n_pairs > 0 ? o[h] : 0.f;
-        if (r < G) {
-          const float L = sm.lsum[0][r] + sm.lsum[1][r] + sm.lsum[2][r] + sm.lsum[3][r];
+        for (int h = 0; h < kHH; ++h)
+          if (h_begin + h < G) po[(h_begin + h) * kHeadDim + r] = item.n_pairs > 0 ? o[h] : 0.f;
+        if (r < kHH && h_begin + r < G) {
+          const float L = sm.lsum[hf][0][r] + sm.lsum[hf][1][r] + sm.lsum[hf][2][r] +
+                          sm.lsum[hf][3][r];
           float mr = -INFINITY;
 #pragma unroll
-          for (int h = 0; h < 16; ++h)
+          for (int h = 0; h < kHH; ++h)
             if (h == r) mr = m[h];
-          pml[2 * r] = item.n_pairs > 0 ? mr : -INFINITY;
-          pml[2 * r + 1] = item.n_pairs > 0 ? L : 0.f;
+          pml[2 * (h_begin + r)] = item.n_pairs > 0 ? mr : -INFINITY;
+          pml[2 * (h_begin + r) + 1] = item.n_pairs > 0 ? L : 0.f;
         }
       } else {
-        const int64_t orow = (static_cast<int64_t>(item.b) * args.T + item.t) * args.Hq + item.g * G;
+        const int64_t orow =
+            (static_cast<int64_t>(item.b) * args.T + item.t) * args.Hq + item.g * G;
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float L = sm.lsum[0][h] + sm.lsum[1][h] + sm.lsum[2][h] + sm.lsum[3][h];
-          const float val = item.n_pairs > 0 ? o[h] / L : 0.f;
-          args.O[(orow + h) * kHeadDim + r] = __float2bfloat16_rn(val);
+        for (int h = 0; h < kHH; ++h) {
+          if (h_begin + h < G) {
+            const float L = sm.lsum[hf][0][h] + sm.lsum[hf][1][h] + sm.lsum[hf][2][h] +
+                            sm.lsum[hf][3][h];
+            const float val = item.n_pairs > 0 ? o[h] / L : 0.f;
+            args.O[(orow + h_begin + h) * kHeadDim + r] = __float2bfloat16_rn(val);
+          }
         }
-        if (r < G) {
-          const float L = sm.lsum[0][r] + sm.lsum[1][r] + sm.lsum[2][r] + sm.lsum[3][r];
+        if (r < kHH && h_begin + r < G) {
+          const float L = sm.lsum[hf][0][r] + sm.lsum[hf][1][r] + sm.lsum[hf][2][r] +
+                          sm.lsum[hf][3][r];
           float mr = -INFINITY;
 #pragma unroll
-          for (int h = 0; h < 16; ++h)
+          for (int h = 0; h < kHH; ++h)
             if (h == r) mr = m[h];
-          args.lse[(static_cast<int64_t>(item.b) * args.Hq + item.g * G + r) * args.T + item.t] =
-              item.n_pairs > 0 ? (mr + __log2f(L)) * kLn2 : -INFINITY;
+          args.lse[(static_cast<int64_t>(item.b) * args.Hq + item.g * G + h_begin + r) * args.T +
+                   item.t] = item.n_pairs > 0 ? (mr + __log2f(L)) * kLn2 : -INFINITY;
         }
       }
-      named_bar_sync(1, 128);  // lsum is reused by the next item
+      // lsum and the staged blocks are reused by the next item
+      named_bar_sync(bar_sync_id, kSoftmaxThreads);
     }
   }
 
@@ -479,7 +643,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int G>
 int launch_attn_g(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                   const AttnArgs& args, int64_t n_items, const DevCtx& ctx, cudaStream_t st) {
-  const size_t smem = 1024 + kStages * kStageBytes + 2 * kQBytes + 2 * kPBytes + sizeof(AttnSmem);
+  const size_t smem =
+      1024 + (kKStages + kVStages) * kPairBytes + 2 * kQBytes + 2 * kPBytes + sizeof(AttnSmem);
   static bool configured = false;
   if (!configured) {
     if (cudaFuncSetAttribute(sparse_attn_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -528,10 +693,15 @@ int launch_attn(const Geometry& g, const void* Q, int q_tokens, const void* K, c
 }  // namespace
 
 int launch_sparse_attn(const Geometry& g, const void* Q, const void* K, const void* V,
-                       const int32_t* idx, void* O, float* lse, int dense, const DevCtx& ctx,
-                       cudaStream_t st) {
+                       const int32_t* idx, void* O, float* lse, int dense, const void* packed,
+                       const DevCtx& ctx, cudaStream_t st) {
   if (g.B == 0 || g.T == 0) return INFLLMV2_OK;
   AttnArgs a{};
+  if (packed) {
+    a.Kp = static_cast<const uint8_t*>(packed);
+    a.Vp = a.Kp + packed_kv_bytes(g) / 2;
+    a.nb = (g.T + kBlock - 1) / kBlock;
+  }
   a.idx = idx;
   a.O = static_cast<__nv_bfloat16*>(O);
   a.lse = lse;

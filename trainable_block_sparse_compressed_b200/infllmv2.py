@@ -26,7 +26,7 @@ ERR_WORKSPACE = -5
 ERR_DEVICE_CHECK = -6
 STATUS_TIMEOUT = 0x1
 STATUS_SEQ_FULL = 0x2
-OP_SELECT, OP_FORWARD, OP_DECODE = 1, 2, 3
+OP_SELECT, OP_FORWARD, OP_DECODE, OP_ATTN = 1, 2, 3, 4
 PATH_DENSE, PATH_SPARSE = 1, 2
 
 # every symbol include/infllmv2.h declares
@@ -80,8 +80,8 @@ def load(path: Optional[str] = None):
     sig = {
         "infllmv2_compress_keys": (ctypes.c_int, [P, vp, vp, vp]),
         "infllmv2_select_blocks": (ctypes.c_int, [P, vp, vp, vp, vp, sz, vp]),
-        "infllmv2_sparse_attn": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp]),
-        "infllmv2_dense_attn": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp]),
+        "infllmv2_sparse_attn": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "infllmv2_dense_attn": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
         "infllmv2_forward": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "infllmv2_decode_step": (ctypes.c_int,
                                  [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
@@ -162,16 +162,22 @@ def select_blocks(p: Params, Q, Kc, idx, ws, stream=None):
                                          nbytes, _stream(stream)))
 
 
-def sparse_attn(p: Params, Q, K, V, idx, O, lse, stream=None):
+def _nbytes(ws) -> int:
+    return ws.numel() * ws.element_size() if ws is not None else 0
+
+
+def sparse_attn(p: Params, Q, K, V, idx, O, lse, ws=None, stream=None):
+    """Block-sparse attention; ws (OP_ATTN bytes) enables the packed K/V gather."""
     _check("infllmv2_sparse_attn",
            load().infllmv2_sparse_attn(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx),
-                                       _ptr(O), _ptr(lse), _stream(stream)))
+                                       _ptr(O), _ptr(lse), _ptr(ws), _nbytes(ws),
+                                       _stream(stream)))
 
 
-def dense_attn(p: Params, Q, K, V, O, lse, stream=None):
+def dense_attn(p: Params, Q, K, V, O, lse, ws=None, stream=None):
     _check("infllmv2_dense_attn",
            load().infllmv2_dense_attn(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
-                                      _ptr(lse), _stream(stream)))
+                                      _ptr(lse), _ptr(ws), _nbytes(ws), _stream(stream)))
 
 
 def forward(p: Params, Q, K, V, O, lse, Kc_ws=None, idx_ws=None, ws=None, stream=None) -> int:
@@ -227,7 +233,8 @@ def prefill(Q, K, V, topk=64, n_init=1, n_local=2, threshold=8192, scale=0.0, st
     O = torch.empty_like(Q)
     lse = torch.empty((B, Hq, T), dtype=torch.float32, device=Q.device)
     if T <= threshold:
-        path = forward(p, Q, K, V, O, lse, stream=stream)
+        ws = alloc_workspace(p, OP_FORWARD, Q.device)
+        path = forward(p, Q, K, V, O, lse, ws=ws, stream=stream)
         return O, lse, path, None
     Kc = torch.empty((B, num_compressed(T), Hkv, 2, d), dtype=Q.dtype, device=Q.device)
     idx = torch.empty((B, Hkv, T, topk), dtype=torch.int32, device=Q.device)

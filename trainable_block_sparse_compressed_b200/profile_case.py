@@ -29,11 +29,12 @@ def prefill(name: str, iters: int):
     idx = torch.empty((w.B, w.Hkv, w.T, w.topk), dtype=torch.int32, device="cuda")
     ws = api.alloc_workspace(p, api.OP_SELECT)
     O = torch.empty_like(Q)
+    aws = api.alloc_workspace(p, api.OP_ATTN)
     lse = torch.empty((w.B, w.Hq, w.T), dtype=torch.float32, device="cuda")
     for _ in range(iters):
         api.compress_keys(p, K, Kc)
         api.select_blocks(p, Q, Kc, idx, ws)
-        api.sparse_attn(p, Q, K, V, idx, O, lse)
+        api.sparse_attn(p, Q, K, V, idx, O, lse, aws)
     torch.cuda.synchronize()
     assert api.get_status() == 0
 
