@@ -18,15 +18,17 @@
 // padding.  Persistent CTAs (one per SM) stream the pairs of their items
 // without draining between items.
 //
-// What bounds this kernel is the gather: every pair moves 64 KB from L2 into
-// shared memory through the SM's copy engine, which serves requests in issue
-// order, and S of a pair cannot start before its K has landed.  K and V travel
-// in separate rings (3 x 32 KB each), each filled by its own producer warp:
-// K is released as soon as its S product completes, V after its P V product,
-// so a wait for a V stage never holds back a K request.  The MMA warp runs a
-// non-blocking event loop that issues each P V the moment its P is written.
-// The softmax is split over two warpgroups by heads (heads 0-7 and 8-15 of
-// the same key rows), halving each thread's dependent chain.
+// What bounds this kernel is shared memory: every pair moves 64 KB from L2
+// into shared memory through the SM's copy engine, and the tensor core reads
+// the same 64 KB back as the A operands of S and P V.  K and V of a pair share
+// one 64 KB stage of a 3-stage ring, requested together by one producer and
+// released after the pair's P V.  Two threads issue the MMAs, one the S
+// products and one the P V products, each in pair order with blocking waits:
+// issuing a tcgen05.mma holds its thread for about as long as the tensor core
+// takes to read the operand, and a barrier wait costs a few hundred cycles
+// even when already complete, so one issuer alone could not keep up.  The
+// softmax is split over two warpgroups by heads (heads 0-7 and 8-15 of the
+// same key rows), halving each thread's dependent chain.
 //
 // Softmax (thread = TMEM lane = key row of S^T, = channel d of O^T, for eight
 // heads): each head keeps a reference maximum m that only moves when a score
@@ -46,24 +48,23 @@
 namespace infllmv2 {
 namespace {
 
-constexpr int kKStages = 3;
-constexpr int kVStages = 3;
+constexpr int kStages = 3;                           // K+V ring depth
 constexpr int kHalves = 2;                           // softmax warpgroups, 8 heads each
 constexpr int kHH = 8;                               // heads per warpgroup
 constexpr int kSlotBytes = 64 * 128;                 // 64 rows x 128 B (one TMA box)
 constexpr int kHalf = 2 * kSlotBytes;                // 128 rows x 64 channels
 constexpr int kPairBytes = 2 * kHalf;                // K or V of one pair: 32 KB
+constexpr int kStageBytes = 2 * kPairBytes;          // K then V of one pair: 64 KB
 constexpr int kQBytes = 16 * 256;                    // 16 rows x 128 channels
 constexpr int kPBytes = 16 * 256;                    // 16 heads x 128 keys
 constexpr int kSoftmaxThreads = 128 * kHalves;
-constexpr int kThreads = 96 + kSoftmaxThreads;    // producers K/Q, MMA, producer V, softmax
+constexpr int kThreads = 96 + kSoftmaxThreads;       // producer, S issuer, P V issuer, softmax
 constexpr uint32_t kTmemCols = 64;                   // S^T x2, PV x2 (16 columns each)
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleSlack = 8.0f;                // log2 units
 
 struct AttnSmem {
-  uint64_t k_full[kKStages], k_empty[kKStages];
-  uint64_t v_full[kVStages], v_empty[kVStages];
+  uint64_t full[kStages], empty[kStages];
   uint64_t q_full[2], q_empty[2];
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full[2];
@@ -183,6 +184,7 @@ __device__ __forceinline__ int item_block(const Item& it, int e) {
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, const DevCtx& ctx,
                                               volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;  // the common case: already complete
   if (*abort_flag) return false;
   if (mbar_wait(bar, parity, ctx.wait_ns)) return true;
   report_status(ctx.status, INFLLMV2_STATUS_TIMEOUT);
@@ -198,9 +200,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t* sK = base;                                    // kKStages x 32 KB
-  uint8_t* sV = sK + kKStages * kPairBytes;              // kVStages x 32 KB
-  uint8_t* sQ = sV + kVStages * kPairBytes;              // 2 x 4 KB
+  uint8_t* sKV = base;                                   // kStages x (K 32 KB, V 32 KB)
+  uint8_t* sQ = sKV + kStages * kStageBytes;             // 2 x 4 KB
   uint8_t* sP = sQ + 2 * kQBytes;                        // 2 x 4 KB
   AttnSmem& sm = *reinterpret_cast<AttnSmem*>(sP + 2 * kPBytes);
 
@@ -214,29 +215,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   // second slot stale, and stale data must be finite (it is multiplied by 0)
   {
     uint4* p = reinterpret_cast<uint4*>(base);
-    const int n16 = ((kKStages + kVStages) * kPairBytes + 2 * kQBytes + 2 * kPBytes) / 16;
+    const int n16 = (kStages * kStageBytes + 2 * kQBytes + 2 * kPBytes) / 16;
     for (int i = threadIdx.x; i < n16; i += blockDim.x) p[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
   }
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kKStages; ++s) {
-      mbar_init(&sm.k_full[s], 1);
-      mbar_init(&sm.k_empty[s], 1);
-    }
-    for (int s = 0; s < kVStages; ++s) {
-      mbar_init(&sm.v_full[s], 1);
-      mbar_init(&sm.v_empty[s], 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&sm.q_full[a], 1);
       mbar_init(&sm.q_empty[a], 1);
       mbar_init(&sm.s_full[a], 1);
-      mbar_init(&sm.s_empty[a], kSoftmaxThreads);
-      mbar_init(&sm.p_full[a], kSoftmaxThreads);
+      // softmax-side barriers take one arrival per warp: 256 per-thread
+      // arrivals per barrier per pair cost shared-memory atomic bandwidth
+      // that the copies into the K / V rings need
+      mbar_init(&sm.s_empty[a], kSoftmaxThreads / 32);
+      mbar_init(&sm.p_full[a], kSoftmaxThreads / 32);
       mbar_init(&sm.pv_full[a], 1);
-      mbar_init(&sm.pv_empty[a], kSoftmaxThreads);
+      mbar_init(&sm.pv_empty[a], kSoftmaxThreads / 32);
     }
-    mbar_init(&sm.drain, 1);
+    mbar_init(&sm.drain, 2);  // one commit from each MMA issuer
     sm.abort_flag = 0;
     fence_mbar_init();
   }
@@ -250,8 +250,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort_flag = &sm.abort_flag;
 
-  if (warp == 0 || warp == 2) {
-    // ------------------------------ producers ------------------------------
+  if (warp == 0) {
+    // ------------------------------ producer ------------------------------
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
@@ -262,43 +262,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       int b, g, blk0, blk1;
       bool two;
     };
-    // packed tiles: one 16 KB bulk copy per block, block b of the pair at
+    // K and V of a pair share one stage and one barrier, requested together.
+    // Packed tiles: one 16 KB bulk copy per block, block b of the pair at
     // slot offset 16 KB; otherwise two 64-channel tensor-map boxes per block,
-    // 128-byte swizzled, halves 16 KB apart
-    auto issue = [&](const PairLoad& pl, bool is_v) -> bool {
-      const int nst = is_v ? kVStages : kKStages;
-      const int s = static_cast<int>(pl.gp % nst);
-      uint64_t* full = is_v ? &sm.v_full[s] : &sm.k_full[s];
-      uint64_t* empty = is_v ? &sm.v_empty[s] : &sm.k_empty[s];
-      if (pl.gp >= nst && !wait_or_abort(empty, ((pl.gp / nst) & 1) ^ 1, ctx, abort_flag))
+    // 128-byte swizzled, halves 16 KB apart.
+    auto issue = [&](const PairLoad& pl) -> bool {
+      const int s = static_cast<int>(pl.gp % kStages);
+      uint64_t* full = &sm.full[s];
+      if (pl.gp >= kStages &&
+          !wait_or_abort(&sm.empty[s], ((pl.gp / kStages) & 1) ^ 1, ctx, abort_flag))
         return false;
-      uint8_t* st = (is_v ? sV : sK) + s * kPairBytes;
-      const uint8_t* packed = is_v ? args.Vp : args.Kp;
-      const CUtensorMap* tm = is_v ? &tmV : &tmK;
       const int64_t tile0 = (static_cast<int64_t>(pl.b) * args.Hkv + pl.g) * args.nb;
-      mbar_arrive_expect_tx(full, (pl.two ? 4 : 2) * kSlotBytes);
-      for (int slot = 0; slot < (pl.two ? 2 : 1); ++slot) {
-        const int blk = slot ? pl.blk1 : pl.blk0;
-        if (packed) {
-          bulk_load(st + slot * kHalf, packed + (tile0 + blk) * kHalf, kHalf, full);
-        } else {
-          tma_load_4d(st + slot * kSlotBytes, tm, full, 0, pl.g, blk * kBlock, pl.b);
-          tma_load_4d(st + kHalf + slot * kSlotBytes, tm, full, 64, pl.g, blk * kBlock, pl.b);
+      mbar_arrive_expect_tx(full, (pl.two ? 8 : 4) * kSlotBytes);
+      for (int v = 0; v < 2; ++v) {
+        uint8_t* st = sKV + s * kStageBytes + v * kPairBytes;
+        const uint8_t* packed = v ? args.Vp : args.Kp;
+        const CUtensorMap* tm = v ? &tmV : &tmK;
+        for (int slot = 0; slot < (pl.two ? 2 : 1); ++slot) {
+          const int blk = slot ? pl.blk1 : pl.blk0;
+          if (packed) {
+            bulk_load(st + slot * kHalf, packed + (tile0 + blk) * kHalf, kHalf, full);
+          } else {
+            tma_load_4d(st + slot * kSlotBytes, tm, full, 0, pl.g, blk * kBlock, pl.b);
+            tma_load_4d(st + kHalf + slot * kSlotBytes, tm, full, 64, pl.g, blk * kBlock, pl.b);
+          }
         }
       }
       return true;
     };
-    // warp 0 issues Q and K, warp 2 issues V: a wait for a free V stage (which
-    // frees only after a softmax and a P V product) never holds back the K
-    // that the next S product needs, and the reverse
-    const bool is_v = warp == 2;
-    int64_t gp = 0;       // pairs issued by this warp
+    int64_t gp = 0;       // pairs issued
     int qk = 0;           // Q loads issued
     bool ok = true;
     for (int64_t k = 0, it; ok && (it = item_of(k, n_items)) < n_items; ++k) {
       const Item item = resolve_item(it, args, lane, true);
       if (item.n_pairs == 0) continue;
-      if (!is_v && lane == 0) {
+      if (lane == 0) {
         const int qb = qk & 1;
         if (qk >= 2) ok = wait_or_abort(&sm.q_empty[qb], ((qk >> 1) & 1) ^ 1, ctx, abort_flag);
         if (ok) {
@@ -318,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         pl.blk0 = item_block(item, 2 * p);
         pl.two = 2 * p + 1 < item.n;
         pl.blk1 = pl.two ? item_block(item, 2 * p + 1) : 0;
-        if (lane == 0) ok = issue(pl, is_v);
+        if (lane == 0) ok = issue(pl);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (ok) ++gp;
       }
@@ -326,62 +324,49 @@ __global__ void __launch_bounds__(kThreads, 1)
     // drain: never leave with copies of this CTA in flight (matters only when
     // a wait above gave up; otherwise these phases completed long ago)
     if (lane == 0) {
-      if (!is_v) {
-        for (int x = 0; x < 2 && x < qk; ++x)
-          mbar_wait(&sm.q_full[x], ((qk - 1 - x) >> 1) & 1, ctx.wait_ns);
-        for (int x = 0; x < kKStages && x < gp; ++x)
-          mbar_wait(&sm.k_full[x], ((gp - 1 - x) / kKStages) & 1, ctx.wait_ns);
-      } else {
-        for (int x = 0; x < kVStages && x < gp; ++x)
-          mbar_wait(&sm.v_full[x], ((gp - 1 - x) / kVStages) & 1, ctx.wait_ns);
-      }
+      for (int x = 0; x < 2 && x < qk; ++x)
+        mbar_wait(&sm.q_full[x], ((qk - 1 - x) >> 1) & 1, ctx.wait_ns);
+      for (int64_t q = gp - 1; q >= 0 && q >= gp - kStages; --q)
+        mbar_wait(&sm.full[q % kStages], (q / kStages) & 1, ctx.wait_ns);
     }
-  } else if (warp == 1) {
-    // ------------------------------ MMA issuer ------------------------------
-    // Lane 0 alone runs a non-blocking event loop: it issues every P V whose
-    // P, V stage and TMEM buffer are ready (in pair order), and the next S^T
-    // when its K stage, Q and S buffer are ready.  It gives up when nothing
-    // has been issued for the wait limit.
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = instr_desc_bf16(128, 16, 0, 0);
-      constexpr uint32_t idesc_pv = instr_desc_bf16(128, 16, 1, 1);
-      int64_t k_item = 0;
-      Item item;
-      item.n_pairs = 0;
-      int p = 0;
-      auto next_item = [&]() {
-        for (int64_t it; (it = item_of(k_item, n_items)) < n_items;) {
-          ++k_item;
-          item = resolve_item(it, args, 0, false);
-          if (item.n_pairs > 0) {
-            p = 0;
-            return true;
-          }
-        }
-        return false;
-      };
-      bool have = next_item();
-      int64_t gp_s = 0;   // S products issued
-      int64_t gp_pv = 0;  // P V products issued
-      int qk = 0;         // items whose Q has been consumed
-      uint64_t t_progress = global_timer_ns();
-      while (true) {
-        bool did = false;
-        // P V products, in order, as soon as P, V and the TMEM buffer are ready
-        while (gp_pv < gp_s) {
-          const int a = static_cast<int>(gp_pv & 1);
-          const int vs = static_cast<int>(gp_pv % kVStages);
-          if (!mbar_test(&sm.p_full[a], (gp_pv >> 1) & 1)) break;
-          if (gp_pv >= 2 && !mbar_test(&sm.pv_empty[a], ((gp_pv >> 1) & 1) ^ 1)) break;
-          if (!mbar_test(&sm.v_full[vs], (gp_pv / kVStages) & 1)) break;
+  } else if (warp == 1 || warp == 2) {
+    // ----------------------------- MMA issuers -----------------------------
+    // Issuing a tcgen05.mma holds the issuing thread for about as long as the
+    // tensor core takes to read its operand (~70 cycles for 128 x 16 bf16),
+    // and a wait on an mbarrier, even one already complete, costs the thread
+    // a few hundred cycles.  One thread doing both for S and P V would spend
+    // a pair's whole budget, so warp 1 issues the S products and warp 2 the
+    // P V products; each one's waits overlap the other's MMAs.  No order
+    // between the two streams is needed: S(p) and P V(p-1) touch disjoint
+    // TMEM and shared memory, a stage is refilled only after its P V (which
+    // follows its S through the softmax), and the softmax folds P V(p) before
+    // it overwrites P(p) with P(p+2).  Each warp resolves items together;
+    // lane 0 waits and issues.
+    const bool pv_role = warp == 2;
+    constexpr uint32_t idesc_s = instr_desc_bf16(128, 16, 0, 0);
+    constexpr uint32_t idesc_pv = instr_desc_bf16(128, 16, 1, 1);
+    int64_t gp = 0;  // pairs issued by this warp
+    int qk = 0;      // items whose Q has been used (S issuer)
+    bool ok = true;
+    for (int64_t k = 0, it; ok && (it = item_of(k, n_items)) < n_items; ++k) {
+      const Item item = resolve_item(it, args, lane, true);
+      if (item.n_pairs == 0) continue;
+      if (lane == 0 && pv_role) {
+        for (int p = 0; ok && p < item.n_pairs; ++p, ++gp) {
+          const int a = static_cast<int>(gp & 1);
+          const int st = static_cast<int>(gp % kStages);
+          ok = wait_or_abort(&sm.p_full[a], (gp >> 1) & 1, ctx, abort_flag) &&
+               wait_or_abort(&sm.full[st], (gp / kStages) & 1, ctx, abort_flag) &&
+               (gp < 2 || wait_or_abort(&sm.pv_empty[a], ((gp >> 1) & 1) ^ 1, ctx, abort_flag));
+          if (!ok) break;
           tc_fence_after();
-          const uint32_t v_addr = smem_u32(sV + vs * kPairBytes);
+          const uint32_t v_addr = smem_u32(sKV + st * kStageBytes + kPairBytes);
           const uint32_t p_addr = smem_u32(sP + a * kPBytes);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            // A: V^T, MN-major 128-byte swizzle: 16 keys = two 8-row groups (2 KB)
-            // (packed tiles: MN-major, no swizzle, channel groups 128 B apart
-            // (SBO), 8-key groups 2 KB apart (LBO), 16 keys = 4 KB)
+            // A: V^T, MN-major.  Packed tiles: no swizzle, channel groups 128 B
+            // apart (SBO), 8-key groups 2 KB apart (LBO), 16 keys = 4 KB.
+            // Boxes: 128-byte swizzle, 16 keys = two 8-row groups (2 KB).
             const uint64_t ad = args.Vp ? smem_desc(v_addr + kk * 4096, 2048, 128, 0)
                                         : smem_desc(v_addr + kk * 2048, kHalf, 1024, 2);
             // B: P^T, MN-major, no swizzle: 8x8 core matrices of 128 B, heads
@@ -390,61 +375,40 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_bf16(tmem + 32 + a * 16, ad, bd, idesc_pv, kk > 0 ? 1u : 0u);
           }
           umma_commit(&sm.pv_full[a]);
-          umma_commit(&sm.v_empty[vs]);
-          ++gp_pv;
-          did = true;
+          umma_commit(&sm.empty[st]);
         }
-        // the next S^T product
-        if (have) {
-          const int qb = qk & 1;
-          const int ks = static_cast<int>(gp_s % kKStages);
-          const int a = static_cast<int>(gp_s & 1);
-          bool ready = gp_s - gp_pv < 2;
-          if (ready && p == 0) ready = mbar_test(&sm.q_full[qb], (qk >> 1) & 1);
-          if (ready) ready = mbar_test(&sm.k_full[ks], (gp_s / kKStages) & 1);
-          if (ready && gp_s >= 2) ready = mbar_test(&sm.s_empty[a], ((gp_s >> 1) & 1) ^ 1);
-          if (ready) {
-            tc_fence_after();
-            const uint32_t k_addr = smem_u32(sK + ks * kPairBytes);
-            const uint32_t q_addr = smem_u32(sQ + qb * kQBytes);
+      } else if (lane == 0) {
+        const int qb = qk & 1;
+        ok = wait_or_abort(&sm.q_full[qb], (qk >> 1) & 1, ctx, abort_flag);
+        const uint32_t q_addr = smem_u32(sQ + qb * kQBytes);
+        for (int p = 0; ok && p < item.n_pairs; ++p, ++gp) {
+          const int st = static_cast<int>(gp % kStages);
+          const int a = static_cast<int>(gp & 1);
+          ok = wait_or_abort(&sm.full[st], (gp / kStages) & 1, ctx, abort_flag) &&
+               (gp < 2 || wait_or_abort(&sm.s_empty[a], ((gp >> 1) & 1) ^ 1, ctx, abort_flag));
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(sKV + st * kStageBytes);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              // packed tiles: K-major, no swizzle, 16 channels = two 128 B
-              // core-matrix columns (LBO), 8-row groups 2 KB apart (SBO);
-              // boxes: K-major 128-byte swizzle, 64-channel halves 16 KB apart
-              const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-              const uint64_t ad = args.Kp ? smem_desc(k_addr + kk * 256, 128, 2048, 0)
-                                          : smem_desc(k_addr + off, 16, 1024, 2);
-              const uint64_t bd =
-                  smem_desc(q_addr + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024, 2);
-              umma_bf16(tmem + a * 16, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
-            }
-            umma_commit(&sm.s_full[a]);
-            umma_commit(&sm.k_empty[ks]);
-            ++gp_s;
-            if (++p == item.n_pairs) {
-              umma_commit(&sm.q_empty[qb]);
-              ++qk;
-              have = next_item();
-            }
-            did = true;
+          for (int kk = 0; kk < 8; ++kk) {
+            // packed tiles: K-major, no swizzle, 16 channels = two 128 B
+            // core-matrix columns (LBO), 8-row groups 2 KB apart (SBO);
+            // boxes: K-major 128-byte swizzle, 64-channel halves 16 KB apart
+            const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+            const uint64_t ad = args.Kp ? smem_desc(k_addr + kk * 256, 128, 2048, 0)
+                                        : smem_desc(k_addr + off, 16, 1024, 2);
+            const uint64_t bd = smem_desc(q_addr + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024, 2);
+            umma_bf16(tmem + a * 16, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
           }
-        } else if (gp_pv == gp_s) {
-          break;
+          umma_commit(&sm.s_full[a]);
+          if (p + 1 == item.n_pairs) umma_commit(&sm.q_empty[qb]);
         }
-        if (did) {
-          t_progress = global_timer_ns();
-        } else if (!*abort_flag && global_timer_ns() - t_progress <= ctx.wait_ns) {
-          // idle: back off so that polling does not contend with the copy
-          // engine's and the other warps' updates of the same barriers
-          __nanosleep(64);
-        } else {
-          if (!*abort_flag) report_status(ctx.status, INFLLMV2_STATUS_TIMEOUT);
-          *abort_flag = 1;
-          break;
-        }
+        ++qk;
       }
-      // drain: all MMAs of this CTA complete before TMEM is released
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+    }
+    if (lane == 0) {
+      // drain: all MMAs of this thread complete before TMEM is released
       umma_commit(&sm.drain);
       mbar_wait(&sm.drain, 0, ctx.wait_ns);
     }
@@ -496,7 +460,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld8(lane_addr + a * 16, x);
           tmem_ld_wait();
           tc_fence_before();
-          mbar_arrive(&sm.s_empty[a]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.s_empty[a]);
           const int e = 2 * p + slot;
           const int blk = e < item.n ? (item.row ? sm.blocks[e] : item.e0 + e) : -1;
           const bool valid = blk >= 0 && blk * kBlock + krow <= item.t;
@@ -550,7 +515,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           *reinterpret_cast<uint4*>(sP + a * kPBytes + p_off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           fence_proxy_async_smem();
-          mbar_arrive(&sm.p_full[a]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.p_full[a]);
         }
         if (p > 0) {
           // fold in P V of the previous pair
@@ -565,7 +531,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld8(lane_addr + 32 + a * 16, pv);
           tmem_ld_wait();
           tc_fence_before();
-          mbar_arrive(&sm.pv_empty[a]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.pv_empty[a]);
 #pragma unroll
           for (int h = 0; h < kHH; ++h) o[h] = o[h] * alpha_prev[h] + pv[h];
         }
@@ -644,7 +611,7 @@ template <int G>
 int launch_attn_g(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                   const AttnArgs& args, int64_t n_items, const DevCtx& ctx, cudaStream_t st) {
   const size_t smem =
-      1024 + (kKStages + kVStages) * kPairBytes + 2 * kQBytes + 2 * kPBytes + sizeof(AttnSmem);
+      1024 + kStages * kStageBytes + 2 * kQBytes + 2 * kPBytes + sizeof(AttnSmem);
   static bool configured = false;
   if (!configured) {
     if (cudaFuncSetAttribute(sparse_attn_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
