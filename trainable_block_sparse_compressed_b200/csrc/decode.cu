@@ -12,12 +12,15 @@
 //                    windows, split over many CTAs (HBM-bound stream of the
 //                    compressed-key cache), plus each split's per-head max and
 //                    sum of exp2 for the softmax;
-//   3. select      : per (sequence, kv head): merge the splits into each
-//                    head's log-sum-exp, group-sum the probabilities, max-pool
-//                    onto 64-token blocks, warp top-k with the forced blocks;
+//   3. select      : per (sequence, kv head), split over CTAs of 128 blocks
+//                    each: merge the splits into each head's log-sum-exp,
+//                    group-sum the probabilities, max-pool onto 64-token
+//                    blocks; the last CTA of the row runs the warp top-k with
+//                    the forced blocks;
 //   4. attention   : sparse_attn.cu in decode mode, the selected blocks split
 //                    into chunks, unnormalised partials;
-//   5. combine     : merge the chunk partials into O and LSE; seqlens += 1.
+//   5. combine     : merge the chunk partials into O and LSE (one CTA per
+//                    head); seqlens += 1.
 #include "common.cuh"
 #include "sm100.cuh"
 #include "topk.cuh"
@@ -34,9 +37,11 @@ constexpr int kScoreRows = 512;     // compressed rows per scoring CTA
 constexpr int kChunkBlocks = 8;     // selected blocks per attention item
 constexpr float kLn2 = 0.6931471805599453f;
 
+constexpr int kPoolBlocks = 128;    // blocks max-pooled per pooling CTA
+
 struct DecodeLayout {
-  int NC, NB, n_split, n_chunks;
-  size_t off_active, off_x, off_ml, off_idx, off_part, total;
+  int NC, NB, n_split, n_chunks, n_pool;
+  size_t off_active, off_x, off_ml, off_idx, off_part, off_bs, off_cnt, total;
 };
 
 DecodeLayout decode_layout(const Geometry& g) {
@@ -45,6 +50,7 @@ DecodeLayout decode_layout(const Geometry& g) {
   L.NB = g.T > 0 ? (g.T - 1) / kBlock + 1 : 0;
   L.n_split = L.NC > 0 ? (L.NC + kScoreRows - 1) / kScoreRows : 1;
   L.n_chunks = (g.topk + kChunkBlocks - 1) / kChunkBlocks;
+  L.n_pool = L.NB > 0 ? (L.NB + kPoolBlocks - 1) / kPoolBlocks : 1;
   auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   const size_t bg = static_cast<size_t>(g.B) * g.Hkv;
   size_t o = 0;
@@ -58,6 +64,10 @@ DecodeLayout decode_layout(const Geometry& g) {
   o = up(o + bg * g.topk * sizeof(int32_t));
   L.off_part = o;
   o = up(o + bg * L.n_chunks * g.G * (kHeadDim + 2) * sizeof(float));
+  L.off_bs = o;
+  o = up(o + bg * static_cast<size_t>(L.NB) * sizeof(float));
+  L.off_cnt = o;
+  o = up(o + bg * sizeof(uint32_t));
   L.total = o;
   return L;
 }
@@ -67,9 +77,11 @@ __global__ void __launch_bounds__(32) decode_append_kernel(
     const __nv_bfloat16* __restrict__ k_new, const __nv_bfloat16* __restrict__ v_new,
     __nv_bfloat16* __restrict__ Kc_, __nv_bfloat16* __restrict__ Vc_,
     __nv_bfloat16* __restrict__ Kcmp, const int32_t* __restrict__ seqlens,
-    int32_t* __restrict__ active, int Hkv, int Lmax, int NC, int* status) {
+    int32_t* __restrict__ active, uint32_t* __restrict__ pool_count, int Hkv, int Lmax, int NC,
+    int* status) {
   const int b = blockIdx.x / Hkv, g = blockIdx.x % Hkv;
   const int tid = threadIdx.x;
+  if (tid == 0) pool_count[blockIdx.x] = 0;  // arrivals of this step's pooling CTAs
   const int pos = seqlens[b];
   const bool act = pos >= 0 && pos < Lmax;
   if (g == 0 && tid == 0) {
@@ -193,86 +205,126 @@ __global__ void __launch_bounds__(256) decode_score_kernel(
 }
 
 // ---- 3. select ---------------------------------------------------------------
-template <int G, int VPL>
+// Pooling CTA (bg, part) owns blocks [part*128, part*128 + 128) of row bg:
+// merges the score splits into each head's log2-sum-exp, sums the G heads'
+// probabilities over the windows overlapping its blocks, max-pools them, and
+// writes the block scores.  The last CTA of the row to finish (an arrival
+// counter that the append kernel zeroed) runs the CTA top-k over the row,
+// PER blocks per thread.
+template <int G, int PER>
 __global__ void __launch_bounds__(256) decode_select_kernel(
     const float* __restrict__ x, const float* __restrict__ ml, const int32_t* __restrict__ seqlens,
-    int32_t* __restrict__ idx, int Hkv, int NC, int Lmax, int n_split, int topk, int n_init,
-    int n_local) {
-  extern __shared__ float sbuf[];  // S[NC] then bs[NB]
+    float* bs_all, uint32_t* pool_count, int32_t* __restrict__ idx, int Hkv, int NC, int NB,
+    int Lmax, int n_split, int n_pool, int topk, int n_init, int n_local) {
+  constexpr int kWin = 4 * kPoolBlocks + 4;  // windows 4*blk0-1 .. 4*blk1+3 (clipped)
+  __shared__ float S[kWin];
   __shared__ float lse2[G];
-  const int bg = blockIdx.x;
+  __shared__ bool last;
+  const int bg = blockIdx.x / n_pool;
+  const int part = blockIdx.x % n_pool;
   const int b = bg / Hkv;
   const int t = seqlens[b];
   int32_t* orow = idx + static_cast<int64_t>(bg) * topk;
   if (!(t >= 0 && t < Lmax)) {
-    for (int k = threadIdx.x; k < topk; k += blockDim.x) orow[k] = -1;
+    if (part == 0)
+      for (int k = threadIdx.x; k < topk; k += blockDim.x) orow[k] = -1;
     return;
   }
   const int v = min(NC, visible_windows(t));
   const int cur = t / kBlock;
-  float* S = sbuf;
-  float* bs = sbuf + NC;
-  if (threadIdx.x < G) {
-    const int h = threadIdx.x;
-    const float* p = ml + static_cast<int64_t>(bg) * n_split * G * 2;
-    float M = -INFINITY;
-    for (int s = 0; s < n_split; ++s) M = fmaxf(M, p[s * G * 2 + 2 * h]);
-    float L = 0.f;
-    if (M > -INFINITY)
-      for (int s = 0; s < n_split; ++s) L += p[s * G * 2 + 2 * h + 1] * fast_exp2(p[s * G * 2 + 2 * h] - M);
-    lse2[h] = M > -INFINITY ? M + __log2f(L) : INFINITY;
-  }
-  __syncthreads();
-  for (int j = threadIdx.x; j < v; j += blockDim.x) {
-    const float* xr = x + (static_cast<int64_t>(bg) * NC + j) * G;
-    float acc = 0.f;
+  const int blk0 = part * kPoolBlocks;
+  const int blk1 = min(cur + 1, blk0 + kPoolBlocks);
+  float* bs = bs_all + static_cast<int64_t>(bg) * NB;
+  if (blk0 < blk1) {
+    if (threadIdx.x < G) {
+      const int h = threadIdx.x;
+      const float* p = ml + static_cast<int64_t>(bg) * n_split * G * 2;
+      float M = -INFINITY;
+      for (int s2 = 0; s2 < n_split; ++s2) M = fmaxf(M, p[s2 * G * 2 + 2 * h]);
+      float L = 0.f;
+      if (M > -INFINITY)
+        for (int s2 = 0; s2 < n_split; ++s2)
+          L += p[s2 * G * 2 + 2 * h + 1] * fast_exp2(p[s2 * G * 2 + 2 * h] - M);
+      lse2[h] = M > -INFINITY ? M + __log2f(L) : INFINITY;
+    }
+    __syncthreads();
+    const int j0 = max(0, 4 * blk0 - 1);
+    const int j1 = min(v, 4 * blk1 + 3);  // exclusive
+    for (int j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
+      const float4* xr = reinterpret_cast<const float4*>(x + (static_cast<int64_t>(bg) * NC + j) * G);
+      float acc = 0.f;
+      if constexpr (G % 4 == 0) {
 #pragma unroll
-    for (int h = 0; h < G; ++h) acc += fast_exp2(xr[h] - lse2[h]);
-    S[j] = acc;
+        for (int h4 = 0; h4 < G / 4; ++h4) {
+          const float4 u = __ldg(xr + h4);
+          acc += fast_exp2(u.x - lse2[4 * h4]) + fast_exp2(u.y - lse2[4 * h4 + 1]) +
+                 fast_exp2(u.z - lse2[4 * h4 + 2]) + fast_exp2(u.w - lse2[4 * h4 + 3]);
+        }
+      } else {
+        const float* xs = x + (static_cast<int64_t>(bg) * NC + j) * G;
+#pragma unroll
+        for (int h = 0; h < G; ++h) acc += fast_exp2(__ldg(xs + h) - lse2[h]);
+      }
+      S[j - j0] = acc;
+    }
+    __syncthreads();
+    for (int blk = blk0 + threadIdx.x; blk < blk1; blk += blockDim.x) {
+      const int j_lo = max(0, 4 * blk - 1), j_hi = min(v - 1, 4 * blk + 3);
+      float mx = -INFINITY;
+      for (int j = j_lo; j <= j_hi; ++j) mx = fmaxf(mx, S[j - j0]);
+      bs[blk] = mx;
+    }
   }
+  // the last pooling CTA of the row selects
+  __threadfence();
   __syncthreads();
-  for (int blk = threadIdx.x; blk <= cur; blk += blockDim.x) {
-    const int j_lo = max(0, 4 * blk - 1), j_hi = min(v - 1, 4 * blk + 3);
-    float mx = -INFINITY;
-    for (int j = j_lo; j <= j_hi; ++j) mx = fmaxf(mx, S[j]);
-    bs[blk] = mx;
-  }
+  if (threadIdx.x == 0) last = atomicAdd(pool_count + bg, 1u) == static_cast<uint32_t>(n_pool - 1);
   __syncthreads();
-  if (threadIdx.x < 32) warp_select_row<VPL>(bs, cur, topk, n_init, n_local, orow);
+  if (!last) return;
+  __threadfence();
+  cta_select_row<256, PER>(bs, cur, topk, n_init, n_local, orow);
+}
+
+// Blocks per thread of the 256-thread CTA top-k for rows of up to nb blocks
+// (0 if too many).
+inline int select_per(int nb) {
+  for (int per = 1; per <= 32; per *= 2)
+    if (256 * per >= nb) return per;
+  return 0;
 }
 
 // ---- 5. combine --------------------------------------------------------------
+// One CTA per (sequence, kv head, head), one thread per channel.
 template <int G>
 __global__ void __launch_bounds__(128) decode_combine_kernel(
     const float* __restrict__ part, const int32_t* __restrict__ active, int32_t* seqlens,
     __nv_bfloat16* __restrict__ O, float* __restrict__ lse, int Hq, int Hkv, int n_chunks,
     int64_t n_items) {
-  const int bg = blockIdx.x;
+  const int bg = blockIdx.x / G, h = blockIdx.x % G;
   const int b = bg / Hkv, g = bg % Hkv;
   const int d = threadIdx.x;
   const bool act = active[b] != 0;
   const float* po = part;
   const float* pml = part + n_items * (G * kHeadDim);
-  for (int h = 0; h < G; ++h) {
-    float M = -INFINITY;
-    for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, pml[(static_cast<int64_t>(bg) * n_chunks + c) * 2 * G + 2 * h]);
-    float acc = 0.f, wsum = 0.f;
-    if (act && M > -INFINITY) {
-      for (int c = 0; c < n_chunks; ++c) {
-        const int64_t itm = static_cast<int64_t>(bg) * n_chunks + c;
-        const float mc = pml[itm * 2 * G + 2 * h];
-        if (mc == -INFINITY) continue;
-        const float w = fast_exp2(mc - M);
-        acc += w * po[itm * G * kHeadDim + h * kHeadDim + d];
-        wsum += w * pml[itm * 2 * G + 2 * h + 1];
-      }
+  float M = -INFINITY;
+  for (int c = 0; c < n_chunks; ++c)
+    M = fmaxf(M, pml[(static_cast<int64_t>(bg) * n_chunks + c) * 2 * G + 2 * h]);
+  float acc = 0.f, wsum = 0.f;
+  if (act && M > -INFINITY) {
+    for (int c = 0; c < n_chunks; ++c) {
+      const int64_t itm = static_cast<int64_t>(bg) * n_chunks + c;
+      const float mc = pml[itm * 2 * G + 2 * h];
+      if (mc == -INFINITY) continue;
+      const float w = fast_exp2(mc - M);
+      acc += w * po[itm * G * kHeadDim + h * kHeadDim + d];
+      wsum += w * pml[itm * 2 * G + 2 * h + 1];
     }
-    const bool ok = act && wsum > 0.f;
-    O[(static_cast<int64_t>(b) * Hq + g * G + h) * kHeadDim + d] =
-        __float2bfloat16_rn(ok ? acc / wsum : 0.f);
-    if (d == 0) lse[static_cast<int64_t>(b) * Hq + g * G + h] = ok ? (M + __log2f(wsum)) * kLn2 : 0.f;
   }
-  if (g == 0 && d == 0 && act) seqlens[b] += 1;
+  const bool ok = act && wsum > 0.f;
+  O[(static_cast<int64_t>(b) * Hq + g * G + h) * kHeadDim + d] =
+      __float2bfloat16_rn(ok ? acc / wsum : 0.f);
+  if (d == 0) lse[static_cast<int64_t>(b) * Hq + g * G + h] = ok ? (M + __log2f(wsum)) * kLn2 : 0.f;
+  if (g == 0 && h == 0 && d == 0 && act) seqlens[b] += 1;
 }
 
 template <int G>
@@ -283,33 +335,31 @@ int launch_decode_g(const Geometry& g, const DecodeLayout& L, const void* q, con
   float* x = reinterpret_cast<float*>(ws + L.off_x);
   float* ml = reinterpret_cast<float*>(ws + L.off_ml);
   float* part = reinterpret_cast<float*>(ws + L.off_part);
+  float* bs = reinterpret_cast<float*>(ws + L.off_bs);
+  uint32_t* pool_count = reinterpret_cast<uint32_t*>(ws + L.off_cnt);
   const int bgn = g.B * g.Hkv;
   decode_append_kernel<<<bgn, 32, 0, st>>>(
       static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new),
       static_cast<__nv_bfloat16*>(Kc_), static_cast<__nv_bfloat16*>(Vc_),
-      static_cast<__nv_bfloat16*>(Kcmp), seqlens, active, g.Hkv, g.T, L.NC, ctx.status);
+      static_cast<__nv_bfloat16*>(Kcmp), seqlens, active, pool_count, g.Hkv, g.T, L.NC,
+      ctx.status);
   if (cudaGetLastError() != cudaSuccess) return INFLLMV2_ERR_CUDA;
   decode_score_kernel<G><<<bgn * L.n_split, 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(Kcmp), seqlens, x, ml,
       g.Hq, g.Hkv, L.NC, g.T, L.n_split, g.scale_log2);
   if (cudaGetLastError() != cudaSuccess) return INFLLMV2_ERR_CUDA;
-  const size_t sel_smem = static_cast<size_t>(L.NC + L.NB) * sizeof(float);
-  const int vpl = topk_vpl(L.NB);
-#define INFLLMV2_SEL(V)                                                                     \
-  do {                                                                                      \
-    if (cudaFuncSetAttribute(decode_select_kernel<G, V>,                                    \
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,                   \
-                             static_cast<int>(sel_smem)) != cudaSuccess)                    \
-      return INFLLMV2_ERR_CUDA;                                                             \
-    decode_select_kernel<G, V><<<bgn, 256, sel_smem, st>>>(x, ml, seqlens, idx, g.Hkv, L.NC, \
-                                                            g.T, L.n_split, g.topk, g.n_init, \
-                                                            g.n_local);                      \
-  } while (0)
-  switch (vpl) {
+  const int per = select_per(L.NB);
+#define INFLLMV2_SEL(V)                                                                        \
+  decode_select_kernel<G, V><<<bgn * L.n_pool, 256, 0, st>>>(                                  \
+      x, ml, seqlens, bs, pool_count, idx, g.Hkv, L.NC, L.NB, g.T, L.n_split, L.n_pool, g.topk, \
+      g.n_init, g.n_local)
+  switch (per) {
+    case 1: INFLLMV2_SEL(1); break;
+    case 2: INFLLMV2_SEL(2); break;
     case 4: INFLLMV2_SEL(4); break;
+    case 8: INFLLMV2_SEL(8); break;
     case 16: INFLLMV2_SEL(16); break;
-    case 64: INFLLMV2_SEL(64); break;
-    case 128: INFLLMV2_SEL(128); break;
+    case 32: INFLLMV2_SEL(32); break;
     default: return INFLLMV2_ERR_UNSUPPORTED;
   }
 #undef INFLLMV2_SEL
@@ -318,7 +368,7 @@ int launch_decode_g(const Geometry& g, const DecodeLayout& L, const void* q, con
                                  st))
     return e;
   const int64_t n_items = static_cast<int64_t>(bgn) * L.n_chunks;
-  decode_combine_kernel<G><<<bgn, 128, 0, st>>>(part, active, seqlens,
+  decode_combine_kernel<G><<<bgn * G, 128, 0, st>>>(part, active, seqlens,
                                                 static_cast<__nv_bfloat16*>(O), lse, g.Hq, g.Hkv,
                                                 L.n_chunks, n_items);
   return cudaGetLastError() == cudaSuccess ? INFLLMV2_OK : INFLLMV2_ERR_CUDA;
@@ -333,8 +383,7 @@ int launch_decode_step(const Geometry& g, const void* q, const void* k_new, cons
                        float* lse, int32_t* idx_out, void* ws, const DevCtx& ctx,
                        cudaStream_t st) {
   const DecodeLayout L = decode_layout(g);
-  if (topk_vpl(L.NB) == 0) return INFLLMV2_ERR_UNSUPPORTED;
-  if (static_cast<size_t>(L.NC + L.NB) * sizeof(float) > 200 * 1024) return INFLLMV2_ERR_UNSUPPORTED;
+  if (select_per(L.NB) == 0) return INFLLMV2_ERR_UNSUPPORTED;
   uint8_t* w = static_cast<uint8_t*>(ws);
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(w + L.off_idx);
   switch (g.G) {

@@ -170,10 +170,14 @@ __device__ __forceinline__ Item resolve_item(int64_t it, const AttnArgs& a, int 
 // CTAs process at the same time are then far apart, so they do not all fetch
 // the same local blocks from the same L2 lines at once, as they would if
 // consecutive tokens went to consecutive CTAs.
+// With few items (decode) the chunks shrink to single items so that every
+// CTA gets work.
 constexpr int kChunkItems = 16;
 __device__ __forceinline__ int64_t item_of(int64_t k, int64_t n_items) {
-  const int64_t chunk = k / kChunkItems;
-  const int64_t it = (chunk * gridDim.x + blockIdx.x) * kChunkItems + k % kChunkItems;
+  const int64_t per_cta = n_items / gridDim.x;
+  const int64_t c = per_cta >= kChunkItems ? kChunkItems : (per_cta > 1 ? per_cta : 1);
+  const int64_t chunk = k / c;
+  const int64_t it = (chunk * gridDim.x + blockIdx.x) * c + k % c;
   return it < n_items ? it : n_items;
 }
 

@@ -85,6 +85,147 @@ __device__ __forceinline__ void warp_select_row(const float* srow, int cur, int 
   for (int k = written + lane; k < topk; k += 32) orow[k] = -1;
 }
 
+// Exclusive prefix sum of one int per thread over a CTA of NT threads (NT a
+// multiple of 32, at most 1024); returns the thread's offset and, in *total,
+// the CTA sum.  `scratch` holds NT / 32 + 1 ints of shared memory.  All
+// threads must call.
+template <int NT>
+__device__ __forceinline__ int cta_exclusive_scan(int v, int* scratch, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) scratch[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < NT / 32 ? scratch[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < NT / 32) scratch[lane] = w;  // inclusive warp totals
+    if (lane == NT / 32 - 1) scratch[NT / 32] = w;
+  }
+  __syncthreads();
+  const int off = (warp > 0 ? scratch[warp - 1] : 0) + x - v;
+  *total = scratch[NT / 32];
+  __syncthreads();  // scratch is reused by the next call
+  return off;
+}
+
+// The same selection as warp_select_row, by a whole CTA of NT threads: thread
+// i holds blocks i*PER .. i*PER+PER-1 (rows of up to NT*PER blocks).  The
+// free_slots-th largest candidate key tau is found by a radix select over
+// four 8-bit digits, most significant first (a 256-bin histogram per digit).
+// Keys above tau are kept; among keys equal to tau the lowest block indices
+// fill the remaining slots (a prefix sum over threads in index order); a
+// second prefix sum places the kept blocks in ascending order.  All threads
+// must call.
+template <int NT, int PER>
+__device__ __forceinline__ void cta_select_row(const float* srow, int cur, int topk, int n_init,
+                                               int n_local, int32_t* orow) {
+  __shared__ int hist[256];
+  __shared__ int scan_buf[NT / 32 + 1];
+  __shared__ int pick[2];  // digit, count of keys above it
+  const int nb = cur + 1;
+  auto forced = [&](int i) { return i < n_init || i > cur - n_local; };
+  const int a = min(n_init, nb);
+  const int lo = max(0, cur - n_local + 1);
+  const int n_forced = a + (nb - lo) - max(0, a - lo);
+  const int free_slots = topk - n_forced;
+  const int n_cand = nb - n_forced;
+  const int base = threadIdx.x * PER;
+
+  uint32_t key[PER];
+#pragma unroll
+  for (int s = 0; s < PER; ++s) {
+    const int i = base + s;
+    key[s] = (i < nb && !forced(i)) ? order_key(srow[i]) : 0u;
+  }
+  const bool take_all = free_slots >= n_cand;
+  uint32_t tau = 0;
+  int need_eq = 0;
+  if (!take_all) {
+    uint32_t prefix = 0, mask = 0;
+    int k = free_slots;  // rank of tau among the keys that match prefix
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int d = threadIdx.x; d < 256; d += NT) hist[d] = 0;
+      __syncthreads();
+#pragma unroll
+      for (int s = 0; s < PER; ++s)
+        if (key[s] != 0u && (key[s] & mask) == prefix) atomicAdd(&hist[(key[s] >> shift) & 255], 1);
+      __syncthreads();
+      if (threadIdx.x < 32) {
+        // suffix sums over the 256 digits, 8 per lane, lane 31 holding the top
+        const int lane = threadIdx.x;
+        int c[8], sum = 0;
+#pragma unroll
+        for (int u = 7; u >= 0; --u) {
+          c[u] = hist[lane * 8 + u];
+          sum += c[u];
+        }
+        int above = sum;  // keys with digits in lanes >= this lane
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_down_sync(0xffffffffu, above, o);
+          if (lane + o < 32) above += y;
+        }
+        int higher = above - sum;  // keys with digits in lanes above this lane
+        int dsel = -1, hsel = 0;
+#pragma unroll
+        for (int u = 7; u >= 0; --u) {
+          if (dsel < 0 && higher < k && higher + c[u] >= k) {
+            dsel = lane * 8 + u;
+            hsel = higher;
+          }
+          higher += c[u];
+        }
+        if (dsel >= 0) {
+          pick[0] = dsel;
+          pick[1] = hsel;
+        }
+      }
+      __syncthreads();
+      const int dsel = pick[0];
+      k -= pick[1];
+      prefix |= static_cast<uint32_t>(dsel) << shift;
+      mask |= 255u << shift;
+      __syncthreads();
+    }
+    tau = prefix;
+    need_eq = k;
+  }
+  // keys equal to tau, ranked by block index
+  int n_eq = 0;
+#pragma unroll
+  for (int s = 0; s < PER; ++s)
+    n_eq += (!take_all && base + s < nb && key[s] != 0u && key[s] == tau) ? 1 : 0;
+  int tot;
+  int eq_rank = cta_exclusive_scan<NT>(n_eq, scan_buf, &tot);
+  bool keep[PER];
+  int n_keep = 0;
+#pragma unroll
+  for (int s = 0; s < PER; ++s) {
+    const int i = base + s;
+    const bool valid = i < nb;
+    const bool is_forced = valid && forced(i);
+    bool kp = is_forced || (valid && (take_all || key[s] > tau));
+    if (valid && !is_forced && !take_all && key[s] == tau) kp = eq_rank++ < need_eq;
+    keep[s] = kp;
+    n_keep += kp ? 1 : 0;
+  }
+  int written;
+  int pos = cta_exclusive_scan<NT>(n_keep, scan_buf, &written);
+#pragma unroll
+  for (int s = 0; s < PER; ++s)
+    if (keep[s]) orow[pos++] = base + s;
+  for (int k2 = written + threadIdx.x; k2 < topk; k2 += NT) orow[k2] = -1;
+}
+
 // Values per lane needed for rows of up to nb_max blocks (0 if too many).
 inline int topk_vpl(int nb_max) {
   if (nb_max <= 32 * 4) return 4;
