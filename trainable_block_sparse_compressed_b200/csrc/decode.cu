@@ -33,7 +33,7 @@ int launch_decode_attn(const Geometry& g, const void* q, const void* Kcache, con
 
 namespace {
 
-constexpr int kScoreRows = 512;     // compressed rows per scoring CTA
+constexpr int kScoreTile = 128;     // compressed keys per scoring tile
 constexpr int kChunkBlocks = 8;     // selected blocks per attention item
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -48,7 +48,7 @@ DecodeLayout decode_layout(const Geometry& g) {
   DecodeLayout L;
   L.NC = num_compressed(g.T);
   L.NB = g.T > 0 ? (g.T - 1) / kBlock + 1 : 0;
-  L.n_split = L.NC > 0 ? (L.NC + kScoreRows - 1) / kScoreRows : 1;
+  L.n_split = L.NC > 0 ? (L.NC + kScoreTile - 1) / kScoreTile : 1;  // score tiles per row
   L.n_chunks = (g.topk + kChunkBlocks - 1) / kChunkBlocks;
   L.n_pool = L.NB > 0 ? (L.NB + kPoolBlocks - 1) / kPoolBlocks : 1;
   auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
@@ -122,85 +122,231 @@ __global__ void __launch_bounds__(32) decode_append_kernel(
 }
 
 // ---- 2. score --------------------------------------------------------------
+// Unit = one tile of 128 compressed keys of one (sequence, kv head).  A
+// persistent CTA walks units blockIdx.x, +gridDim.x, ...: warp 0 loads the
+// tile's hi and lo planes (4 boxes of 128 rows x 64 channels, 128-byte
+// swizzle) and the G query heads of the group into a 2-stage ring; warp 1
+// issues D[128 keys x 16 heads] = Kc . q^T with tcgen05.mma over K = 256
+// (q . hi + q . lo: the query tile is the B operand of both halves) into a
+// double-buffered TMEM accumulator; warps 2-5 (thread = key) write the scaled
+// scores x[j, h] and each tile's per-head max and sum of exp2, which the
+// select kernel merges into the head's log-sum-exp.  Units past the visible
+// keys of their sequence are skipped by all roles alike.
+constexpr int kDStages = 2;
+constexpr int kDHalf = kScoreTile * 64 * 2;       // 128 rows x 64 channels: 16 KB
+constexpr int kDKcBytes = 4 * kDHalf;             // hi and lo planes: 64 KB
+constexpr int kDQBytes = 2 * 16 * 128;            // 16 head rows x 2 halves of 64 channels
+constexpr int kDStageBytes = kDKcBytes + kDQBytes;  // 68 KB (a multiple of 1 KB)
+constexpr int kDThreads = 192;
+
+struct DScoreSmem {
+  uint64_t full[kDStages], empty[kDStages];
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  float red_m[4][16], red_l[4][16];
+};
+
+struct DUnit {
+  int bg, tile, b, g, v;
+  bool active;
+};
+
+__device__ __forceinline__ DUnit decode_unit(int64_t u, const int32_t* seqlens, int Hkv, int NC,
+                                             int n_tpb, int Lmax) {
+  DUnit r;
+  r.bg = static_cast<int>(u / n_tpb);
+  r.tile = static_cast<int>(u % n_tpb);
+  r.b = r.bg / Hkv;
+  r.g = r.bg % Hkv;
+  const int t = seqlens[r.b];
+  r.v = (t >= 0 && t < Lmax) ? min(NC, visible_windows(t)) : 0;
+  r.active = r.tile * kScoreTile < r.v;
+  return r;
+}
+
+__device__ __forceinline__ bool dwait(uint64_t* bar, uint32_t parity, const DevCtx& ctx,
+                                      volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  if (*abort_flag) return false;
+  if (mbar_wait(bar, parity, ctx.wait_ns)) return true;
+  report_status(ctx.status, INFLLMV2_STATUS_TIMEOUT);
+  *abort_flag = 1;
+  return false;
+}
+
 template <int G>
-__global__ void __launch_bounds__(256) decode_score_kernel(
-    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ Kcmp,
-    const int32_t* __restrict__ seqlens, float* __restrict__ x_out, float* __restrict__ ml,
-    int Hq, int Hkv, int NC, int Lmax, int n_split, float scale_log2) {
-  __shared__ float sq[G][kHeadDim];
-  __shared__ float red_m[8][G], red_l[8][G];
-  const int split = blockIdx.x % n_split;
-  const int bg = blockIdx.x / n_split;
-  const int b = bg / Hkv, g = bg % Hkv;
-  const int t = seqlens[b];
-  const int v = (t >= 0 && t < Lmax) ? min(NC, visible_windows(t)) : 0;
-  for (int i = threadIdx.x; i < G * kHeadDim; i += blockDim.x) {
-    const int h = i / kHeadDim, d = i % kHeadDim;
-    sq[h][d] = __bfloat162float(q[(static_cast<int64_t>(b) * Hq + g * G + h) * kHeadDim + d]) *
-               scale_log2;
+__global__ void __launch_bounds__(kDThreads, 1) decode_score_kernel(
+    const __grid_constant__ CUtensorMap tmKc, const __grid_constant__ CUtensorMap tmQ,
+    const int32_t* __restrict__ seqlens, float* __restrict__ x_out, float* __restrict__ ml, int B,
+    int Hkv, int NC, int n_tpb, int Lmax, float scale_log2, DevCtx ctx) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  DScoreSmem& sm = *reinterpret_cast<DScoreSmem*>(base + kDStages * kDStageBytes);
+  const int warp = warp_id(), lane = lane_id();
+  const int64_t n_units = static_cast<int64_t>(B) * Hkv * n_tpb;
+
+  // query rows past G stay zero (padding columns of the product)
+  for (int s = 0; s < kDStages; ++s)
+    for (int i = threadIdx.x; i < kDQBytes / 16; i += blockDim.x)
+      reinterpret_cast<uint4*>(base + s * kDStageBytes + kDKcBytes)[i] = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_smem();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kDStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&sm.acc_full[a], 1);
+      mbar_init(&sm.acc_empty[a], 4);  // one arrival per epilogue warp
+    }
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    fence_mbar_init();
   }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 32);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
-  float m[G], l[G];
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort_flag = &sm.abort_flag;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmKc);
+      tma_prefetch_desc(&tmQ);
+      int n = 0;
+      for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
+        const DUnit d = decode_unit(u, seqlens, Hkv, NC, n_tpb, Lmax);
+        if (!d.active) continue;
+        const int s = n % kDStages;
+        if (n >= kDStages && !dwait(&sm.empty[s], ((n / kDStages) & 1) ^ 1, ctx, abort_flag)) break;
+        uint8_t* dst = base + s * kDStageBytes;
+        mbar_arrive_expect_tx(&sm.full[s], kDKcBytes + 2 * G * 128);
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-    m[h] = -INFINITY;
-    l[h] = 0.f;
-  }
-  const int j_end = min(v, (split + 1) * kScoreRows);
-  for (int j = split * kScoreRows + threadIdx.x; j < j_end; j += blockDim.x) {
-    const __nv_bfloat16* row = Kcmp + ((static_cast<int64_t>(b) * NC + j) * Hkv + g) * kKcRow;
-    float acc[G];
+        for (int x = 0; x < 4; ++x)  // hi d[0:64], hi d[64:128], lo d[0:64], lo d[64:128]
+          tma_load_4d(dst + x * kDHalf, &tmKc, &sm.full[s], 64 * x, d.g, d.tile * kScoreTile, d.b);
+        tma_load_4d(dst + kDKcBytes, &tmQ, &sm.full[s], 0, d.g * G, 0, d.b);
+        tma_load_4d(dst + kDKcBytes + 2048, &tmQ, &sm.full[s], 64, d.g * G, 0, d.b);
+        ++n;
+      }
+      // drain: never leave with copies of this CTA in flight
+      for (int q = n - 1; q >= 0 && q >= n - kDStages; --q)
+        mbar_wait(&sm.full[q % kDStages], (q / kDStages) & 1, ctx.wait_ns);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = instr_desc_bf16(128, 16, 0, 0);
+      int n = 0;
+      for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
+        const DUnit d = decode_unit(u, seqlens, Hkv, NC, n_tpb, Lmax);
+        if (!d.active) continue;
+        const int s = n % kDStages, a = n & 1;
+        if (!dwait(&sm.full[s], (n / kDStages) & 1, ctx, abort_flag)) break;
+        if (n >= 2 && !dwait(&sm.acc_empty[a], ((n >> 1) & 1) ^ 1, ctx, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t kc_addr = smem_u32(base + s * kDStageBytes);
+        const uint32_t q_addr = kc_addr + kDKcBytes;
 #pragma unroll
-    for (int h = 0; h < G; ++h) acc[h] = 0.f;
-#pragma unroll 4
-    for (int d0 = 0; d0 < kHeadDim; d0 += 8) {
-      const uint4 u = __ldg(reinterpret_cast<const uint4*>(row + d0));
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(row + kHeadDim + d0));
-      const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&u);
-      const __nv_bfloat162* lv = reinterpret_cast<const __nv_bfloat162*>(&w);
+        for (int k = 0; k < 16; ++k) {
+          // k < 8: hi plane, k >= 8: lo plane; both against the same q
+          const uint32_t off = ((k >> 2) & 1) * kDHalf + (k & 3) * 32;
+          const uint64_t ad = smem_desc(kc_addr + (k >> 3) * 2 * kDHalf + off, 16, 1024, 2);
+          const uint64_t bd = smem_desc(q_addr + ((k >> 2) & 1) * 2048 + (k & 3) * 32, 16, 1024, 2);
+          umma_bf16(tmem + a * 16, ad, bd, idesc, k > 0 ? 1u : 0u);
+        }
+        umma_commit(&sm.empty[s]);
+        umma_commit(&sm.acc_full[a]);
+        ++n;
+      }
+      umma_commit(&sm.drain);
+      mbar_wait(&sm.drain, 0, ctx.wait_ns);
+    }
+  } else {
+    const int quad = warp & 3;
+    const int ew = warp - 2;            // epilogue warp 0..3
+    const int r = quad * 32 + lane;     // TMEM lane = key within the tile
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    int n = 0;
+    for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
+      const DUnit d = decode_unit(u, seqlens, Hkv, NC, n_tpb, Lmax);
+      float* mlo = ml + (static_cast<int64_t>(d.bg) * n_tpb + d.tile) * G * 2;
+      if (!d.active) {
+        if (r < G) {
+          mlo[2 * r] = -INFINITY;
+          mlo[2 * r + 1] = 0.f;
+        }
+        continue;
+      }
+      const int a = n & 1;
+      const bool ok = !*abort_flag && mbar_wait(&sm.acc_full[a], (n >> 1) & 1, ctx.wait_ns);
+      if (named_bar_or(2, 128, !ok)) {
+        if (!ok) report_status(ctx.status, INFLLMV2_STATUS_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      float x[16];
+      tmem_ld16(lane_addr + a * 16, x);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.acc_empty[a]);
+      const int j = d.tile * kScoreTile + r;
+      const bool valid = j < d.v;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float2 fh = __bfloat1622float2(hv[k]);
-        const float2 fl = __bfloat1622float2(lv[k]);
-        const float2 f = make_float2(fh.x + fl.x, fh.y + fl.y);
+      for (int h = 0; h < G; ++h) x[h] = valid ? x[h] * scale_log2 : -INFINITY;
+      if (valid) {
+        float* xo = x_out + (static_cast<int64_t>(d.bg) * NC + j) * G;
+        if constexpr (G % 4 == 0) {
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          acc[h] = fmaf(f.x, sq[h][d0 + 2 * k], acc[h]);
-          acc[h] = fmaf(f.y, sq[h][d0 + 2 * k + 1], acc[h]);
+          for (int h4 = 0; h4 < G / 4; ++h4)
+            reinterpret_cast<float4*>(xo)[h4] =
+                make_float4(x[4 * h4], x[4 * h4 + 1], x[4 * h4 + 2], x[4 * h4 + 3]);
+        } else {
+#pragma unroll
+          for (int h = 0; h < G; ++h) xo[h] = x[h];
         }
       }
-    }
-    float* xo = x_out + (static_cast<int64_t>(bg) * NC + j) * G;
+      // per-head max and sum of exp2 over the tile's valid keys
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      xo[h] = acc[h];
-      const float mn = fmaxf(m[h], acc[h]);
-      l[h] = l[h] * fast_exp2(m[h] - mn) + fast_exp2(acc[h] - mn);
-      m[h] = mn;
+      for (int h = 0; h < G; ++h) {
+        const float wm = warp_max(x[h]);
+        if (lane == 0) sm.red_m[ew][h] = wm;
+      }
+      named_bar_sync(1, 128);
+      float tl[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float M = fmaxf(fmaxf(sm.red_m[0][h], sm.red_m[1][h]),
+                              fmaxf(sm.red_m[2][h], sm.red_m[3][h]));
+        tl[h] = M > -INFINITY ? warp_sum(fast_exp2(x[h] - M)) : 0.f;
+      }
+      if (lane == 0) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) sm.red_l[ew][h] = tl[h];
+      }
+      named_bar_sync(1, 128);
+      if (r < G) {
+        const float M = fmaxf(fmaxf(sm.red_m[0][r], sm.red_m[1][r]),
+                              fmaxf(sm.red_m[2][r], sm.red_m[3][r]));
+        mlo[2 * r] = M;
+        mlo[2 * r + 1] = sm.red_l[0][r] + sm.red_l[1][r] + sm.red_l[2][r] + sm.red_l[3][r];
+      }
+      named_bar_sync(1, 128);  // red_m / red_l are rewritten by the next unit
+      ++n;
     }
   }
-  // CTA reduction of (m, l) per head
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    float mw = warp_max(m[h]);
-    float lw = mw > -INFINITY ? warp_sum(l[h] * fast_exp2(m[h] - mw)) : 0.f;
-    if (lane == 0) {
-      red_m[warp][h] = mw;
-      red_l[warp][h] = lw;
-    }
-  }
+  tc_fence_before();
   __syncthreads();
-  if (threadIdx.x < G) {
-    const int h = threadIdx.x;
-    float M = -INFINITY;
-    for (int w = 0; w < 8; ++w) M = fmaxf(M, red_m[w][h]);
-    float L = 0.f;
-    if (M > -INFINITY)
-      for (int w = 0; w < 8; ++w) L += red_l[w][h] * fast_exp2(red_m[w][h] - M);
-    float* o = ml + (static_cast<int64_t>(bg) * n_split + split) * G * 2;
-    o[2 * h] = M;
-    o[2 * h + 1] = L;
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 32);
   }
 }
 
@@ -344,10 +490,40 @@ int launch_decode_g(const Geometry& g, const DecodeLayout& L, const void* q, con
       static_cast<__nv_bfloat16*>(Kcmp), seqlens, active, pool_count, g.Hkv, g.T, L.NC,
       ctx.status);
   if (cudaGetLastError() != cudaSuccess) return INFLLMV2_ERR_CUDA;
-  decode_score_kernel<G><<<bgn * L.n_split, 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(Kcmp), seqlens, x, ml,
-      g.Hq, g.Hkv, L.NC, g.T, L.n_split, g.scale_log2);
-  if (cudaGetLastError() != cudaSuccess) return INFLLMV2_ERR_CUDA;
+  if (L.NC > 0) {
+    CUtensorMap tk, tq;
+    {
+      const uint64_t dims[4] = {static_cast<uint64_t>(kKcRow), static_cast<uint64_t>(g.Hkv),
+                                static_cast<uint64_t>(L.NC), static_cast<uint64_t>(g.B)};
+      const uint64_t strides[3] = {static_cast<uint64_t>(kKcRow) * 2,
+                                   static_cast<uint64_t>(g.Hkv) * kKcRow * 2,
+                                   static_cast<uint64_t>(L.NC) * g.Hkv * kKcRow * 2};
+      const uint32_t box[4] = {64u, 1u, static_cast<uint32_t>(kScoreTile), 1u};
+      if (int e = make_tmap_bf16_4d(&tk, Kcmp, dims, strides, box)) return e;
+    }
+    {
+      const uint64_t dims[4] = {static_cast<uint64_t>(kHeadDim), static_cast<uint64_t>(g.Hq), 1u,
+                                static_cast<uint64_t>(g.B)};
+      const uint64_t strides[3] = {static_cast<uint64_t>(kHeadDim) * 2,
+                                   static_cast<uint64_t>(g.Hq) * kHeadDim * 2,
+                                   static_cast<uint64_t>(g.Hq) * kHeadDim * 2};
+      const uint32_t box[4] = {64u, static_cast<uint32_t>(G), 1u, 1u};
+      if (int e = make_tmap_bf16_4d(&tq, q, dims, strides, box)) return e;
+    }
+    const size_t smem = 1024 + kDStages * kDStageBytes + sizeof(DScoreSmem);
+    static bool configured = false;
+    if (!configured) {
+      if (cudaFuncSetAttribute(decode_score_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem)) != cudaSuccess)
+        return INFLLMV2_ERR_CUDA;
+      configured = true;
+    }
+    const int64_t n_units = static_cast<int64_t>(bgn) * L.n_split;
+    const int grid = static_cast<int>(n_units < sm_count() ? n_units : sm_count());
+    decode_score_kernel<G><<<grid, kDThreads, smem, st>>>(tk, tq, seqlens, x, ml, g.B, g.Hkv, L.NC,
+                                                          L.n_split, g.T, g.scale_log2, ctx);
+    if (cudaGetLastError() != cudaSuccess) return INFLLMV2_ERR_CUDA;
+  }
   const int per = select_per(L.NB);
 #define INFLLMV2_SEL(V)                                                                        \
   decode_select_kernel<G, V><<<bgn * L.n_pool, 256, 0, st>>>(                                  \
