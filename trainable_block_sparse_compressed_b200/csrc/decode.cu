@@ -132,7 +132,7 @@ __global__ void __launch_bounds__(32) decode_append_kernel(
 // scores x[j, h] and each tile's per-head max and sum of exp2, which the
 // select kernel merges into the head's log-sum-exp.  Units past the visible
 // keys of their sequence are skipped by all roles alike.
-constexpr int kDStages = 2;
+constexpr int kDStages = 3;
 constexpr int kDHalf = kScoreTile * 64 * 2;       // 128 rows x 64 channels: 16 KB
 constexpr int kDKcBytes = 4 * kDHalf;             // hi and lo planes: 64 KB
 constexpr int kDQBytes = 2 * 16 * 128;            // 16 head rows x 2 halves of 64 channels
@@ -145,7 +145,7 @@ struct DScoreSmem {
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
-  float red_m[4][16], red_l[4][16];
+  float xs[kScoreTile][17];  // the tile's scaled scores, transposed for the per-head reductions
 };
 
 struct DUnit {
@@ -155,6 +155,7 @@ struct DUnit {
 
 __device__ __forceinline__ DUnit decode_unit(int64_t u, const int32_t* seqlens, int Hkv, int NC,
                                              int n_tpb, int Lmax) {
+  // seqlens: the sequences' positions (shared memory copy when B is small)
   DUnit r;
   r.bg = static_cast<int>(u / n_tpb);
   r.tile = static_cast<int>(u % n_tpb);
@@ -185,8 +186,11 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_score_kernel(
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   DScoreSmem& sm = *reinterpret_cast<DScoreSmem*>(base + kDStages * kDStageBytes);
+  __shared__ int32_t s_seq[256];
   const int warp = warp_id(), lane = lane_id();
   const int64_t n_units = static_cast<int64_t>(B) * Hkv * n_tpb;
+  for (int i = threadIdx.x; i < B && i < 256; i += blockDim.x) s_seq[i] = seqlens[i];
+  const int32_t* seq = B <= 256 ? s_seq : seqlens;
 
   // query rows past G stay zero (padding columns of the product)
   for (int s = 0; s < kDStages; ++s)
@@ -222,7 +226,7 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_score_kernel(
       tma_prefetch_desc(&tmQ);
       int n = 0;
       for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
-        const DUnit d = decode_unit(u, seqlens, Hkv, NC, n_tpb, Lmax);
+        const DUnit d = decode_unit(u, seq, Hkv, NC, n_tpb, Lmax);
         if (!d.active) continue;
         const int s = n % kDStages;
         if (n >= kDStages && !dwait(&sm.empty[s], ((n / kDStages) & 1) ^ 1, ctx, abort_flag)) break;
@@ -244,7 +248,7 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_score_kernel(
       constexpr uint32_t idesc = instr_desc_bf16(128, 16, 0, 0);
       int n = 0;
       for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
-        const DUnit d = decode_unit(u, seqlens, Hkv, NC, n_tpb, Lmax);
+        const DUnit d = decode_unit(u, seq, Hkv, NC, n_tpb, Lmax);
         if (!d.active) continue;
         const int s = n % kDStages, a = n & 1;
         if (!dwait(&sm.full[s], (n / kDStages) & 1, ctx, abort_flag)) break;
@@ -269,12 +273,12 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_score_kernel(
     }
   } else {
     const int quad = warp & 3;
-    const int ew = warp - 2;            // epilogue warp 0..3
+    const int ew = warp - 2;            // epilogue warp 0..3 (heads ew, ew+4, ...)
     const int r = quad * 32 + lane;     // TMEM lane = key within the tile
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     int n = 0;
     for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
-      const DUnit d = decode_unit(u, seqlens, Hkv, NC, n_tpb, Lmax);
+      const DUnit d = decode_unit(u, seq, Hkv, NC, n_tpb, Lmax);
       float* mlo = ml + (static_cast<int64_t>(d.bg) * n_tpb + d.tile) * G * 2;
       if (!d.active) {
         if (r < G) {
@@ -313,32 +317,26 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_score_kernel(
           for (int h = 0; h < G; ++h) xo[h] = x[h];
         }
       }
-      // per-head max and sum of exp2 over the tile's valid keys
+      // per-head max and sum of exp2 over the tile's keys: transpose through
+      // shared memory, then warp ew reduces heads ew, ew+4, ... (4 keys per lane)
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float wm = warp_max(x[h]);
-        if (lane == 0) sm.red_m[ew][h] = wm;
-      }
+      for (int h = 0; h < G; ++h) sm.xs[r][h] = x[h];
       named_bar_sync(1, 128);
-      float tl[G];
+      for (int h = ew; h < G; h += 4) {
+        float v[4];
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float M = fmaxf(fmaxf(sm.red_m[0][h], sm.red_m[1][h]),
-                              fmaxf(sm.red_m[2][h], sm.red_m[3][h]));
-        tl[h] = M > -INFINITY ? warp_sum(fast_exp2(x[h] - M)) : 0.f;
+        for (int i = 0; i < 4; ++i) v[i] = sm.xs[lane + 32 * i][h];
+        const float M = warp_max(fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3])));
+        float L = 0.f;
+        if (M > -INFINITY)
+          L = warp_sum(fast_exp2(v[0] - M) + fast_exp2(v[1] - M) + fast_exp2(v[2] - M) +
+                       fast_exp2(v[3] - M));
+        if (lane == 0) {
+          mlo[2 * h] = M;
+          mlo[2 * h + 1] = L;
+        }
       }
-      if (lane == 0) {
-#pragma unroll
-        for (int h = 0; h < G; ++h) sm.red_l[ew][h] = tl[h];
-      }
-      named_bar_sync(1, 128);
-      if (r < G) {
-        const float M = fmaxf(fmaxf(sm.red_m[0][r], sm.red_m[1][r]),
-                              fmaxf(sm.red_m[2][r], sm.red_m[3][r]));
-        mlo[2 * r] = M;
-        mlo[2 * r + 1] = sm.red_l[0][r] + sm.red_l[1][r] + sm.red_l[2][r] + sm.red_l[3][r];
-      }
-      named_bar_sync(1, 128);  // red_m / red_l are rewritten by the next unit
+      named_bar_sync(1, 128);  // xs is rewritten by the next unit
       ++n;
     }
   }
@@ -382,16 +380,33 @@ __global__ void __launch_bounds__(256) decode_select_kernel(
   const int blk1 = min(cur + 1, blk0 + kPoolBlocks);
   float* bs = bs_all + static_cast<int64_t>(bg) * NB;
   if (blk0 < blk1) {
-    if (threadIdx.x < G) {
-      const int h = threadIdx.x;
+    {
+      // 16 threads per head merge the score tiles' (max, sum) pairs
+      const int h = threadIdx.x >> 4, sub = threadIdx.x & 15;
       const float* p = ml + static_cast<int64_t>(bg) * n_split * G * 2;
-      float M = -INFINITY;
-      for (int s2 = 0; s2 < n_split; ++s2) M = fmaxf(M, p[s2 * G * 2 + 2 * h]);
-      float L = 0.f;
-      if (M > -INFINITY)
-        for (int s2 = 0; s2 < n_split; ++s2)
-          L += p[s2 * G * 2 + 2 * h + 1] * fast_exp2(p[s2 * G * 2 + 2 * h] - M);
-      lse2[h] = M > -INFINITY ? M + __log2f(L) : INFINITY;
+      float M = -INFINITY, L = 0.f;
+      if (h < G) {
+        for (int s2 = sub; s2 < n_split; s2 += 16) {
+          const float2 e = *reinterpret_cast<const float2*>(p + (s2 * G + h) * 2);
+          const float mn = fmaxf(M, e.x);
+          if (mn > -INFINITY) {
+            L = L * fast_exp2(M - mn) + e.y * fast_exp2(e.x - mn);
+            M = mn;
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) {
+        const float M2 = __shfl_xor_sync(0xffffffffu, M, o);
+        const float L2 = __shfl_xor_sync(0xffffffffu, L, o);
+        const float mn = fmaxf(M, M2);
+        if (mn > -INFINITY) {
+          L = (M > -INFINITY ? L * fast_exp2(M - mn) : 0.f) +
+              (M2 > -INFINITY ? L2 * fast_exp2(M2 - mn) : 0.f);
+          M = mn;
+        }
+      }
+      if (h < G && sub == 0) lse2[h] = M > -INFINITY ? M + __log2f(L) : INFINITY;
     }
     __syncthreads();
     const int j0 = max(0, 4 * blk0 - 1);

@@ -155,9 +155,15 @@ __device__ __forceinline__ void cta_select_row(const float* srow, int cur, int t
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int d = threadIdx.x; d < 256; d += NT) hist[d] = 0;
       __syncthreads();
+      // keys cluster in few digits (block scores span a narrow exponent
+      // range), so lanes with equal digits add once per warp
 #pragma unroll
-      for (int s = 0; s < PER; ++s)
-        if (key[s] != 0u && (key[s] & mask) == prefix) atomicAdd(&hist[(key[s] >> shift) & 255], 1);
+      for (int s = 0; s < PER; ++s) {
+        const bool part = key[s] != 0u && (key[s] & mask) == prefix;
+        const uint32_t d = part ? (key[s] >> shift) & 255u : 256u;
+        const uint32_t peers = __match_any_sync(0xffffffffu, d);
+        if (part && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[d], __popc(peers));
+      }
       __syncthreads();
       if (threadIdx.x < 32) {
         // suffix sums over the 256 digits, 8 per lane, lane 31 holding the top
