@@ -44,7 +44,8 @@ constexpr int kStages = 2;
 constexpr int kHalfBytes = kRows * 64 * 2; // one 64-channel half of a 128-row tile
 constexpr int kTileBytes = 2 * kHalfBytes; // 32 KB: the query tile
 constexpr int kKcBytes = 4 * kHalfBytes;   // 64 KB: hi and lo planes of 128 compressed keys
-constexpr int kThreads = 192;
+constexpr int kEpiThreads = 256;          // two epilogue warpgroups, 64 columns each
+constexpr int kThreads = 64 + kEpiThreads;
 constexpr uint32_t kTmemCols = 256;
 
 struct ScoreSmem {
@@ -57,6 +58,7 @@ struct ScoreSmem {
   uint32_t tmem_base;
   int abort_flag;
   float lse2[kRows];                 // per query row: log2-domain LSE
+  float part_m[kRows], part_l[kRows];  // pass 1: the upper column half's running max / sum
   float carry[3][4][kRows];          // S of the window just before each 32-lane quadrant
 };
 
@@ -102,7 +104,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&sm.acc_full[a], 1);
-      mbar_init(&sm.acc_empty[a], 128);
+      mbar_init(&sm.acc_empty[a], kEpiThreads / 32);  // one arrival per epilogue warp
     }
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
@@ -112,10 +114,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  if (threadIdx.x >= 64) {
-    const int r = threadIdx.x - 64;
-    for (int k = 0; k < 3 * 4; ++k) (&sm.carry[0][0][0])[k * kRows + r] = -INFINITY;
-  }
+  for (int i = threadIdx.x; i < 3 * 4 * kRows; i += blockDim.x) (&sm.carry[0][0][0])[i] = -INFINITY;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -182,12 +181,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&sm.drain, 0, ctx.wait_ns);
     }
   } else {
-    // ---------------- epilogue: 4 warps, thread <-> TMEM lane ----------------
+    // ---------------- epilogue: 8 warps, thread <-> TMEM lane ----------------
+    // Two warpgroups split the accumulator's 128 columns: warpgroup hf reads
+    // columns 64 hf .. 64 hf + 63 of its lanes.  Pass 1: each keeps a partial
+    // running max / sum of its row over its half, merged at the end of the
+    // pass.  Pass 2: the columns are (token, head) pairs, so warpgroup hf owns
+    // tokens hf TPT/2 .. (hf+1) TPT/2 - 1.  Two warps per scheduler keep the
+    // exp2 / shuffle chains of the epilogue overlapped.
+    constexpr int TPH = TPT / 2;     // tokens per warpgroup in pass 2 (G <= 64)
+    const int hf = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;  // TMEM lane this thread reads
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + hf * 64;
     const int64_t slab = score_row_offset(T);
     float* srow_base = scores + (static_cast<int64_t>(b) * Hkv + g) * slab;
+    constexpr uint32_t bar_sync_all = 1, bar_or_all = 2;  // 256 threads
+    const uint32_t bar_sync_half = 3 + hf;                // the 128 threads of this warpgroup
 
     // pass-1 row identity
     const int my_tok = r / G;
@@ -197,79 +206,94 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     for (int it = 0; it < n_it; ++it) {
       const int a = it & 1;
-      // all 128 threads take the same decision, so the named barriers below
-      // are always reached by the whole group
+      // all 256 threads take the same decision, so the named barriers below
+      // are always reached by every thread that waits at them
       const bool ok = !*abort_flag && mbar_wait(&sm.acc_full[a], (it >> 1) & 1, ctx.wait_ns);
-      if (named_bar_or(2, 128, !ok)) {
+      if (named_bar_or(bar_or_all, kEpiThreads, !ok)) {
         if (!ok) report_status(ctx.status, INFLLMV2_STATUS_TIMEOUT);
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      float x[kRows];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float* xc = x + 32 * c;
-        tmem_ld32(lane_addr + a * 128 + 32 * c, *reinterpret_cast<float(*)[32]>(xc));
-      }
+      float x[64];
+      tmem_ld32(lane_addr + a * 128, *reinterpret_cast<float(*)[32]>(x));
+      tmem_ld32(lane_addr + a * 128 + 32, *reinterpret_cast<float(*)[32]>(x + 32));
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(&sm.acc_empty[a]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.acc_empty[a]);
 
       if (it < n_t) {
         // ---- pass 1: running max / sum of row r over its visible windows ----
-        const int j0 = it * kKcTile;
-        const int nv = min(kKcTile, my_v - j0);  // valid columns (may be <= 0)
+        const int j0 = it * kKcTile + hf * 64;
+        const int nv = min(64, my_v - j0);  // valid columns of this half (may be <= 0)
         float tmax = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < kKcTile; ++c)
+        for (int c = 0; c < 64; ++c)
           if (c < nv) tmax = fmaxf(tmax, x[c]);
         const float m_new = fmaxf(m_run, tmax);
         if (m_new > -INFINITY) {
           const float mb = m_new * scale_log2;
           float acc = 0.f;
 #pragma unroll
-          for (int c = 0; c < kKcTile; ++c)
+          for (int c = 0; c < 64; ++c)
             if (c < nv) acc += fast_exp2(fmaf(x[c], scale_log2, -mb));
           l_run = l_run * fast_exp2((m_run - m_new) * scale_log2) + acc;
           m_run = m_new;
         }
         if (it == n_t - 1) {
-          sm.lse2[r] = my_v > 0 ? m_run * scale_log2 + __log2f(l_run) : INFINITY;
-          named_bar_sync(1, 128);
+          // merge the two halves of row r
+          if (hf == 1) {
+            sm.part_m[r] = m_run;
+            sm.part_l[r] = l_run;
+          }
+          named_bar_sync(bar_sync_all, kEpiThreads);
+          if (hf == 0) {
+            const float m2 = sm.part_m[r], l2 = sm.part_l[r];
+            const float mm = fmaxf(m_run, m2);
+            float ll = 0.f;
+            if (mm > -INFINITY)
+              ll = (m_run > -INFINITY ? l_run * fast_exp2((m_run - mm) * scale_log2) : 0.f) +
+                   (m2 > -INFINITY ? l2 * fast_exp2((m2 - mm) * scale_log2) : 0.f);
+            sm.lse2[r] = my_v > 0 ? mm * scale_log2 + __log2f(ll) : INFINITY;
+          }
+          named_bar_sync(bar_sync_all, kEpiThreads);
         }
       } else {
         // ---- pass 2: lane r is compressed key j; columns are (token, head) rows ----
         const int i = it - n_t;
         const int j = i * kKcTile + r;
-        float S[TPT];
+        float S[TPH];
 #pragma unroll
-        for (int tok = 0; tok < TPT; ++tok) {
+        for (int tl = 0; tl < TPH; ++tl) {
+          const int tok = hf * TPH + tl;
           const int t = t0 + tok;
           const int v = t < T ? min(n_c, visible_windows(t)) : 0;
           float acc = 0.f;
 #pragma unroll
           for (int h = 0; h < G; ++h)
-            acc += fast_exp2(fmaf(x[tok * G + h], scale_log2, -sm.lse2[tok * G + h]));
-          S[tok] = j < v ? acc : -INFINITY;
+            acc += fast_exp2(fmaf(x[tl * G + h], scale_log2, -sm.lse2[tok * G + h]));
+          S[tl] = j < v ? acc : -INFINITY;
         }
         const int cb = i % 3;
         if (lane == 31) {
 #pragma unroll
-          for (int tok = 0; tok < TPT; ++tok) {
+          for (int tl = 0; tl < TPH; ++tl) {
+            const int tok = hf * TPH + tl;
             if (quad < 3)
-              sm.carry[cb][quad + 1][tok] = S[tok];
+              sm.carry[cb][quad + 1][tok] = S[tl];
             else
-              sm.carry[(i + 1) % 3][0][tok] = S[tok];
+              sm.carry[(i + 1) % 3][0][tok] = S[tl];
           }
         }
-        named_bar_sync(1, 128);
+        named_bar_sync(bar_sync_half, kEpiThreads / 2);
         const int blk = i * (kKcTile / 4) + quad * 8 + (lane >> 2);
 #pragma unroll
-        for (int tok = 0; tok < TPT; ++tok) {
-          float m4 = fmaxf(S[tok], __shfl_xor_sync(0xffffffffu, S[tok], 1));
+        for (int tl = 0; tl < TPH; ++tl) {
+          const int tok = hf * TPH + tl;
+          float m4 = fmaxf(S[tl], __shfl_xor_sync(0xffffffffu, S[tl], 1));
           m4 = fmaxf(m4, __shfl_xor_sync(0xffffffffu, m4, 2));
-          float prev = __shfl_up_sync(0xffffffffu, S[tok], 1);
+          float prev = __shfl_up_sync(0xffffffffu, S[tl], 1);
           if (lane == 0) prev = sm.carry[cb][quad][tok];
           const int t = t0 + tok;
           if ((lane & 3) == 0 && t < T && blk <= t / kBlock)
@@ -280,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // blocks past the last compressed-key tile: at most block 32*n_t, whose
     // only visible window can be the last one of the final tile.
     if (!*abort_flag) {
-      for (int tok = r; tok < TPT; tok += 128) {
+      for (int tok = hf * TPH + r; tok < (hf + 1) * TPH; tok += 128) {
         const int t = t0 + tok;
         if (t >= T) continue;
         const int cur = t / kBlock;
