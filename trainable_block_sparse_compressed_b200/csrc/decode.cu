@@ -15,7 +15,7 @@
 //   3. select      : per (sequence, kv head), split over CTAs of 128 blocks
 //                    each: merge the splits into each head's log-sum-exp,
 //                    group-sum the probabilities, max-pool onto 64-token
-//                    blocks; the last CTA of the row runs the warp top-k with
+//                    blocks; then one CTA per row runs the exact top-k with
 //                    the forced blocks;
 //   4. attention   : sparse_attn.cu in decode mode, the selected blocks split
 //                    into chunks, unnormalised partials;
@@ -41,7 +41,7 @@ constexpr int kPoolBlocks = 128;    // blocks max-pooled per pooling CTA
 
 struct DecodeLayout {
   int NC, NB, n_split, n_chunks, n_pool;
-  size_t off_active, off_x, off_ml, off_idx, off_part, off_bs, off_cnt, total;
+  size_t off_active, off_x, off_ml, off_idx, off_part, off_bs, total;
 };
 
 DecodeLayout decode_layout(const Geometry& g) {
@@ -66,8 +66,6 @@ DecodeLayout decode_layout(const Geometry& g) {
   o = up(o + bg * L.n_chunks * g.G * (kHeadDim + 2) * sizeof(float));
   L.off_bs = o;
   o = up(o + bg * static_cast<size_t>(L.NB) * sizeof(float));
-  L.off_cnt = o;
-  o = up(o + bg * sizeof(uint32_t));
   L.total = o;
   return L;
 }
@@ -77,11 +75,9 @@ __global__ void __launch_bounds__(32) decode_append_kernel(
     const __nv_bfloat16* __restrict__ k_new, const __nv_bfloat16* __restrict__ v_new,
     __nv_bfloat16* __restrict__ Kc_, __nv_bfloat16* __restrict__ Vc_,
     __nv_bfloat16* __restrict__ Kcmp, const int32_t* __restrict__ seqlens,
-    int32_t* __restrict__ active, uint32_t* __restrict__ pool_count, int Hkv, int Lmax, int NC,
-    int* status) {
+    int32_t* __restrict__ active, int Hkv, int Lmax, int NC, int* status) {
   const int b = blockIdx.x / Hkv, g = blockIdx.x % Hkv;
   const int tid = threadIdx.x;
-  if (tid == 0) pool_count[blockIdx.x] = 0;  // arrivals of this step's pooling CTAs
   const int pos = seqlens[b];
   const bool act = pos >= 0 && pos < Lmax;
   if (g == 0 && tid == 0) {
@@ -352,28 +348,19 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_score_kernel(
 // Pooling CTA (bg, part) owns blocks [part*128, part*128 + 128) of row bg:
 // merges the score splits into each head's log2-sum-exp, sums the G heads'
 // probabilities over the windows overlapping its blocks, max-pools them, and
-// writes the block scores.  The last CTA of the row to finish (an arrival
-// counter that the append kernel zeroed) runs the CTA top-k over the row,
-// PER blocks per thread.
-template <int G, int PER>
-__global__ void __launch_bounds__(256) decode_select_kernel(
+// writes the block scores; decode_topk_kernel then selects per row.
+template <int G>
+__global__ void __launch_bounds__(256) decode_pool_kernel(
     const float* __restrict__ x, const float* __restrict__ ml, const int32_t* __restrict__ seqlens,
-    float* bs_all, uint32_t* pool_count, int32_t* __restrict__ idx, int Hkv, int NC, int NB,
-    int Lmax, int n_split, int n_pool, int topk, int n_init, int n_local) {
+    float* __restrict__ bs_all, int Hkv, int NC, int NB, int Lmax, int n_split, int n_pool) {
   constexpr int kWin = 4 * kPoolBlocks + 4;  // windows 4*blk0-1 .. 4*blk1+3 (clipped)
   __shared__ float S[kWin];
   __shared__ float lse2[G];
-  __shared__ bool last;
   const int bg = blockIdx.x / n_pool;
   const int part = blockIdx.x % n_pool;
   const int b = bg / Hkv;
   const int t = seqlens[b];
-  int32_t* orow = idx + static_cast<int64_t>(bg) * topk;
-  if (!(t >= 0 && t < Lmax)) {
-    if (part == 0)
-      for (int k = threadIdx.x; k < topk; k += blockDim.x) orow[k] = -1;
-    return;
-  }
+  if (!(t >= 0 && t < Lmax)) return;
   const int v = min(NC, visible_windows(t));
   const int cur = t / kBlock;
   const int blk0 = part * kPoolBlocks;
@@ -386,6 +373,7 @@ __global__ void __launch_bounds__(256) decode_select_kernel(
       const float* p = ml + static_cast<int64_t>(bg) * n_split * G * 2;
       float M = -INFINITY, L = 0.f;
       if (h < G) {
+#pragma unroll 4
         for (int s2 = sub; s2 < n_split; s2 += 16) {
           const float2 e = *reinterpret_cast<const float2*>(p + (s2 * G + h) * 2);
           const float mn = fmaxf(M, e.x);
@@ -436,14 +424,23 @@ __global__ void __launch_bounds__(256) decode_select_kernel(
       bs[blk] = mx;
     }
   }
-  // the last pooling CTA of the row selects
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) last = atomicAdd(pool_count + bg, 1u) == static_cast<uint32_t>(n_pool - 1);
-  __syncthreads();
-  if (!last) return;
-  __threadfence();
-  cta_select_row<256, PER>(bs, cur, topk, n_init, n_local, orow);
+}
+
+// One CTA of 256 threads per (sequence, kv head): the exact top-k over the
+// row's block scores, PER blocks per thread.
+template <int PER>
+__global__ void __launch_bounds__(256) decode_topk_kernel(
+    const float* __restrict__ bs_all, const int32_t* __restrict__ seqlens, int32_t* __restrict__ idx,
+    int Hkv, int NB, int Lmax, int topk, int n_init, int n_local) {
+  const int bg = blockIdx.x;
+  const int t = seqlens[bg / Hkv];
+  int32_t* orow = idx + static_cast<int64_t>(bg) * topk;
+  if (!(t >= 0 && t < Lmax)) {
+    for (int k = threadIdx.x; k < topk; k += blockDim.x) orow[k] = -1;
+    return;
+  }
+  cta_select_row<256, PER>(bs_all + static_cast<int64_t>(bg) * NB, t / kBlock, topk, n_init,
+                           n_local, orow);
 }
 
 // Blocks per thread of the 256-thread CTA top-k for rows of up to nb blocks
@@ -497,12 +494,11 @@ int launch_decode_g(const Geometry& g, const DecodeLayout& L, const void* q, con
   float* ml = reinterpret_cast<float*>(ws + L.off_ml);
   float* part = reinterpret_cast<float*>(ws + L.off_part);
   float* bs = reinterpret_cast<float*>(ws + L.off_bs);
-  uint32_t* pool_count = reinterpret_cast<uint32_t*>(ws + L.off_cnt);
   const int bgn = g.B * g.Hkv;
   decode_append_kernel<<<bgn, 32, 0, st>>>(
       static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new),
       static_cast<__nv_bfloat16*>(Kc_), static_cast<__nv_bfloat16*>(Vc_),
-      static_cast<__nv_bfloat16*>(Kcmp), seqlens, active, pool_count, g.Hkv, g.T, L.NC,
+      static_cast<__nv_bfloat16*>(Kcmp), seqlens, active, g.Hkv, g.T, L.NC,
       ctx.status);
   if (cudaGetLastError() != cudaSuccess) return INFLLMV2_ERR_CUDA;
   if (L.NC > 0) {
@@ -540,10 +536,12 @@ int launch_decode_g(const Geometry& g, const DecodeLayout& L, const void* q, con
     if (cudaGetLastError() != cudaSuccess) return INFLLMV2_ERR_CUDA;
   }
   const int per = select_per(L.NB);
-#define INFLLMV2_SEL(V)                                                                        \
-  decode_select_kernel<G, V><<<bgn * L.n_pool, 256, 0, st>>>(                                  \
-      x, ml, seqlens, bs, pool_count, idx, g.Hkv, L.NC, L.NB, g.T, L.n_split, L.n_pool, g.topk, \
-      g.n_init, g.n_local)
+  decode_pool_kernel<G><<<bgn * L.n_pool, 256, 0, st>>>(x, ml, seqlens, bs, g.Hkv, L.NC, L.NB, g.T,
+                                                       L.n_split, L.n_pool);
+  if (cudaGetLastError() != cudaSuccess) return INFLLMV2_ERR_CUDA;
+#define INFLLMV2_SEL(V)                                                                     \
+  decode_topk_kernel<V><<<bgn, 256, 0, st>>>(bs, seqlens, idx, g.Hkv, L.NB, g.T, g.topk, \
+                                             g.n_init, g.n_local)
   switch (per) {
     case 1: INFLLMV2_SEL(1); break;
     case 2: INFLLMV2_SEL(2); break;

@@ -215,12 +215,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                               : static_cast<int64_t>(args.Hkv) * args.B * args.T;
   const float scale_log2 = args.scale_log2;
 
-  // zero the operand buffers once: a pair with a single block leaves its
-  // second slot stale, and stale data must be finite (it is multiplied by 0)
+  // A pair with a single block leaves its second slot stale.  Stale K rows
+  // only produce scores that the softmax masks to -inf, but stale V rows are
+  // multiplied by P = 0, so they must be finite: zero, once, the V bytes that
+  // second blocks occupy in either layout (packed: 16..32 KB of the V pair,
+  // boxes: 8..16 KB and 24..32 KB).
   {
-    uint4* p = reinterpret_cast<uint4*>(base);
-    const int n16 = (kStages * kStageBytes + 2 * kQBytes + 2 * kPBytes) / 16;
-    for (int i = threadIdx.x; i < n16; i += blockDim.x) p[i] = make_uint4(0, 0, 0, 0);
+    constexpr int kZero = (kPairBytes - kSlotBytes) / 16;  // 8..32 KB of the V pair
+    for (int i = threadIdx.x; i < kStages * kZero; i += blockDim.x) {
+      const int st = i / kZero, k = i % kZero;
+      reinterpret_cast<uint4*>(base + st * kStageBytes + kPairBytes + kSlotBytes)[k] =
+          make_uint4(0, 0, 0, 0);
+    }
+    // query rows past G (padding heads) stay zero as well
+    for (int i = threadIdx.x; i < 2 * kQBytes / 16; i += blockDim.x)
+      reinterpret_cast<uint4*>(sQ)[i] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
   }
   if (threadIdx.x == 0) {

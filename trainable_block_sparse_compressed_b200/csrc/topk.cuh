@@ -119,18 +119,29 @@ __device__ __forceinline__ int cta_exclusive_scan(int v, int* scratch, int* tota
 
 // The same selection as warp_select_row, by a whole CTA of NT threads: thread
 // i holds blocks i*PER .. i*PER+PER-1 (rows of up to NT*PER blocks).  The
-// free_slots-th largest candidate key tau is found by a radix select over
-// four 8-bit digits, most significant first (a 256-bin histogram per digit).
-// Keys above tau are kept; among keys equal to tau the lowest block indices
-// fill the remaining slots (a prefix sum over threads in index order); a
-// second prefix sum places the kept blocks in ascending order.  All threads
-// must call.
+// free_slots-th largest candidate key tau is found bit by bit, most
+// significant first, with a CTA-wide count per bit (warp reductions, one
+// barrier per round over a double-buffered array of warp counts).  Keys
+// above tau are kept; among keys equal to tau the lowest block indices fill
+// the remaining slots (a prefix sum over threads in index order); a second
+// prefix sum places the kept blocks in ascending order.  All threads must
+// call.
+template <int NT>
+__device__ __forceinline__ int cta_count(int v, int (*buf)[NT / 32], int round) {
+  const int s = __reduce_add_sync(0xffffffffu, v);
+  if ((threadIdx.x & 31) == 0) buf[round & 1][threadIdx.x >> 5] = s;
+  __syncthreads();
+  int tot = 0;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) tot += buf[round & 1][w];
+  return tot;
+}
+
 template <int NT, int PER>
 __device__ __forceinline__ void cta_select_row(const float* srow, int cur, int topk, int n_init,
                                                int n_local, int32_t* orow) {
-  __shared__ int hist[256];
+  __shared__ int cnt_buf[2][NT / 32];
   __shared__ int scan_buf[NT / 32 + 1];
-  __shared__ int pick[2];  // digit, count of keys above it
   const int nb = cur + 1;
   auto forced = [&](int i) { return i < n_init || i > cur - n_local; };
   const int a = min(n_init, nb);
@@ -150,60 +161,18 @@ __device__ __forceinline__ void cta_select_row(const float* srow, int cur, int t
   uint32_t tau = 0;
   int need_eq = 0;
   if (!take_all) {
-    uint32_t prefix = 0, mask = 0;
-    int k = free_slots;  // rank of tau among the keys that match prefix
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int d = threadIdx.x; d < 256; d += NT) hist[d] = 0;
-      __syncthreads();
-      // keys cluster in few digits (block scores span a narrow exponent
-      // range), so lanes with equal digits add once per warp
+    int round = 0;
+    for (int bit = 31; bit >= 0; --bit, ++round) {
+      const uint32_t c = tau | (1u << bit);
+      int n = 0;
 #pragma unroll
-      for (int s = 0; s < PER; ++s) {
-        const bool part = key[s] != 0u && (key[s] & mask) == prefix;
-        const uint32_t d = part ? (key[s] >> shift) & 255u : 256u;
-        const uint32_t peers = __match_any_sync(0xffffffffu, d);
-        if (part && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[d], __popc(peers));
-      }
-      __syncthreads();
-      if (threadIdx.x < 32) {
-        // suffix sums over the 256 digits, 8 per lane, lane 31 holding the top
-        const int lane = threadIdx.x;
-        int c[8], sum = 0;
-#pragma unroll
-        for (int u = 7; u >= 0; --u) {
-          c[u] = hist[lane * 8 + u];
-          sum += c[u];
-        }
-        int above = sum;  // keys with digits in lanes >= this lane
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_down_sync(0xffffffffu, above, o);
-          if (lane + o < 32) above += y;
-        }
-        int higher = above - sum;  // keys with digits in lanes above this lane
-        int dsel = -1, hsel = 0;
-#pragma unroll
-        for (int u = 7; u >= 0; --u) {
-          if (dsel < 0 && higher < k && higher + c[u] >= k) {
-            dsel = lane * 8 + u;
-            hsel = higher;
-          }
-          higher += c[u];
-        }
-        if (dsel >= 0) {
-          pick[0] = dsel;
-          pick[1] = hsel;
-        }
-      }
-      __syncthreads();
-      const int dsel = pick[0];
-      k -= pick[1];
-      prefix |= static_cast<uint32_t>(dsel) << shift;
-      mask |= 255u << shift;
-      __syncthreads();
+      for (int s = 0; s < PER; ++s) n += key[s] >= c ? 1 : 0;
+      if (cta_count<NT>(n, cnt_buf, round) >= free_slots) tau = c;
     }
-    tau = prefix;
-    need_eq = k;
+    int n = 0;
+#pragma unroll
+    for (int s = 0; s < PER; ++s) n += key[s] > tau ? 1 : 0;
+    need_eq = free_slots - cta_count<NT>(n, cnt_buf, round);
   }
   // keys equal to tau, ranked by block index
   int n_eq = 0;
