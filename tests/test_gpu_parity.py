@@ -108,6 +108,23 @@ def test_select_blocks_all_rows(cuda_lib, case):
     assert exact >= 0.8 * len(det), f"only {exact}/{len(det)} rows exact"
 
 
+TIE_CASES = [(1, 1500, 32, 2, 16), (2, 700, 8, 1, 6), (1, 2111, 32, 2, 12)]
+
+
+@pytest.mark.parametrize("case", TIE_CASES, ids=[f"B{c[0]}_T{c[1]}_Hq{c[2]}_k{c[4]}" for c in TIE_CASES])
+def test_select_exact_ties_go_to_lower_blocks(cuda_lib, case):
+    """Every key equal: every visible window scores alike, so all block scores
+    with a visible window are exactly equal (on the GPU as in the oracle) and
+    the free slots go to the lowest-index free blocks -- compared exactly."""
+    B, T, Hq, Hkv, topk = case
+    w = wl.small_workload(B=B, T=T, Hq=Hq, Hkv=Hkv, topk=topk, needles=0, seed=21)
+    data = wl.make_prefill(w)
+    data["K"][:] = data["K"][:, :1]  # every token carries the first token's key
+    got = _run_select(cuda_lib, w, data)
+    ref, _ = orc.select_blocks(wl.bf16_to_f64(data["Q"]), wl.bf16_to_f64(data["K"]), _oparams(w))
+    assert np.array_equal(got, ref)
+
+
 # ---------------------------------------------------------------------------
 # attention with the oracle's selection
 # ---------------------------------------------------------------------------
@@ -273,9 +290,11 @@ def test_prefill_128k_sampled(cuda_lib):
 # ---------------------------------------------------------------------------
 # decode
 # ---------------------------------------------------------------------------
-def _decode_setup(api, w, L0, steps, B):
+def _decode_setup(api, w, L0, steps, B, mutate=None):
     import torch
     data = wl.make_decode(w, L=L0, steps=steps, B=B)
+    if mutate is not None:
+        mutate(data)
     Lmax = L0 + steps
     p = api.make_params(B, Lmax, w.Hq, w.Hkv, topk=w.topk, n_init=w.n_init, n_local=w.n_local)
     NC = api.num_compressed(Lmax)
@@ -407,3 +426,34 @@ def test_timeout_selftest_reports_and_context_survives(cuda_lib):
     assert api.get_status() == 0
     # the context still runs real work
     test_compress_keys(cuda_lib, 1000, 2, 2)
+
+
+def test_decode_exact_ties_go_to_lower_blocks(cuda_lib):
+    """Decode with every cached and appended key equal: the block scores tie
+    exactly and the selection must equal the oracle's lowest-index choice."""
+    import torch
+    api = cuda_lib
+    w = wl.WORKLOADS["sparse_decode_B16_L131072_Hq32_Hkv2"]
+    B, L0, steps = 2, 3000, 20
+
+    def same_keys(d):
+        d["K0"][:] = d["K0"][:, :1]
+        d["k_new"][:] = d["K0"][:, 0][None]
+
+    data, p, Kc, Vc, Kcmp, seqlens, ws = _decode_setup(api, w, L0, steps, B, mutate=same_keys)
+    op = orc.Params(topk=w.topk)
+    st = orc.DecodeState.from_prefill(wl.bf16_to_f64(data["K0"]), wl.bf16_to_f64(data["V0"]), op)
+    O = torch.empty((B, w.Hq, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, w.Hq), dtype=torch.float32, device="cuda")
+    idx = torch.empty((B, w.Hkv, w.topk), dtype=torch.int32, device="cuda")
+    for s in range(steps):
+        api.decode_step(p, gpu_bf16(data["q"][s]), gpu_bf16(data["k_new"][s]),
+                        gpu_bf16(data["v_new"][s]), Kc, Vc, Kcmp, seqlens, O, lse, idx, ws)
+        torch.cuda.synchronize()
+        O_ref, L_ref, i_ref = orc.decode_step(st, wl.bf16_to_f64(data["q"][s]),
+                                              wl.bf16_to_f64(data["k_new"][s]),
+                                              wl.bf16_to_f64(data["v_new"][s]), op)
+        assert np.array_equal(idx.cpu().numpy(), i_ref), s
+        assert np.abs(f64(O) - O_ref).max() <= O_ATOL
+        assert np.abs(f64(lse) - L_ref).max() <= LSE_ATOL
+    assert api.get_status() == 0
