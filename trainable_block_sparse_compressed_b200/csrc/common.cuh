@@ -9,6 +9,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/infllmv2.h"
 
 namespace infllmv2 {
@@ -80,6 +82,22 @@ __device__ __forceinline__ void store_kc_pair(const float (&m)[8], __nv_bfloat16
 // Host helpers (api.cu).
 cudaError_t get_dev_ctx(DevCtx* ctx);
 int sm_count();
+
+// Raises a kernel's dynamic shared memory limit to `bytes` on the current
+// device, once per device (`done` holds one bit per device id < 64; others
+// are set on every call, which is harmless).
+template <typename F>
+inline int set_smem_limit(F* func, size_t bytes, std::atomic<uint64_t>& done) {
+  int d = -1;
+  if (cudaGetDevice(&d) != cudaSuccess) return INFLLMV2_ERR_CUDA;
+  const uint64_t bit = (d >= 0 && d < 64) ? (uint64_t{1} << d) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return INFLLMV2_OK;
+  if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(bytes)) != cudaSuccess)
+    return INFLLMV2_ERR_CUDA;
+  done.fetch_or(bit, std::memory_order_release);
+  return INFLLMV2_OK;
+}
 
 // Tensor maps (tma.cpp).
 int make_tmap_bf16_4d(CUtensorMap* map, const void* base, const uint64_t dims[4],

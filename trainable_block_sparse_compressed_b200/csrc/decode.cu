@@ -522,13 +522,8 @@ int launch_decode_g(const Geometry& g, const DecodeLayout& L, const void* q, con
       if (int e = make_tmap_bf16_4d(&tq, q, dims, strides, box)) return e;
     }
     const size_t smem = 1024 + kDStages * kDStageBytes + sizeof(DScoreSmem);
-    static bool configured = false;
-    if (!configured) {
-      if (cudaFuncSetAttribute(decode_score_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem)) != cudaSuccess)
-        return INFLLMV2_ERR_CUDA;
-      configured = true;
-    }
+    static std::atomic<uint64_t> smem_set{0};
+    if (int e = set_smem_limit(decode_score_kernel<G>, smem, smem_set)) return e;
     const int64_t n_units = static_cast<int64_t>(bgn) * L.n_split;
     const int grid = static_cast<int>(n_units < sm_count() ? n_units : sm_count());
     decode_score_kernel<G><<<grid, kDThreads, smem, st>>>(tk, tq, seqlens, x, ml, g.B, g.Hkv, L.NC,

@@ -328,13 +328,8 @@ int launch_score_g(const Geometry& g, const CUtensorMap& tq, const CUtensorMap& 
                    const DevCtx& ctx, cudaStream_t st) {
   constexpr int TPT = kRows / G;
   const size_t smem = 1024 + kTileBytes + kKcBytes * kStages + sizeof(ScoreSmem);
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(score_blocks_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return INFLLMV2_ERR_CUDA;
-    configured = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  if (int e = set_smem_limit(score_blocks_kernel<G>, smem, smem_set)) return e;
   const int n_qt = (g.T + TPT - 1) / TPT;
   const unsigned grid = static_cast<unsigned>(n_qt) * g.B * g.Hkv;
   score_blocks_kernel<G><<<grid, kThreads, smem, st>>>(tq, tk, scores, g.B, g.T, g.Hkv, g.n_c,

@@ -68,7 +68,7 @@ struct AttnSmem {
   uint64_t q_full[2], q_empty[2];
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full[2];
-  uint64_t pv_full[2], pv_empty[2];
+  uint64_t pv_full[2];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -247,7 +247,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.s_empty[a], kSoftmaxThreads / 32);
       mbar_init(&sm.p_full[a], kSoftmaxThreads / 32);
       mbar_init(&sm.pv_full[a], 1);
-      mbar_init(&sm.pv_empty[a], kSoftmaxThreads / 32);
     }
     mbar_init(&sm.drain, 2);  // one commit from each MMA issuer
     sm.abort_flag = 0;
@@ -368,9 +367,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int p = 0; ok && p < item.n_pairs; ++p, ++gp) {
           const int a = static_cast<int>(gp & 1);
           const int st = static_cast<int>(gp % kStages);
-          ok = wait_or_abort(&sm.p_full[a], (gp >> 1) & 1, ctx, abort_flag) &&
-               wait_or_abort(&sm.full[st], (gp / kStages) & 1, ctx, abort_flag) &&
-               (gp < 2 || wait_or_abort(&sm.pv_empty[a], ((gp >> 1) & 1) ^ 1, ctx, abort_flag));
+          // P(q) complete implies everything else P V(q) needs: each softmax
+          // warp arrives on p_full(q) only after it has read P V(q-2) out of
+          // this TMEM buffer, and after S(q), which was issued once the
+          // stage's K and V had landed
+          ok = wait_or_abort(&sm.p_full[a], (gp >> 1) & 1, ctx, abort_flag);
           if (!ok) break;
           tc_fence_after();
           const uint32_t v_addr = smem_u32(sKV + st * kStageBytes + kPairBytes);
@@ -543,9 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float pv[kHH];
           tmem_ld8(lane_addr + 32 + a * 16, pv);
           tmem_ld_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.pv_empty[a]);
+          tc_fence_before();  // orders this read before P(q+2), see the P V issuer
 #pragma unroll
           for (int h = 0; h < kHH; ++h) o[h] = o[h] * alpha_prev[h] + pv[h];
         }
@@ -625,13 +624,8 @@ int launch_attn_g(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMa
                   const AttnArgs& args, int64_t n_items, const DevCtx& ctx, cudaStream_t st) {
   const size_t smem =
       1024 + kStages * kStageBytes + 2 * kQBytes + 2 * kPBytes + sizeof(AttnSmem);
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(sparse_attn_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return INFLLMV2_ERR_CUDA;
-    configured = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  if (int e = set_smem_limit(sparse_attn_kernel<G>, smem, smem_set)) return e;
   const int64_t grid = n_items < sm_count() ? n_items : sm_count();
   sparse_attn_kernel<G><<<static_cast<unsigned>(grid), kThreads, smem, st>>>(tq, tk, tv, args, ctx);
   return cudaGetLastError() == cudaSuccess ? INFLLMV2_OK : INFLLMV2_ERR_CUDA;
