@@ -57,16 +57,18 @@ constexpr int kPairBytes = 2 * kHalf;                // K or V of one pair: 32 K
 constexpr int kStageBytes = 2 * kPairBytes;          // K then V of one pair: 64 KB
 constexpr int kQBytes = 16 * 256;                    // 16 rows x 128 channels
 constexpr int kPBytes = 16 * 256;                    // 16 heads x 128 keys
+constexpr int kSBufs = 4;                            // S^T TMEM buffers (pair q uses q % 4)
 constexpr int kSoftmaxThreads = 128 * kHalves;
 constexpr int kThreads = 96 + kSoftmaxThreads;       // producer, S issuer, P V issuer, softmax
-constexpr uint32_t kTmemCols = 64;                   // S^T x2, PV x2 (16 columns each)
+constexpr uint32_t kTmemCols = 128;                  // S^T x4 (cols 0-63), PV x2 (64-95)
+constexpr uint32_t kPVCol = 64;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleSlack = 8.0f;                // log2 units
 
 struct AttnSmem {
   uint64_t full[kStages], empty[kStages];
   uint64_t q_full[2], q_empty[2];
-  uint64_t s_full[2], s_empty[2];
+  uint64_t s_full[kSBufs];
   uint64_t p_full[2];
   uint64_t pv_full[2];
   uint64_t drain;
@@ -240,14 +242,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(&sm.q_full[a], 1);
       mbar_init(&sm.q_empty[a], 1);
-      mbar_init(&sm.s_full[a], 1);
       // softmax-side barriers take one arrival per warp: 256 per-thread
       // arrivals per barrier per pair cost shared-memory atomic bandwidth
       // that the copies into the K / V rings need
-      mbar_init(&sm.s_empty[a], kSoftmaxThreads / 32);
       mbar_init(&sm.p_full[a], kSoftmaxThreads / 32);
       mbar_init(&sm.pv_full[a], 1);
     }
+    for (int a = 0; a < kSBufs; ++a) mbar_init(&sm.s_full[a], 1);
     mbar_init(&sm.drain, 2);  // one commit from each MMA issuer
     sm.abort_flag = 0;
     fence_mbar_init();
@@ -386,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // B: P^T, MN-major, no swizzle: 8x8 core matrices of 128 B, heads
             // 0-7 / 8-15 128 B apart (SBO), 8-key groups 256 B apart (LBO)
             const uint64_t bd = smem_desc(p_addr + kk * 512, 256, 128, 0);
-            umma_bf16(tmem + 32 + a * 16, ad, bd, idesc_pv, kk > 0 ? 1u : 0u);
+            umma_bf16(tmem + kPVCol + a * 16, ad, bd, idesc_pv, kk > 0 ? 1u : 0u);
           }
           umma_commit(&sm.pv_full[a]);
           umma_commit(&sm.empty[st]);
@@ -397,9 +398,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t q_addr = smem_u32(sQ + qb * kQBytes);
         for (int p = 0; ok && p < item.n_pairs; ++p, ++gp) {
           const int st = static_cast<int>(gp % kStages);
-          const int a = static_cast<int>(gp & 1);
-          ok = wait_or_abort(&sm.full[st], (gp / kStages) & 1, ctx, abort_flag) &&
-               (gp < 2 || wait_or_abort(&sm.s_empty[a], ((gp >> 1) & 1) ^ 1, ctx, abort_flag));
+          // S(q) overwrites the TMEM buffer of S(q-4).  The stage of pair q
+          // is refilled only after P V(q-3) completed, which followed P(q-3),
+          // which every softmax warp wrote after reading S(q-3): the wait for
+          // the stage covers the buffer too.
+          const int a = static_cast<int>(gp % kSBufs);
+          ok = wait_or_abort(&sm.full[st], (gp / kStages) & 1, ctx, abort_flag);
           if (!ok) break;
           tc_fence_after();
           const uint32_t k_addr = smem_u32(sKV + st * kStageBytes);
@@ -464,8 +468,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int p = 0; p <= item.n_pairs; ++p) {
         float alpha[kHH];
         if (p < item.n_pairs) {
-          const int a = static_cast<int>(gp & 1);
-          if (!*abort_flag && !mbar_wait(&sm.s_full[a], (gp >> 1) & 1, ctx.wait_ns)) {
+          const int a = static_cast<int>(gp % kSBufs);
+          const int pb = static_cast<int>(gp & 1);
+          if (!*abort_flag && !mbar_wait(&sm.s_full[a], (gp / kSBufs) & 1, ctx.wait_ns)) {
             report_status(ctx.status, INFLLMV2_STATUS_TIMEOUT);
             *abort_flag = 1;
           }
@@ -474,8 +479,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld8(lane_addr + a * 16, x);
           tmem_ld_wait();
           tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.s_empty[a]);
           const int e = 2 * p + slot;
           const int blk = e < item.n ? (item.row ? sm.blocks[e] : item.e0 + e) : -1;
           const bool valid = blk >= 0 && blk * kBlock + krow <= item.t;
@@ -527,10 +530,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
             pk[h >> 1] = *reinterpret_cast<uint32_t*>(&b2);
           }
-          *reinterpret_cast<uint4*>(sP + a * kPBytes + p_off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(sP + pb * kPBytes + p_off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.p_full[a]);
+          if (lane == 0) mbar_arrive(&sm.p_full[pb]);
         }
         if (p > 0) {
           // fold in P V of the previous pair
@@ -542,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           float pv[kHH];
-          tmem_ld8(lane_addr + 32 + a * 16, pv);
+          tmem_ld8(lane_addr + kPVCol + a * 16, pv);
           tmem_ld_wait();
           tc_fence_before();  // orders this read before P(q+2), see the P V issuer
 #pragma unroll
