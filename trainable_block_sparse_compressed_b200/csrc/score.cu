@@ -13,11 +13,15 @@
 // One CTA owns a 128-row query tile: 128/G consecutive tokens x the G heads
 // of one group, rows ordered (token, head) -- exactly the box a single TMA
 // load of the BSHD query tensor produces.  Compressed-key tiles of 128 rows
-// stream through a 2-stage TMA ring.  Both passes run the same tcgen05.mma
-// (M = N = 128, bf16 in, fp32 accumulate in tensor memory) over K = 2 x 128:
-// each compressed key is the bf16 pair hi + lo, so q . Kc = q . hi + q . lo
-// is accumulated in one tile (a single bf16 rounding of the keys would move
-// block scores by up to ~1e-2 relative):
+// stream through a 2-stage TMA ring.  Both passes run tcgen05.mma (M = N =
+// 128, bf16 in, fp32 accumulate in tensor memory).  Pass 2 runs over K =
+// 2 x 128: each compressed key is the bf16 pair hi + lo, so q . Kc = q . hi +
+// q . lo is accumulated in one tile (a single bf16 rounding of the keys would move
+// block scores by up to ~1e-2 relative).  Pass 1 only needs each row's
+// log-sum-exp, which scales all of that head's probabilities by one common
+// factor; the hi plane alone keeps that factor within ~2e-4 of exact (a fp64
+// emulation over the T=2048 and T=32768 workloads stays inside the selection
+// band on every row), so pass 1 reads and multiplies the hi plane only:
 //
 //   pass 1  D = Q  x Kc^T : a TMEM lane is a query row; each thread keeps the
 //           running max / sum of its row -> per-row LSE, no cross-lane work;
@@ -137,9 +141,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             !wait_or_abort(&sm.kc_empty[s], ((it / kStages) & 1) ^ 1, ctx, abort_flag))
           break;
         uint8_t* dst = sKc + s * kKcBytes;
-        mbar_arrive_expect_tx(&sm.kc_full[s], kKcBytes);
-#pragma unroll
-        for (int x = 0; x < 4; ++x)  // hi d[0:64], hi d[64:128], lo d[0:64], lo d[64:128]
+        // pass 1 needs the hi plane only, pass 2 hi and lo
+        const int nbox = it < n_t ? 2 : 4;
+        mbar_arrive_expect_tx(&sm.kc_full[s], nbox * kHalfBytes);
+        for (int x = 0; x < nbox; ++x)  // hi d[0:64], hi d[64:128], lo d[0:64], lo d[64:128]
           tma_load_4d(dst + x * kHalfBytes, &tmKc, &sm.kc_full[s], 64 * x, g, i * kKcTile, b);
         ++issued;
       }
@@ -165,9 +170,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t kc_addr = smem_u32(sKc + s * kKcBytes);
         const bool pass1 = it < n_t;
-        // q . Kc = q . hi + q . lo: K = 2 x 128, the query tile used twice
+        // pass 2: q . Kc = q . hi + q . lo, K = 2 x 128 with the query tile
+        // used twice; pass 1: q . hi, K = 128
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
+          if (pass1 && k >= 8) break;
           const uint32_t off = ((k >> 2) & 1) * kHalfBytes + (k & 3) * 32;
           const uint64_t qd = smem_desc(q_addr + off, 16, 1024, 2);
           const uint64_t kd = smem_desc(kc_addr + (k >> 3) * kTileBytes + off, 16, 1024, 2);

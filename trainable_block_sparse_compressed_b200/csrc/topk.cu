@@ -1,6 +1,7 @@
 // topk.cu -- prefill block selection: one warp per (batch, kv head, token)
 // row of the causally packed block-score workspace (see topk.cuh for the
-// selection rule).
+// selection rule).  Each warp holds as few keys per lane as its own row
+// needs (row t has t/64 + 1 blocks), up to VPL.
 #include "common.cuh"
 #include "topk.cuh"
 
@@ -17,7 +18,18 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ sco
   const int t = static_cast<int>(row % T);
   const int64_t bg = row / T;
   const float* srow = scores + bg * score_row_offset(T) + score_row_offset(t);
-  warp_select_row<VPL>(srow, t / kBlock, topk, n_init, n_local, idx + row * topk);
+  const int cur = t / kBlock;
+  int32_t* orow = idx + row * topk;
+  if (VPL > 4 && cur < 32 * 4)
+    warp_select_row<4>(srow, cur, topk, n_init, n_local, orow);
+  else if (VPL > 16 && cur < 32 * 16)
+    warp_select_row<16>(srow, cur, topk, n_init, n_local, orow);
+  else if (VPL > 32 && cur < 32 * 32)
+    warp_select_row<32>(srow, cur, topk, n_init, n_local, orow);
+  else if (VPL > 64 && cur < 32 * 64)
+    warp_select_row<64>(srow, cur, topk, n_init, n_local, orow);
+  else
+    warp_select_row<VPL>(srow, cur, topk, n_init, n_local, orow);
 }
 
 }  // namespace
