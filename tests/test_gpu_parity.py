@@ -457,3 +457,38 @@ def test_decode_exact_ties_go_to_lower_blocks(cuda_lib):
         assert np.abs(f64(O) - O_ref).max() <= O_ATOL
         assert np.abs(f64(lse) - L_ref).max() <= LSE_ATOL
     assert api.get_status() == 0
+
+
+@pytest.mark.parametrize("G", [1, 4, 8])
+def test_decode_small_groups(cuda_lib, G):
+    """Decode with GQA groups smaller than 16 heads: the scoring product pads
+    the query side to 16 rows and must use only the group's G columns."""
+    import torch
+    api = cuda_lib
+    Hkv = 2
+    w = wl.Workload(f"decode_G{G}", B=2, T=2500, Hq=G * Hkv, Hkv=Hkv, topk=12, seed=40 + G,
+                    decode_steps=6, needles_per_seq=2)
+    B, L0, steps = w.B, w.T, w.decode_steps
+    data, p, Kc, Vc, Kcmp, seqlens, ws = _decode_setup(api, w, L0, steps, B)
+    op = orc.Params(topk=w.topk)
+    st = orc.DecodeState.from_prefill(wl.bf16_to_f64(data["K0"]), wl.bf16_to_f64(data["V0"]), op)
+    O = torch.empty((B, w.Hq, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, w.Hq), dtype=torch.float32, device="cuda")
+    idx = torch.empty((B, Hkv, w.topk), dtype=torch.int32, device="cuda")
+    for s in range(steps):
+        api.decode_step(p, gpu_bf16(data["q"][s]), gpu_bf16(data["k_new"][s]),
+                        gpu_bf16(data["v_new"][s]), Kc, Vc, Kcmp, seqlens, O, lse, idx, ws)
+        torch.cuda.synchronize()
+        qf = wl.bf16_to_f64(data["q"][s])
+        O_ref, L_ref, i_ref = orc.decode_step(st, qf, wl.bf16_to_f64(data["k_new"][s]),
+                                              wl.bf16_to_f64(data["v_new"][s]), op)
+        gi, Og, Lg = idx.cpu().numpy(), f64(O), f64(lse)
+        for b in range(B):
+            for g in range(Hkv):
+                r = orc.select_query(qf[b, g * G:(g + 1) * G], st.Kc[b][:, g], L0 + s, op)
+                check_selection_row(r, gi[b, g], w.topk)
+                if np.array_equal(gi[b, g], i_ref[b, g]):
+                    hs = slice(g * G, (g + 1) * G)
+                    assert np.abs(Og[b, hs] - O_ref[b, hs]).max() <= O_ATOL
+                    assert np.abs(Lg[b, hs] - L_ref[b, hs]).max() <= LSE_ATOL
+    assert api.get_status() == 0

@@ -124,8 +124,9 @@ __global__ void __launch_bounds__(32) decode_append_kernel(
 // swizzle) and the G query heads of the group into a 2-stage ring; warp 1
 // issues D[128 keys x 16 heads] = Kc . q^T with tcgen05.mma over K = 256
 // (q . hi + q . lo: the query tile is the B operand of both halves) into a
-// double-buffered TMEM accumulator; warps 2-5 (thread = key) write the scaled
-// scores x[j, h] and each tile's per-head max and sum of exp2, which the
+// TMEM accumulator (4 buffers); warps 2-9, two warpgroups taking alternate
+// tiles (thread = key), write the scaled scores x[j, h] and each tile's
+// per-head max and sum of exp2, which the
 // select kernel merges into the head's log-sum-exp.  Units past the visible
 // keys of their sequence are skipped by all roles alike.
 constexpr int kDStages = 3;
@@ -133,15 +134,18 @@ constexpr int kDHalf = kScoreTile * 64 * 2;       // 128 rows x 64 channels: 16 
 constexpr int kDKcBytes = 4 * kDHalf;             // hi and lo planes: 64 KB
 constexpr int kDQBytes = 2 * 16 * 128;            // 16 head rows x 2 halves of 64 channels
 constexpr int kDStageBytes = kDKcBytes + kDQBytes;  // 68 KB (a multiple of 1 KB)
-constexpr int kDThreads = 192;
+constexpr int kDAcc = 4;                          // TMEM accumulators (16 columns each)
+constexpr int kDThreads = 64 + 256;               // producer, MMA, two epilogue warpgroups
 
 struct DScoreSmem {
   uint64_t full[kDStages], empty[kDStages];
-  uint64_t acc_full[2], acc_empty[2];
+  uint64_t acc_full[kDAcc], acc_empty[kDAcc];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
-  float xs[kScoreTile][17];  // the tile's scaled scores, transposed for the per-head reductions
+  // per epilogue warpgroup: the tile's scaled scores, transposed for the
+  // per-head reductions
+  float xs[2][kScoreTile][17];
 };
 
 struct DUnit {
@@ -198,16 +202,16 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_score_kernel(
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < kDAcc; ++a) {
       mbar_init(&sm.acc_full[a], 1);
-      mbar_init(&sm.acc_empty[a], 4);  // one arrival per epilogue warp
+      mbar_init(&sm.acc_empty[a], 4);  // one arrival per warp of the owning warpgroup
     }
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(&sm.tmem_base, 32);
+    tmem_alloc(&sm.tmem_base, kDAcc * 16);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -246,9 +250,9 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_score_kernel(
       for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
         const DUnit d = decode_unit(u, seq, Hkv, NC, n_tpb, Lmax);
         if (!d.active) continue;
-        const int s = n % kDStages, a = n & 1;
+        const int s = n % kDStages, a = n % kDAcc;
         if (!dwait(&sm.full[s], (n / kDStages) & 1, ctx, abort_flag)) break;
-        if (n >= 2 && !dwait(&sm.acc_empty[a], ((n >> 1) & 1) ^ 1, ctx, abort_flag)) break;
+        if (n >= kDAcc && !dwait(&sm.acc_empty[a], ((n / kDAcc) & 1) ^ 1, ctx, abort_flag)) break;
         tc_fence_after();
         const uint32_t kc_addr = smem_u32(base + s * kDStageBytes);
         const uint32_t q_addr = kc_addr + kDKcBytes;
@@ -268,24 +272,33 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_score_kernel(
       mbar_wait(&sm.drain, 0, ctx.wait_ns);
     }
   } else {
+    // two warpgroups take the active tiles alternately (tile n -> warpgroup
+    // n & 1, accumulator n % 4); each synchronises only within itself
+    const int wg = (warp - 2) >> 2;
     const int quad = warp & 3;
-    const int ew = warp - 2;            // epilogue warp 0..3 (heads ew, ew+4, ...)
+    const int ew = warp & 3;            // warp within the warpgroup (heads ew, ew+4, ...)
     const int r = quad * 32 + lane;     // TMEM lane = key within the tile
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-    int n = 0;
-    for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
+    const uint32_t bar_sync = 1 + 2 * wg, bar_or = 2 + 2 * wg;
+    float (*xs)[17] = sm.xs[wg];
+    int n = 0, k = 0;  // active tiles seen, units seen
+    for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x, ++k) {
       const DUnit d = decode_unit(u, seq, Hkv, NC, n_tpb, Lmax);
       float* mlo = ml + (static_cast<int64_t>(d.bg) * n_tpb + d.tile) * G * 2;
       if (!d.active) {
-        if (r < G) {
+        if (wg == (k & 1) && r < G) {
           mlo[2 * r] = -INFINITY;
           mlo[2 * r + 1] = 0.f;
         }
         continue;
       }
-      const int a = n & 1;
-      const bool ok = !*abort_flag && mbar_wait(&sm.acc_full[a], (n >> 1) & 1, ctx.wait_ns);
-      if (named_bar_or(2, 128, !ok)) {
+      const int mine = (n & 1) == wg;
+      const int a = n % kDAcc;
+      const int use = n / kDAcc;  // earlier uses of accumulator a
+      ++n;
+      if (!mine) continue;
+      const bool ok = !*abort_flag && mbar_wait(&sm.acc_full[a], use & 1, ctx.wait_ns);
+      if (named_bar_or(bar_or, 128, !ok)) {
         if (!ok) report_status(ctx.status, INFLLMV2_STATUS_TIMEOUT);
         *abort_flag = 1;
         break;
@@ -314,33 +327,53 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_score_kernel(
         }
       }
       // per-head max and sum of exp2 over the tile's keys: transpose through
-      // shared memory, then warp ew reduces heads ew, ew+4, ... (4 keys per lane)
+      // shared memory, then warp ew reduces heads ew, ew+4, ... (4 keys per
+      // lane), all of its heads' shuffle chains interleaved
 #pragma unroll
-      for (int h = 0; h < G; ++h) sm.xs[r][h] = x[h];
-      named_bar_sync(1, 128);
-      for (int h = ew; h < G; h += 4) {
-        float v[4];
+      for (int h = 0; h < G; ++h) xs[r][h] = x[h];
+      named_bar_sync(bar_sync, 128);
+      constexpr int kHW = (G + 3) / 4;  // heads per warp
+      float v[kHW][4], M[kHW], L[kHW];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = sm.xs[lane + 32 * i][h];
-        const float M = warp_max(fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3])));
-        float L = 0.f;
-        if (M > -INFINITY)
-          L = warp_sum(fast_exp2(v[0] - M) + fast_exp2(v[1] - M) + fast_exp2(v[2] - M) +
-                       fast_exp2(v[3] - M));
-        if (lane == 0) {
-          mlo[2 * h] = M;
-          mlo[2 * h + 1] = L;
+      for (int i = 0; i < kHW; ++i) {
+        const int h = ew + 4 * i;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) v[i][c] = h < G ? xs[lane + 32 * c][h] : -INFINITY;
+        M[i] = fmaxf(fmaxf(v[i][0], v[i][1]), fmaxf(v[i][2], v[i][3]));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+        for (int i = 0; i < kHW; ++i) M[i] = fmaxf(M[i], __shfl_xor_sync(0xffffffffu, M[i], o));
+      }
+#pragma unroll
+      for (int i = 0; i < kHW; ++i)
+        L[i] = M[i] > -INFINITY ? fast_exp2(v[i][0] - M[i]) + fast_exp2(v[i][1] - M[i]) +
+                                      fast_exp2(v[i][2] - M[i]) + fast_exp2(v[i][3] - M[i])
+                                : 0.f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+        for (int i = 0; i < kHW; ++i) L[i] += __shfl_xor_sync(0xffffffffu, L[i], o);
+      }
+      if (lane == 0) {
+#pragma unroll
+        for (int i = 0; i < kHW; ++i) {
+          const int h = ew + 4 * i;
+          if (h < G) {
+            mlo[2 * h] = M[i];
+            mlo[2 * h + 1] = L[i];
+          }
         }
       }
-      named_bar_sync(1, 128);  // xs is rewritten by the next unit
-      ++n;
+      named_bar_sync(bar_sync, 128);  // xs is rewritten by this warpgroup's next tile
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 32);
+    tmem_dealloc(tmem, kDAcc * 16);
   }
 }
 
