@@ -170,7 +170,8 @@ def attended_keys(idx_np, T):
 # ---------------------------------------------------------------------------
 # our implementation
 # ---------------------------------------------------------------------------
-def run_prefill(api, wl, w, steps, warmup, dist, flush, time_e2e=True, clocks=None):
+def run_prefill(api, wl, w, steps, warmup, dist, flush, time_e2e=True, clocks=None,
+                chunk_len=0):
     import numpy as np
     import torch
     data = wl.make_prefill(w)
@@ -245,11 +246,43 @@ def run_prefill(api, wl, w, steps, warmup, dist, flush, time_e2e=True, clocks=No
                useful_attn_flops=useful_attn_flops, useful_score_flops=useful_score_flops,
                executed_score_flops=executed_score_flops, executed_attn_flops=executed_attn_flops,
                clocks=clk, launches_per_step=5)
+    if chunk_len:
+        out["chunk"] = time_chunk(api, p, Q, K, V, Kc, chunk_len, steps, warmup, flush)
     if time_e2e:
         out.update(e2e_prefill(api, p, Qh, Kh, Vh, O.shape, lse.shape, Kc, idx, ws, steps, dist))
     del Q, K, V, Kc, idx, ws, O, lse
     torch.cuda.empty_cache()
     return out
+
+
+def time_chunk(api, p, Q, K, V, Kc, n, steps, warmup, flush):
+    """Chunked prefill: the last n tokens' queries over the sequence's full
+    caches (K, V and the compressed keys the main step computed)."""
+    import torch
+    B, T, Hq = Q.shape[0], Q.shape[1], Q.shape[2]
+    q0 = T - n
+    Qc = Q[:, q0:].contiguous()
+    O = torch.empty_like(Qc)
+    lse = torch.empty((B, Hq, n), dtype=torch.float32, device="cuda")
+    idx = torch.empty((B, p.Hkv, n, p.topk), dtype=torch.int32, device="cuda")
+    ws = torch.empty(api.prefill_chunk_workspace_bytes(p, q0, n), dtype=torch.uint8,
+                     device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        flush()
+        api.prefill_chunk(p, q0, n, Qc, K, V, Kc, O, lse, idx, ws)
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(steps):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        api.prefill_chunk(p, q0, n, Qc, K, V, Kc, O, lse, idx, ws)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    assert api.get_status() == 0
+    return dict(q_offset=q0, q_len=n, ms=sum(ms) / len(ms))
 
 
 def e2e_prefill(api, p, Qh, Kh, Vh, o_shape, lse_shape, Kc, idx, ws, steps, dist):
@@ -468,12 +501,20 @@ def main():
         flush_buf.zero_()
 
     clocks = ClockSampler(dist.local)
-    main_r = run_prefill(api, wl, w, args.steps, args.warmup, dist, flush, True, clocks)
+    main_r = run_prefill(api, wl, w, args.steps, args.warmup, dist, flush, True, clocks,
+                         chunk_len=0 if args.no_extras else 8192)
     ms = dist.max(main_r["ms"])
     e2e_ms = dist.max(main_r["e2e_ms"])
     value = whole_job_rate(main_r["tokens"], dist.world, ms)
 
     extras = {}
+    if "chunk" in main_r:
+        c = main_r["chunk"]
+        cms = dist.max(c["ms"])
+        extras["prefill_chunk_T131072_last8192"] = {
+            "tokens_per_s": whole_job_rate(w.B * c["q_len"], dist.world, cms), "ms_per_chunk": cms,
+            "q_offset": c["q_offset"], "q_len": c["q_len"],
+            "timing": "queries of tokens 122880..131071 over the full caches; L2 flushed"}
     if not args.no_extras:
         side = run_prefill(api, wl, wl.WORKLOADS[SIDE], args.steps, args.warmup, dist, flush,
                            False, None)

@@ -169,6 +169,33 @@ int infllmv2_forward(const infllmv2_params* p, const void* Q, const void* K,
                      int32_t* path_used, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Chunked prefill: queries for the tokens q_offset .. q_offset+q_len-1 of a
+ * sequence whose keys, values and compressed keys are already in the caches
+ * (the chunk's own tokens included).  Each query row t gets exactly what
+ * infllmv2_forward gives row t of the whole sequence: the same switch (dense
+ * iff p->T <= p->switch_threshold), selection over the compressed keys
+ * visible at t and the blocks <= t/64, attention over keys <= t.  Serving
+ * splits a long prompt into such chunks (reportify digest, Performance
+ * Evaluation: prefill and decode over a growing cache).
+ *   p->T = q_offset + q_len: the tokens in the caches (INVALID_ARG otherwise);
+ *   Q [B, q_len, Hq, d] bf16 (in); K, V [B, T, Hkv, d] bf16 (in);
+ *   Kc [B, n_c(T), Hkv, 2, d] bf16 (in: compressed keys of the caches, e.g. from
+ *     infllmv2_compress_keys or the decode steps' appends; unused when dense);
+ *   O [B, q_len, Hq, d] bf16, lse [B, Hq, q_len] fp32 (out);
+ *   idx [B, Hkv, q_len, topk] int32 (out; unused and may be NULL when dense);
+ *   path_used: host int32 (may be NULL);
+ *   ws: at least infllmv2_prefill_chunk_workspace_bytes(p, q_offset, q_len)
+ *     bytes (dense: may be smaller, down to 0; the K/V gather then uses
+ *     tensor-map boxes instead of packed tiles).
+ */
+size_t infllmv2_prefill_chunk_workspace_bytes(const infllmv2_params* p, int32_t q_offset,
+                                              int32_t q_len);
+int infllmv2_prefill_chunk(const infllmv2_params* p, int32_t q_offset, int32_t q_len,
+                           const void* Q, const void* K, const void* V, const void* Kc,
+                           void* O, float* lse, int32_t* idx, int32_t* path_used, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/*
  * One decode step for B sequences (reportify digest, Performance Evaluation:
  * the operator speed-up is reported for both prefill and decode).  p->T is the cache
  * capacity Lmax in tokens; the compressed-key cache holds n_c(Lmax) rows.

@@ -331,6 +331,44 @@ def forward(Q, K, V, p: Params, rows=None):
     return O, L, "sparse", idx
 
 
+def chunk_forward(Qc, K, V, q0: int, p: Params, rows=None):
+    """Chunked prefill: the queries Qc [B, Tq, Hq, d] are tokens q0 .. q0+Tq-1
+    of sequences whose keys and values K, V [B, q0+Tq, Hkv, d] are all known.
+    Row i is what forward() gives token q0+i of the whole sequence: the same
+    length switch on T = q0+Tq, selection over the compressed keys visible at
+    t = q0+i and blocks <= t/64, attention over keys <= t.
+
+    Returns (O [B, Tq, Hq, d], LSE [B, Hq, Tq], path, idx [B, Hkv, Tq, topk]
+    or None); ``rows``: optional list of (b, g, i).
+    """
+    B, Tq, Hq, d = Qc.shape
+    T = K.shape[1]
+    assert T == q0 + Tq
+    Hkv = K.shape[2]
+    G = Hq // Hkv
+    if rows is None:
+        rows = [(b, g, i) for b in range(B) for g in range(Hkv) for i in range(Tq)]
+    dense = uses_dense(T, p)
+    Kc = None if dense else compress_keys(K, p)
+    O = np.full((B, Tq, Hq, d), np.nan)
+    L = np.full((B, Hq, Tq), np.nan)
+    idx = None if dense else np.full((B, Hkv, Tq, p.topk), -1, dtype=np.int32)
+    sc = p.sm_scale(d)
+    for (b, g, i) in rows:
+        t = q0 + i
+        qg = Qc[b, i, g * G:(g + 1) * G]
+        if dense:
+            keys = np.arange(t + 1)
+        else:
+            r = select_query(qg, Kc[b, :, g, :], t, p)
+            idx[b, g, i] = r.idx
+            keys = selected_keys(r.idx, t, p)
+        o, lse = attend(qg, K[b, :, g], V[b, :, g], keys, sc)
+        O[b, i, g * G:(g + 1) * G] = o
+        L[b, g * G:(g + 1) * G, i] = lse
+    return O, L, ("dense" if dense else "sparse"), idx
+
+
 # --------------------------------------------------------------------------
 # decode: one new token per sequence
 # --------------------------------------------------------------------------

@@ -106,3 +106,30 @@ def test_empty_problems_are_noops(lib):
     p = api.make_params(1, 0, 32, 2, topk=8)
     assert lib.infllmv2_sparse_attn(ctypes.byref(p), None, None, None, None, None, None, None, 0,
                                     None) == api.OK
+
+
+def test_prefill_chunk_rejected_on_host(lib):
+    p = api.make_params(1, 1000, 32, 2, topk=8, switch_threshold=0)
+    P = ctypes.byref(p)
+    args = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, None)
+    # the chunk must end at p->T
+    assert lib.infllmv2_prefill_chunk(P, 400, 500, *args) == api.ERR_INVALID_ARG
+    assert lib.infllmv2_prefill_chunk(P, -1, 1001, *args) == api.ERR_INVALID_ARG
+    assert lib.infllmv2_prefill_chunk(P, 400, 600, FAKE + 8, *args[1:]) == api.ERR_UNSUPPORTED
+    assert lib.infllmv2_prefill_chunk(P, 1000, 0, *args) == api.OK  # no queries
+    with pytest.raises(api.InfLLMV2Error):
+        api.prefill_chunk_workspace_bytes(p, 10, 10)
+
+
+def test_prefill_chunk_workspace_sizes(lib):
+    p = api.make_params(1, 131072, 32, 2, topk=64, switch_threshold=8192)
+    # the whole sequence as one chunk needs what forward needs
+    assert api.prefill_chunk_workspace_bytes(p, 0, 131072) == api.workspace_bytes(p, api.OP_FORWARD)
+    # a tail chunk: the block scores of its rows only, then the packed K/V of all tokens
+    q0, n = 131072 - 4096, 4096
+    rows = sum(t // 64 + 1 for t in range(q0, q0 + n))
+    sel = 2 * rows * 4
+    assert api.prefill_chunk_workspace_bytes(p, q0, n) == \
+        (-(-sel // 256) * 256) + api.workspace_bytes(p, api.OP_ATTN)
+    d = api.make_params(1, 4096, 32, 2, switch_threshold=8192)
+    assert api.prefill_chunk_workspace_bytes(d, 1000, 3096) == api.workspace_bytes(d, api.OP_ATTN)

@@ -492,3 +492,92 @@ def test_decode_small_groups(cuda_lib, G):
                     assert np.abs(Og[b, hs] - O_ref[b, hs]).max() <= O_ATOL
                     assert np.abs(Lg[b, hs] - L_ref[b, hs]).max() <= LSE_ATOL
     assert api.get_status() == 0
+
+
+# ---------------------------------------------------------------------------
+# chunked prefill over existing caches
+# ---------------------------------------------------------------------------
+CHUNKS = [
+    # (B, T, Hq, Hkv, topk, q0, threshold)
+    (1, 2000, 32, 2, 8, 1000, 0),     # unaligned chunk start, G = 16
+    (2, 1400, 8, 2, 6, 640, 0),       # block-aligned start, G = 4, two sequences
+    (1, 1100, 16, 1, 5, 1093, 0),     # a 7-token chunk
+    (1, 3000, 32, 2, 64, 2048, 8192), # dense: the sequence is below the threshold
+]
+
+
+def _run_chunk(api, B, T, Hq, Hkv, topk, q0, threshold, seed):
+    import torch
+    w = wl.small_workload(B=B, T=T, Hq=Hq, Hkv=Hkv, topk=topk, needles=2, seed=seed,
+                          threshold=threshold)
+    data = wl.make_prefill(w)
+    p = _params(api, w)
+    Q, K, V = gpu_bf16(data["Q"]), gpu_bf16(data["K"]), gpu_bf16(data["V"])
+    n_c = api.num_compressed(T)
+    Kc = torch.empty((B, max(n_c, 1), Hkv, 2, 128), dtype=torch.bfloat16, device="cuda")
+    if n_c:
+        api.compress_keys(p, K, Kc)
+    Tq = T - q0
+    Qc = Q[:, q0:].contiguous()
+    O = torch.empty_like(Qc)
+    lse = torch.empty((B, Hq, Tq), dtype=torch.float32, device="cuda")
+    idx = torch.full((B, Hkv, Tq, topk), -7, dtype=torch.int32, device="cuda")
+    ws = torch.empty(api.prefill_chunk_workspace_bytes(p, q0, Tq), dtype=torch.uint8,
+                     device="cuda")
+    path = api.prefill_chunk(p, q0, Tq, Qc, K, V, Kc, O, lse, idx, ws)
+    torch.cuda.synchronize()
+    assert api.get_status() == 0
+    return w, data, (Q, K, V, Kc), path, f64(O), f64(lse), idx.cpu().numpy()
+
+
+@pytest.mark.parametrize("case", CHUNKS, ids=[f"B{c[0]}_T{c[1]}_q0_{c[5]}_thr{c[6]}" for c in CHUNKS])
+def test_prefill_chunk_against_the_oracle(cuda_lib, case):
+    B, T, Hq, Hkv, topk, q0, threshold = case
+    w, data, _, path, Og, Lg, ig = _run_chunk(cuda_lib, *case, seed=50 + q0)
+    Qf, Kf, Vf = (wl.bf16_to_f64(data[x]) for x in "QKV")
+    op = _oparams(w)
+    O_ref, L_ref, path_ref, idx_ref = orc.chunk_forward(Qf[:, q0:], Kf, Vf, q0, op)
+    assert path == (cuda_lib.PATH_DENSE if path_ref == "dense" else cuda_lib.PATH_SPARSE)
+    G = Hq // Hkv
+    sc = op.sm_scale(128)
+    if path_ref == "sparse":
+        Kc = orc.compress_keys(Kf, op)
+        for b in range(B):
+            for g in range(Hkv):
+                for i in range(T - q0):
+                    t = q0 + i
+                    r = orc.select_query(Qf[b, t, g * G:(g + 1) * G], Kc[b, :, g], t, op)
+                    check_selection_row(r, ig[b, g, i], topk)
+    for b in range(B):
+        for g in range(Hkv):
+            hs = slice(g * G, (g + 1) * G)
+            for i in range(T - q0):
+                t = q0 + i
+                if path_ref == "sparse":
+                    keys = orc.selected_keys(ig[b, g, i], t, op)  # the GPU's own selection
+                else:
+                    keys = np.arange(t + 1)
+                o, l = orc.attend(Qf[b, t, hs], Kf[b, :, g], Vf[b, :, g], keys, sc)
+                assert np.abs(Og[b, i, hs] - o).max() <= O_ATOL
+                assert np.abs(Lg[b, hs, i] - l).max() <= LSE_ATOL
+
+
+def test_prefill_chunk_equals_the_whole_sequence_rows(cuda_lib):
+    """The chunk's rows are bit-identical to the same rows of a whole-sequence
+    forward on the GPU: every row's arithmetic is independent of how the
+    queries are grouped into tiles."""
+    import torch
+    api = cuda_lib
+    B, T, Hq, Hkv, topk, q0 = 1, 3000, 32, 2, 16, 1337
+    w, data, (Q, K, V, Kc), path, Og, Lg, ig = _run_chunk(api, B, T, Hq, Hkv, topk, q0, 0, 77)
+    p = _params(api, w)
+    O = torch.empty_like(Q)
+    lse = torch.empty((B, Hq, T), dtype=torch.float32, device="cuda")
+    idx = torch.empty((B, Hkv, T, topk), dtype=torch.int32, device="cuda")
+    Kc2 = torch.empty_like(Kc)
+    ws = api.alloc_workspace(p, api.OP_FORWARD)
+    assert api.forward(p, Q, K, V, O, lse, Kc2, idx, ws) == api.PATH_SPARSE
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy()[:, :, q0:], ig)
+    assert np.array_equal(f64(O)[:, q0:], Og)
+    assert np.array_equal(f64(lse)[:, :, q0:], Lg)

@@ -401,3 +401,21 @@ def test_planted_oracle_mistakes_are_caught(monkeypatch, attr, bad):
         except (AssertionError, IndexError, ValueError):
             caught += 1
     assert caught >= 1, f"no golden pin caught a broken {attr}"
+
+
+@pytest.mark.parametrize("q0,Tq,threshold", [(0, 700, 0), (300, 400, 0), (333, 367, 0),
+                                              (640, 60, 0), (500, 200, 8192)])
+def test_chunk_forward_equals_the_whole_sequence_rows(q0, Tq, threshold):
+    """A chunk of queries over the full caches gives exactly the rows q0..q0+Tq-1
+    of the whole-sequence forward (sparse and dense), including the selection."""
+    w = wl.small_workload(B=2, T=q0 + Tq, Hq=8, Hkv=2, topk=5, needles=1, seed=31,
+                          threshold=threshold)
+    d = wl.make_prefill(w)
+    Q, K, V = (wl.bf16_to_f64(d[x]) for x in "QKV")
+    p = orc.Params(topk=w.topk, n_init=w.n_init, n_local=w.n_local, threshold=threshold)
+    O, L, path, idx = orc.forward(Q, K, V, p)
+    Oc, Lc, path_c, idx_c = orc.chunk_forward(Q[:, q0:], K, V, q0, p)
+    assert path_c == path
+    assert np.array_equal(Oc, O[:, q0:]) and np.array_equal(Lc, L[:, :, q0:])
+    if idx is not None:
+        assert np.array_equal(idx_c, idx[:, :, q0:])

@@ -81,6 +81,8 @@ int validate(const infllmv2_params* p, bool needs_topk, Geometry* g) {
   if (static_cast<int64_t>(p->T) > (1 << 22)) return INFLLMV2_ERR_UNSUPPORTED;
   g->B = p->B;
   g->T = p->T;
+  g->q0 = 0;
+  g->Tq = p->T;
   g->Hq = p->Hq;
   g->Hkv = p->Hkv;
   g->G = G;
@@ -118,9 +120,21 @@ int check_ptrs(std::initializer_list<const void*> ptrs) {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Block scores of the query rows q0 .. q0+Tq-1 (causally packed).
 size_t select_ws_bytes(const Geometry& g) {
-  return static_cast<size_t>(g.B) * g.Hkv * static_cast<size_t>(score_row_offset(g.T)) *
+  return static_cast<size_t>(g.B) * g.Hkv *
+         static_cast<size_t>(score_row_offset(g.q0 + g.Tq) - score_row_offset(g.q0)) *
          sizeof(float);
+}
+
+// validate() plus the query range of a prefill chunk.
+int validate_chunk(const infllmv2_params* p, int32_t q_offset, int32_t q_len, Geometry* g) {
+  if (int e = validate(p, true, g)) return e;
+  if (q_offset < 0 || q_len < 0 || static_cast<int64_t>(q_offset) + q_len != p->T)
+    return INFLLMV2_ERR_INVALID_ARG;
+  g->q0 = q_offset;
+  g->Tq = q_len;
+  return INFLLMV2_OK;
 }
 
 int ctx_or_error(DevCtx* ctx) {
@@ -245,6 +259,46 @@ int infllmv2_forward(const infllmv2_params* p, const void* Q, const void* K, con
   if (int e = infllmv2_select_blocks(p, Q, Kc_ws, idx_ws, ws, ws_bytes, stream)) return e;
   return infllmv2_sparse_attn(p, Q, K, V, idx_ws, O, lse, static_cast<uint8_t*>(ws) + sel,
                               ws_bytes - sel, stream);
+}
+
+size_t infllmv2_prefill_chunk_workspace_bytes(const infllmv2_params* p, int32_t q_offset,
+                                              int32_t q_len) {
+  Geometry g;
+  if (validate_chunk(p, q_offset, q_len, &g) != INFLLMV2_OK) return SIZE_MAX;
+  return p->T <= p->switch_threshold ? packed_kv_bytes(g)
+                                     : align256(select_ws_bytes(g)) + packed_kv_bytes(g);
+}
+
+int infllmv2_prefill_chunk(const infllmv2_params* p, int32_t q_offset, int32_t q_len,
+                           const void* Q, const void* K, const void* V, const void* Kc, void* O,
+                           float* lse, int32_t* idx, int32_t* path_used, void* ws,
+                           size_t ws_bytes, void* stream) {
+  Geometry g;
+  if (int e = validate_chunk(p, q_offset, q_len, &g)) return e;
+  const bool dense = p->T <= p->switch_threshold;
+  if (path_used) *path_used = dense ? INFLLMV2_PATH_DENSE : INFLLMV2_PATH_SPARSE;
+  if (g.B == 0 || g.Tq == 0) return INFLLMV2_OK;
+  if (int e = check_ptrs({Q, K, V, O, lse})) return e;
+  if (!dense) {
+    if (int e = check_ptrs({idx, ws})) return e;
+    if (g.n_c > 0)
+      if (int e = check_ptrs({Kc})) return e;
+  }
+  const size_t sel = dense ? 0 : align256(select_ws_bytes(g));
+  if (ws_bytes < sel) return INFLLMV2_ERR_WORKSPACE;
+  DevCtx ctx;
+  if (int e = ctx_or_error(&ctx)) return e;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!dense) {
+    if (int e = launch_score_blocks(g, Q, Kc, static_cast<float*>(ws), ctx, st)) return e;
+    if (int e = launch_topk(g, static_cast<float*>(ws), idx, st)) return e;
+  }
+  uint8_t* rest = ws ? static_cast<uint8_t*>(ws) + sel : nullptr;
+  const bool pack = rest && ws_bytes - sel >= packed_kv_bytes(g);
+  if (pack)
+    if (int e = launch_pack_kv(g, K, V, rest, st)) return e;
+  return launch_sparse_attn(g, Q, K, V, dense ? nullptr : idx, O, lse, dense ? 1 : 0,
+                            pack ? rest : nullptr, ctx, st);
 }
 
 int infllmv2_decode_step(const infllmv2_params* p, const void* q, const void* k_new,

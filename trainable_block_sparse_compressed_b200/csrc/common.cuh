@@ -29,7 +29,8 @@ constexpr int kKcRow = 2 * kHeadDim;  // elements per (window, kv head)
 
 // Everything a kernel needs about one call, resolved on the host.
 struct Geometry {
-  int B, T, Hq, Hkv, G;   // G = Hq / Hkv
+  int B, T, Hq, Hkv, G;   // G = Hq / Hkv; T: tokens of the sequence (keys)
+  int q0, Tq;             // the queries are tokens q0 .. q0+Tq-1 (prefill: 0, T)
   int n_c;                // compressed rows of T tokens
   int topk, n_init, n_local;
   float scale;            // softmax scale

@@ -79,7 +79,8 @@ template <int G>
 __global__ void __launch_bounds__(kThreads, 1)
     score_blocks_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmKc, float* __restrict__ scores,
-                        int B, int T, int Hkv, int n_c, float scale_log2, DevCtx ctx) {
+                        int B, int q0, int Tq, int Hkv, int n_c, float scale_log2,
+                        DevCtx ctx) {
   constexpr int TPT = kRows / G;  // tokens per tile
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -89,12 +90,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   ScoreSmem& sm = *reinterpret_cast<ScoreSmem*>(base + kTileBytes + kKcBytes * kStages);
 
   // heaviest (latest) query tiles first
-  const int n_qt = (T + TPT - 1) / TPT;
+  // queries are tokens q0 .. q0+Tq-1 (a whole prefill: q0 = 0); keys and
+  // compressed keys cover tokens 0 .. q0+Tq-1
+  const int q_end = q0 + Tq;
+  const int n_qt = (Tq + TPT - 1) / TPT;
   const int bg = blockIdx.x % (B * Hkv);
   const int qt = n_qt - 1 - static_cast<int>(blockIdx.x / (B * Hkv));
   const int b = bg / Hkv, g = bg % Hkv;
-  const int t0 = qt * TPT;
-  const int t_last = min(t0 + TPT - 1, T - 1);
+  const int t0 = q0 + qt * TPT;
+  const int t_last = min(t0 + TPT - 1, q_end - 1);
   const int v_max = min(n_c, visible_windows(t_last));
   const int n_t = (v_max + kKcTile - 1) / kKcTile;
   const int n_it = 2 * n_t;
@@ -131,8 +135,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmKc);
       mbar_arrive_expect_tx(&sm.q_full, kTileBytes);
-      tma_load_4d(sQ, &tmQ, &sm.q_full, 0, g * G, t0, b);
-      tma_load_4d(sQ + kHalfBytes, &tmQ, &sm.q_full, 64, g * G, t0, b);
+      tma_load_4d(sQ, &tmQ, &sm.q_full, 0, g * G, t0 - q0, b);
+      tma_load_4d(sQ + kHalfBytes, &tmQ, &sm.q_full, 64, g * G, t0 - q0, b);
       int issued = 0;
       for (int it = 0; it < n_it; ++it) {
         const int s = it % kStages;
@@ -200,7 +204,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;  // TMEM lane this thread reads
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + hf * 64;
-    const int64_t slab = score_row_offset(T);
+    // the queries' rows of the causally packed workspace, from row q0 on
+    const int64_t row0 = score_row_offset(q0);
+    const int64_t slab = score_row_offset(q_end) - row0;
     float* srow_base = scores + (static_cast<int64_t>(b) * Hkv + g) * slab;
     constexpr uint32_t bar_sync_all = 1, bar_or_all = 2;  // 256 threads
     const uint32_t bar_sync_half = 3 + hf;                // the 128 threads of this warpgroup
@@ -208,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // pass-1 row identity
     const int my_tok = r / G;
     const int my_t = t0 + my_tok;
-    const int my_v = my_t < T ? min(n_c, visible_windows(my_t)) : 0;
+    const int my_v = my_t < q_end ? min(n_c, visible_windows(my_t)) : 0;
     float m_run = -INFINITY, l_run = 0.f;
 
     for (int it = 0; it < n_it; ++it) {
@@ -275,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int tl = 0; tl < TPH; ++tl) {
           const int tok = hf * TPH + tl;
           const int t = t0 + tok;
-          const int v = t < T ? min(n_c, visible_windows(t)) : 0;
+          const int v = t < q_end ? min(n_c, visible_windows(t)) : 0;
           float acc = 0.f;
 #pragma unroll
           for (int h = 0; h < G; ++h)
@@ -303,8 +309,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           float prev = __shfl_up_sync(0xffffffffu, S[tl], 1);
           if (lane == 0) prev = sm.carry[cb][quad][tok];
           const int t = t0 + tok;
-          if ((lane & 3) == 0 && t < T && blk <= t / kBlock)
-            srow_base[score_row_offset(t) + blk] = fmaxf(m4, prev);
+          if ((lane & 3) == 0 && t < q_end && blk <= t / kBlock)
+            srow_base[score_row_offset(t) - row0 + blk] = fmaxf(m4, prev);
         }
       }
     }
@@ -313,10 +319,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!*abort_flag) {
       for (int tok = hf * TPH + r; tok < (hf + 1) * TPH; tok += 128) {
         const int t = t0 + tok;
-        if (t >= T) continue;
+        if (t >= q_end) continue;
         const int cur = t / kBlock;
         for (int blk = n_t * (kKcTile / 4); blk <= cur; ++blk)
-          srow_base[score_row_offset(t) + blk] =
+          srow_base[score_row_offset(t) - row0 + blk] =
               blk == n_t * (kKcTile / 4) ? sm.carry[n_t % 3][0][tok] : -INFINITY;
       }
     }
@@ -337,9 +343,9 @@ int launch_score_g(const Geometry& g, const CUtensorMap& tq, const CUtensorMap& 
   const size_t smem = 1024 + kTileBytes + kKcBytes * kStages + sizeof(ScoreSmem);
   static std::atomic<uint64_t> smem_set{0};
   if (int e = set_smem_limit(score_blocks_kernel<G>, smem, smem_set)) return e;
-  const int n_qt = (g.T + TPT - 1) / TPT;
+  const int n_qt = (g.Tq + TPT - 1) / TPT;
   const unsigned grid = static_cast<unsigned>(n_qt) * g.B * g.Hkv;
-  score_blocks_kernel<G><<<grid, kThreads, smem, st>>>(tq, tk, scores, g.B, g.T, g.Hkv, g.n_c,
+  score_blocks_kernel<G><<<grid, kThreads, smem, st>>>(tq, tk, scores, g.B, g.q0, g.Tq, g.Hkv, g.n_c,
                                                        g.scale_log2, ctx);
   return cudaGetLastError() == cudaSuccess ? INFLLMV2_OK : INFLLMV2_ERR_CUDA;
 }
@@ -348,15 +354,15 @@ int launch_score_g(const Geometry& g, const CUtensorMap& tq, const CUtensorMap& 
 
 int launch_score_blocks(const Geometry& g, const void* Q, const void* Kc, float* scores,
                         const DevCtx& ctx, cudaStream_t st) {
-  if (g.B == 0 || g.T == 0) return INFLLMV2_OK;
+  if (g.B == 0 || g.Tq == 0) return INFLLMV2_OK;
   const int TPT = kRows / g.G;
   CUtensorMap tq, tk;
   {
     const uint64_t dims[4] = {static_cast<uint64_t>(kHeadDim), static_cast<uint64_t>(g.Hq),
-                              static_cast<uint64_t>(g.T), static_cast<uint64_t>(g.B)};
+                              static_cast<uint64_t>(g.Tq), static_cast<uint64_t>(g.B)};
     const uint64_t strides[3] = {static_cast<uint64_t>(kHeadDim) * 2,
                                  static_cast<uint64_t>(g.Hq) * kHeadDim * 2,
-                                 static_cast<uint64_t>(g.T) * g.Hq * kHeadDim * 2};
+                                 static_cast<uint64_t>(g.Tq) * g.Hq * kHeadDim * 2};
     const uint32_t box[4] = {64u, static_cast<uint32_t>(g.G), static_cast<uint32_t>(TPT), 1u};
     if (int e = make_tmap_bf16_4d(&tq, Q, dims, strides, box)) return e;
   }

@@ -88,7 +88,8 @@ struct AttnArgs {
   float* lse;
   float* part;              // decode partials: [items][G][128] o, then [items][G][2] (m, l)
   const int32_t* seqlens;   // decode: query position of each sequence
-  int B, T, Hq, Hkv, topk;  // T: tokens (prefill) or cache capacity (decode)
+  int B, T, Hq, Hkv, topk;  // T: key tokens (prefill) or cache capacity (decode)
+  int q0, Tq;               // prefill: the queries are tokens q0 .. q0+Tq-1
   int mode;                 // 0 sparse prefill, 1 dense prefill, 2 decode
   int n_chunks, chunk_blocks;
   float scale_log2;
@@ -146,19 +147,19 @@ __device__ __forceinline__ Item resolve_item(int64_t it, const AttnArgs& a, int 
     r.e0 = c * a.chunk_blocks;
     r.n = max(0, min(a.chunk_blocks, nv - r.e0));
   } else {
-    const int64_t per_g = static_cast<int64_t>(a.B) * a.T;
+    const int64_t per_g = static_cast<int64_t>(a.B) * a.Tq;
     r.g = static_cast<int>(it / per_g);
     const int64_t rem = it % per_g;
-    r.b = static_cast<int>(rem / a.T);
-    r.t = static_cast<int>(rem % a.T);
-    r.qtok = r.t;
+    r.b = static_cast<int>(rem / a.Tq);
+    r.qtok = static_cast<int>(rem % a.Tq);  // the query's row in Q, O and lse
+    r.t = a.q0 + r.qtok;                    // its token position
     r.cur = r.t / kBlock;
     r.e0 = 0;
     if (a.mode == 1) {
       r.row = nullptr;
       r.n = r.cur + 1;
     } else {
-      r.row = a.idx + ((static_cast<int64_t>(r.b) * a.Hkv + r.g) * a.T + r.t) * a.topk;
+      r.row = a.idx + ((static_cast<int64_t>(r.b) * a.Hkv + r.g) * a.Tq + r.qtok) * a.topk;
       r.n = collective ? count_valid(r.row, a.topk, r.cur, lane)
                        : count_valid_1(r.row, a.topk, r.cur);
     }
@@ -214,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = warp_id(), lane = lane_id();
   const int64_t n_items = args.mode == 2
                               ? static_cast<int64_t>(args.B) * args.Hkv * args.n_chunks
-                              : static_cast<int64_t>(args.Hkv) * args.B * args.T;
+                              : static_cast<int64_t>(args.Hkv) * args.B * args.Tq;
   const float scale_log2 = args.scale_log2;
 
   // A pair with a single block leaves its second slot stale.  Stale K rows
@@ -588,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         const int64_t orow =
-            (static_cast<int64_t>(item.b) * args.T + item.t) * args.Hq + item.g * G;
+            (static_cast<int64_t>(item.b) * args.Tq + item.qtok) * args.Hq + item.g * G;
 #pragma unroll
         for (int h = 0; h < kHH; ++h) {
           if (h_begin + h < G) {
@@ -605,8 +606,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int h = 0; h < kHH; ++h)
             if (h == r) mr = m[h];
-          args.lse[(static_cast<int64_t>(item.b) * args.Hq + item.g * G + h_begin + r) * args.T +
-                   item.t] = item.n_pairs > 0 ? (mr + __log2f(L)) * kLn2 : -INFINITY;
+          args.lse[(static_cast<int64_t>(item.b) * args.Hq + item.g * G + h_begin + r) * args.Tq +
+                   item.qtok] = item.n_pairs > 0 ? (mr + __log2f(L)) * kLn2 : -INFINITY;
         }
       }
       // lsum and the staged blocks are reused by the next item
@@ -672,7 +673,7 @@ int launch_attn(const Geometry& g, const void* Q, int q_tokens, const void* K, c
 int launch_sparse_attn(const Geometry& g, const void* Q, const void* K, const void* V,
                        const int32_t* idx, void* O, float* lse, int dense, const void* packed,
                        const DevCtx& ctx, cudaStream_t st) {
-  if (g.B == 0 || g.T == 0) return INFLLMV2_OK;
+  if (g.B == 0 || g.Tq == 0) return INFLLMV2_OK;
   AttnArgs a{};
   if (packed) {
     a.Kp = static_cast<const uint8_t*>(packed);
@@ -687,10 +688,12 @@ int launch_sparse_attn(const Geometry& g, const void* Q, const void* K, const vo
   a.Hq = g.Hq;
   a.Hkv = g.Hkv;
   a.topk = g.topk;
+  a.q0 = g.q0;
+  a.Tq = g.Tq;
   a.mode = dense ? 1 : 0;
   a.scale_log2 = g.scale_log2;
-  const int64_t n_items = static_cast<int64_t>(g.B) * g.Hkv * g.T;
-  return launch_attn(g, Q, g.T, K, V, g.T, a, n_items, ctx, st);
+  const int64_t n_items = static_cast<int64_t>(g.B) * g.Hkv * g.Tq;
+  return launch_attn(g, Q, g.Tq, K, V, g.T, a, n_items, ctx, st);
 }
 
 int launch_decode_attn(const Geometry& g, const void* q, const void* Kcache, const void* Vcache,

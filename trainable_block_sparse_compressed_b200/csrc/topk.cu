@@ -11,13 +11,17 @@ namespace {
 template <int VPL>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ scores,
                                                     int32_t* __restrict__ idx, int B, int Hkv,
-                                                    int T, int topk, int n_init, int n_local) {
+                                                    int q0, int Tq, int topk, int n_init,
+                                                    int n_local) {
+  // rows: (batch, kv head, query token q0 .. q0+Tq-1); the workspace holds
+  // the causally packed score rows of those tokens, from row q0 on
   const int64_t row = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int64_t n_rows = static_cast<int64_t>(B) * Hkv * T;
+  const int64_t n_rows = static_cast<int64_t>(B) * Hkv * Tq;
   if (row >= n_rows) return;
-  const int t = static_cast<int>(row % T);
-  const int64_t bg = row / T;
-  const float* srow = scores + bg * score_row_offset(T) + score_row_offset(t);
+  const int t = q0 + static_cast<int>(row % Tq);
+  const int64_t bg = row / Tq;
+  const int64_t row0 = score_row_offset(q0);
+  const float* srow = scores + bg * (score_row_offset(q0 + Tq) - row0) + score_row_offset(t) - row0;
   const int cur = t / kBlock;
   int32_t* orow = idx + row * topk;
   if (VPL > 4 && cur < 32 * 4)
@@ -35,14 +39,14 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ sco
 }  // namespace
 
 int launch_topk(const Geometry& g, const float* scores, int32_t* idx, cudaStream_t st) {
-  if (g.B == 0 || g.T == 0) return INFLLMV2_OK;
-  const int nb_max = (g.T - 1) / kBlock + 1;
-  const int64_t rows = static_cast<int64_t>(g.B) * g.Hkv * g.T;
+  if (g.B == 0 || g.Tq == 0) return INFLLMV2_OK;
+  const int nb_max = (g.q0 + g.Tq - 1) / kBlock + 1;
+  const int64_t rows = static_cast<int64_t>(g.B) * g.Hkv * g.Tq;
   const unsigned blocks = static_cast<unsigned>((rows + 7) / 8);
   const int vpl = topk_vpl(nb_max);
 #define INFLLMV2_TOPK(V)                                                             \
-  topk_kernel<V><<<blocks, 256, 0, st>>>(scores, idx, g.B, g.Hkv, g.T, g.topk, g.n_init, \
-                                         g.n_local)
+  topk_kernel<V><<<blocks, 256, 0, st>>>(scores, idx, g.B, g.Hkv, g.q0, g.Tq, g.topk, \
+                                         g.n_init, g.n_local)
   switch (vpl) {
     case 4: INFLLMV2_TOPK(4); break;
     case 16: INFLLMV2_TOPK(16); break;

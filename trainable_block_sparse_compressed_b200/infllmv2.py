@@ -35,7 +35,8 @@ EXPORTS = (
     "infllmv2_dense_attn", "infllmv2_forward", "infllmv2_decode_step",
     "infllmv2_workspace_bytes", "infllmv2_num_compressed", "infllmv2_get_status",
     "infllmv2_set_wait_limit", "infllmv2_selftest_timeout", "infllmv2_strerror",
-    "infllmv2_version", "infllmv2_decode_step_noalloc",
+    "infllmv2_version", "infllmv2_decode_step_noalloc", "infllmv2_prefill_chunk",
+    "infllmv2_prefill_chunk_workspace_bytes",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -88,6 +89,9 @@ def load(path: Optional[str] = None):
         "infllmv2_decode_step_noalloc": (ctypes.c_int,
                                          [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]),
         "infllmv2_workspace_bytes": (sz, [P, i32]),
+        "infllmv2_prefill_chunk": (ctypes.c_int, [P, i32, i32, vp, vp, vp, vp, vp, vp, vp,
+                                                  vp, vp, sz, vp]),
+        "infllmv2_prefill_chunk_workspace_bytes": (sz, [P, i32, i32]),
         "infllmv2_num_compressed": (i32, [i32]),
         "infllmv2_get_status": (ctypes.c_int, [vp, ctypes.POINTER(i32)]),
         "infllmv2_set_wait_limit": (None, [ctypes.c_int64]),
@@ -188,6 +192,26 @@ def forward(p: Params, Q, K, V, O, lse, Kc_ws=None, idx_ws=None, ws=None, stream
            load().infllmv2_forward(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(lse),
                                    _ptr(Kc_ws), _ptr(idx_ws), ctypes.byref(path), _ptr(ws), nbytes,
                                    _stream(stream)))
+    return int(path.value)
+
+
+def prefill_chunk_workspace_bytes(p: Params, q_offset: int, q_len: int) -> int:
+    n = load().infllmv2_prefill_chunk_workspace_bytes(ctypes.byref(p), q_offset, q_len)
+    if n == ctypes.c_size_t(-1).value:
+        raise InfLLMV2Error("infllmv2_prefill_chunk_workspace_bytes", ERR_INVALID_ARG)
+    return int(n)
+
+
+def prefill_chunk(p: Params, q_offset: int, q_len: int, Q, K, V, Kc, O, lse, idx=None, ws=None,
+                  stream=None) -> int:
+    """Queries for tokens q_offset .. q_offset+q_len-1 over caches of p.T tokens;
+    returns PATH_DENSE or PATH_SPARSE."""
+    path = ctypes.c_int32(0)
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check("infllmv2_prefill_chunk",
+           load().infllmv2_prefill_chunk(ctypes.byref(p), q_offset, q_len, _ptr(Q), _ptr(K),
+                                         _ptr(V), _ptr(Kc), _ptr(O), _ptr(lse), _ptr(idx),
+                                         ctypes.byref(path), _ptr(ws), nbytes, _stream(stream)))
     return int(path.value)
 
 
