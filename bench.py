@@ -83,6 +83,15 @@ class Dist:
             self.pg.destroy_process_group()
 
 
+def main_config(w, world: int) -> dict:
+    """The workload description both arms report."""
+    return {"workload": MAIN, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "d": 128,
+            "topk": w.topk, "n_init": w.n_init, "n_local": w.n_local,
+            "switch_threshold": w.threshold, "needles": w.needles,
+            "parallelism": f"replicas x{world}",
+            "l2": "flushed between timed steps (256 MB write, outside the events)"}
+
+
 def whole_job_rate(units_per_rank: float, world: int, ms_max: float) -> float:
     """Units all ranks processed per second, timed by the slowest rank."""
     return units_per_rank * world / (ms_max / 1e3)
@@ -480,8 +489,7 @@ def main():
                 "ms_per_step": 1e3 * w.T / value, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                 "impl": "reference",
-                "config": {"workload": MAIN, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv,
-                           "d": 128, "topk": w.topk, "n_init": w.n_init, "n_local": w.n_local},
+                "config": main_config(w, int(os.environ.get("WORLD_SIZE", "1"))),
                 "cpu_baseline": dict(res, value=value),
                 "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0},
@@ -553,11 +561,7 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": MAIN, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "d": 128,
-                   "topk": w.topk, "n_init": w.n_init, "n_local": w.n_local,
-                   "switch_threshold": w.threshold, "needles": w.needles,
-                   "parallelism": f"replicas x{dist.world}",
-                   "l2": "flushed between timed steps (256 MB write, outside the events)"},
+        "config": main_config(w, dist.world),
         "useful_tflops": whole_job_rate(useful, dist.world, ms) / 1e12,
         "executed_tflops": whole_job_rate(
             main_r["executed_attn_flops"] + main_r["executed_score_flops"], dist.world, ms) / 1e12,

@@ -97,3 +97,14 @@ def test_bench_traffic_lookup_requires_the_current_kernel_source(monkeypatch, tm
     monkeypatch.setattr(bench, "kernel_source_hash", lambda name: "changed")
     assert bench.profiled_traffic("k.cu", "wl") is None
     assert bench.profiled_traffic("other.cu", "wl") is None
+
+
+def test_both_bench_arms_report_the_same_config():
+    sys.path.insert(0, ROOT)
+    import bench
+    w = wl.WORKLOADS[bench.MAIN]
+    c = bench.main_config(w, 1)
+    assert c["workload"] == bench.MAIN and c["T"] == 131072 and c["Hq"] == 32 and c["Hkv"] == 2
+    assert c["topk"] == 64 and c["n_init"] == 1 and c["n_local"] == 2
+    src = open(os.path.join(ROOT, "bench.py")).read()
+    assert src.count("main_config(w,") == 2  # the reference arm and ours
