@@ -107,4 +107,4 @@ def test_both_bench_arms_report_the_same_config():
     assert c["workload"] == bench.MAIN and c["T"] == 131072 and c["Hq"] == 32 and c["Hkv"] == 2
     assert c["topk"] == 64 and c["n_init"] == 1 and c["n_local"] == 2
     src = open(os.path.join(ROOT, "bench.py")).read()
-    assert src.count("main_config(w,") == 2  # the reference arm and ours
+    assert src.count("\"config\": main_config(w,") == 2  # the reference arm and ours
