@@ -9,9 +9,9 @@
 //                    hi + lo exactly as compress.cu does, so incremental and
 //                    batch compressed keys are bit-identical);
 //   2. score       : x[j, h] = scale*log2(e) * q_h . Kc[j] for the visible
-//                    windows, split over many CTAs (HBM-bound stream of the
-//                    compressed-key cache), plus each split's per-head max and
-//                    sum of exp2 for the softmax;
+//                    windows, tiles of 128 compressed keys on tcgen05 (an
+//                    HBM-bound stream of the compressed-key cache), plus each
+//                    tile's per-head max and sum of exp2 for the softmax;
 //   3. select      : per (sequence, kv head), split over CTAs of 128 blocks
 //                    each: merge the splits into each head's log-sum-exp,
 //                    group-sum the probabilities, max-pool onto 64-token

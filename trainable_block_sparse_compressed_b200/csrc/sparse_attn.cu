@@ -13,10 +13,14 @@
 //   S^T[128 keys x 16 heads]  = K_pair (A, K-major)   x Q^T (B, K-major)
 //   O^T[128 d    x 16 heads]  = V_pair^T (A, MN-major) x P^T (B, MN-major)
 //
-// A "pair" is two selected 64-key blocks gathered by TMA into one 128-row
-// operand (K and V: 2 x 2 boxes of 64 rows x 128 B).  Heads beyond G are
-// padding.  Persistent CTAs (one per SM) stream the pairs of their items
-// without draining between items.
+// A "pair" is two selected 64-key blocks gathered into one 128-row operand:
+// from the packed tiles of pack.cu (one 16 KB bulk copy per block and
+// tensor, already in the MMA's canonical layout) or, without a workspace and
+// in decode mode, by TMA boxes straight from K and V (2 boxes of 64 rows x
+// 128 B per block and tensor, 128-byte swizzle).  Heads beyond G are padding.
+// Persistent CTAs (one per SM) stream the pairs of their items without
+// draining between items.  Queries may be a chunk q0 .. q0+Tq-1 of a longer
+// sequence (chunked prefill); keys are addressed by their absolute position.
 //
 // What bounds this kernel is shared memory: every pair moves 64 KB from L2
 // into shared memory through the SM's copy engine, and the tensor core reads
@@ -26,7 +30,12 @@
 // products and one the P V products, each in pair order with blocking waits:
 // issuing a tcgen05.mma holds its thread for about as long as the tensor core
 // takes to read the operand, and a barrier wait costs a few hundred cycles
-// even when already complete, so one issuer alone could not keep up.  The
+// even when already complete, so one issuer alone could not keep up.  Each
+// issuer waits only for what no other wait implies: the S issuer for its
+// stage (S has four TMEM buffers, and a refilled stage means the softmax has
+// read S four pairs back), the P V issuer for P (written only after the
+// softmax read out P V two pairs back, and after S, issued once the stage
+// had landed).  The
 // softmax is split over two warpgroups by heads (heads 0-7 and 8-15 of the
 // same key rows), halving each thread's dependent chain.
 //
@@ -34,9 +43,9 @@
 // heads): each head keeps a reference maximum m that only moves when a score
 // exceeds it by more than 8 (log2 units), so the common pair needs a single
 // barrier-OR and no cross-lane reduction; P = exp2(s - m) <= 256 stays exact
-// enough in bf16.  Each pair's P V lands in a fresh TMEM buffer and is folded
-// into an fp32 register accumulator with the rescale of its own reference, so
-// the accumulator is never rescaled inside tensor memory.
+// enough in bf16.  Each pair's P V lands in one of two TMEM buffers and is
+// folded into an fp32 register accumulator with the rescale of its own
+// reference, so the accumulator is never rescaled inside tensor memory.
 //
 // Decode mode: one query token per sequence at t = seqlens[b]; the selected
 // blocks of each (sequence, kv head) are split into chunks so that enough
