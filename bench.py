@@ -25,6 +25,7 @@ import io
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -147,9 +148,15 @@ def load_peaks():
 
 
 def kernel_source_hash(name: str) -> str:
+    """Hash of a kernel source's code: comments and whitespace removed, so that
+    counters taken on a kernel stay attached to it across comment edits."""
     path = os.path.join(ROOT, "trainable_block_sparse_compressed_b200", "csrc", name)
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    with open(path, encoding="utf-8") as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    src = " ".join(src.split())
+    return hashlib.sha256(src.encode()).hexdigest()[:16]
 
 
 def profiled_traffic(kernel_file: str, workload: str):

@@ -108,3 +108,17 @@ def test_both_bench_arms_report_the_same_config():
     assert c["topk"] == 64 and c["n_init"] == 1 and c["n_local"] == 2
     src = open(os.path.join(ROOT, "bench.py")).read()
     assert src.count("\"config\": main_config(w,") == 2  # the reference arm and ours
+
+
+def test_kernel_code_hash_ignores_comments_but_not_code(monkeypatch, tmp_path):
+    sys.path.insert(0, ROOT)
+    import bench
+    d = tmp_path / "trainable_block_sparse_compressed_b200" / "csrc"
+    d.mkdir(parents=True)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (d / "k.cu").write_text("// a kernel\nint f(int x) {  return x + 1; }  /* note */\n")
+    h0 = bench.kernel_source_hash("k.cu")
+    (d / "k.cu").write_text("// the kernel, described anew\n/* more\n text */\nint f(int x) { return x + 1; }\n")
+    assert bench.kernel_source_hash("k.cu") == h0
+    (d / "k.cu").write_text("int f(int x) { return x + 2; }\n")
+    assert bench.kernel_source_hash("k.cu") != h0
