@@ -58,6 +58,8 @@ extern "C" {
 /* Device status bits (infllmv2_get_status). */
 #define INFLLMV2_STATUS_TIMEOUT        0x1
 #define INFLLMV2_STATUS_SEQ_FULL       0x2  /* decode: seqlens[b] reached the cache capacity */
+#define INFLLMV2_STATUS_CHECK          0x4  /* bounds-checked build only: an index check failed
+                                               and its access was skipped */
 
 /* The method's knobs.  Source of each: the sequence-length switch and the
  * block size (skill write-up, Implementation Steps 2-3); compressed keys that

@@ -38,6 +38,15 @@ def test_library_exports_every_declared_symbol(lib):
         assert re.search(rf"\bT {name}\b", nm), name
 
 
+def test_checked_build_exports_every_declared_symbol():
+    """libinfllmv2_checks.so (device index checks) offers the same ABI."""
+    from trainable_block_sparse_compressed_b200 import build
+    path = build.build(checks=True)
+    nm = os.popen(f"nm -D --defined-only {path}").read()
+    for name in declared_symbols():
+        assert re.search(rf"\bT {name}\b", nm), name
+
+
 def test_host_helpers(lib):
     assert lib.infllmv2_version() == 100
     assert api.num_compressed(31) == 0

@@ -64,6 +64,17 @@ __device__ __forceinline__ void report_status(int* status, int bit) {
   atomicOr(status, bit);
 }
 
+// Index checks of the bounds-checked build (compiled with -DINFLLMV2_CHECKS,
+// libinfllmv2_checks.so): a failed check sets INFLLMV2_STATUS_CHECK and the
+// caller skips the access.  In the regular build the check is the constant
+// true and generates no code.
+#ifdef INFLLMV2_CHECKS
+#define INFLLMV2_CHECK(status, cond) \
+  ((cond) ? true : (report_status((status), INFLLMV2_STATUS_CHECK), false))
+#else
+#define INFLLMV2_CHECK(status, cond) true
+#endif
+
 // Stores 8 channels of a compressed key (fp32 means) as the (hi, lo) pair:
 // hi at dst[0..7], lo at dst[kHeadDim .. kHeadDim+7].
 __device__ __forceinline__ void store_kc_pair(const float (&m)[8], __nv_bfloat16* dst) {

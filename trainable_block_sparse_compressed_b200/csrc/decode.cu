@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_score_kernel(
       const bool valid = j < d.v;
 #pragma unroll
       for (int h = 0; h < G; ++h) x[h] = valid ? x[h] * scale_log2 : -INFINITY;
-      if (valid) {
+      if (valid && INFLLMV2_CHECK(ctx.status, j < NC && d.bg < B * Hkv)) {
         float* xo = x_out + (static_cast<int64_t>(d.bg) * NC + j) * G;
         if constexpr (G % 4 == 0) {
 #pragma unroll
@@ -385,7 +385,8 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_score_kernel(
 template <int G>
 __global__ void __launch_bounds__(256) decode_pool_kernel(
     const float* __restrict__ x, const float* __restrict__ ml, const int32_t* __restrict__ seqlens,
-    float* __restrict__ bs_all, int Hkv, int NC, int NB, int Lmax, int n_split, int n_pool) {
+    float* __restrict__ bs_all, int Hkv, int NC, int NB, int Lmax, int n_split, int n_pool,
+    int* status) {
   constexpr int kWin = 4 * kPoolBlocks + 4;  // windows 4*blk0-1 .. 4*blk1+3 (clipped)
   __shared__ float S[kWin];
   __shared__ float lse2[G];
@@ -447,14 +448,14 @@ __global__ void __launch_bounds__(256) decode_pool_kernel(
 #pragma unroll
         for (int h = 0; h < G; ++h) acc += fast_exp2(__ldg(xs + h) - lse2[h]);
       }
-      S[j - j0] = acc;
+      if (INFLLMV2_CHECK(status, j - j0 >= 0 && j - j0 < kWin)) S[j - j0] = acc;
     }
     __syncthreads();
     for (int blk = blk0 + threadIdx.x; blk < blk1; blk += blockDim.x) {
       const int j_lo = max(0, 4 * blk - 1), j_hi = min(v - 1, 4 * blk + 3);
       float mx = -INFINITY;
       for (int j = j_lo; j <= j_hi; ++j) mx = fmaxf(mx, S[j - j0]);
-      bs[blk] = mx;
+      if (INFLLMV2_CHECK(status, blk < NB)) bs[blk] = mx;
     }
   }
 }
@@ -565,7 +566,7 @@ int launch_decode_g(const Geometry& g, const DecodeLayout& L, const void* q, con
   }
   const int per = select_per(L.NB);
   decode_pool_kernel<G><<<bgn * L.n_pool, 256, 0, st>>>(x, ml, seqlens, bs, g.Hkv, L.NC, L.NB, g.T,
-                                                       L.n_split, L.n_pool);
+                                                       L.n_split, L.n_pool, ctx.status);
   if (cudaGetLastError() != cudaSuccess) return INFLLMV2_ERR_CUDA;
 #define INFLLMV2_SEL(V)                                                                     \
   decode_topk_kernel<V><<<bgn, 256, 0, st>>>(bs, seqlens, idx, g.Hkv, L.NB, g.T, g.topk, \

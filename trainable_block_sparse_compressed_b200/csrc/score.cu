@@ -309,7 +309,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           float prev = __shfl_up_sync(0xffffffffu, S[tl], 1);
           if (lane == 0) prev = sm.carry[cb][quad][tok];
           const int t = t0 + tok;
-          if ((lane & 3) == 0 && t < q_end && blk <= t / kBlock)
+          if ((lane & 3) == 0 && t < q_end && blk <= t / kBlock &&
+              INFLLMV2_CHECK(ctx.status, blk >= 0 && score_row_offset(t) - row0 + blk < slab))
             srow_base[score_row_offset(t) - row0 + blk] = fmaxf(m4, prev);
         }
       }
@@ -322,7 +323,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (t >= q_end) continue;
         const int cur = t / kBlock;
         for (int blk = n_t * (kKcTile / 4); blk <= cur; ++blk)
-          srow_base[score_row_offset(t) - row0 + blk] =
+          if (INFLLMV2_CHECK(ctx.status, score_row_offset(t) - row0 + blk < slab))
+            srow_base[score_row_offset(t) - row0 + blk] =
               blk == n_t * (kKcTile / 4) ? sm.carry[n_t % 3][0][tok] : -INFINITY;
       }
     }

@@ -303,6 +303,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const CUtensorMap* tm = v ? &tmV : &tmK;
         for (int slot = 0; slot < (pl.two ? 2 : 1); ++slot) {
           const int blk = slot ? pl.blk1 : pl.blk0;
+          // (checked build) a skipped copy leaves the stage short, so the
+          // bounded waits on it expire and the kernel aborts cleanly
+          if (!INFLLMV2_CHECK(ctx.status, pl.b >= 0 && pl.b < args.B && pl.g >= 0 &&
+                                              pl.g < args.Hkv && blk >= 0 &&
+                                              static_cast<int64_t>(blk) * kBlock < args.T))
+            continue;
           if (packed) {
             bulk_load(st + slot * kHalf, packed + (tile0 + blk) * kHalf, kHalf, full);
           } else {
@@ -596,7 +602,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           pml[2 * (h_begin + r)] = item.n_pairs > 0 ? mr : -INFINITY;
           pml[2 * (h_begin + r) + 1] = item.n_pairs > 0 ? L : 0.f;
         }
-      } else {
+      } else if (INFLLMV2_CHECK(ctx.status, item.b >= 0 && item.b < args.B && item.qtok >= 0 &&
+                                                item.qtok < args.Tq && item.g >= 0 &&
+                                                item.g < args.Hkv)) {
         const int64_t orow =
             (static_cast<int64_t>(item.b) * args.Tq + item.qtok) * args.Hq + item.g * G;
 #pragma unroll

@@ -68,11 +68,13 @@ def make_params(B, T, Hq, Hkv, head_dim=128, topk=64, n_init=1, n_local=2,
 
 
 def load(path: Optional[str] = None):
-    """Loads the shared library once; raises if it is missing."""
+    """Loads the shared library once; raises if it is missing.  The
+    environment variable INFLLMV2_LIB may name another build of it (the
+    bounds-checked libinfllmv2_checks.so)."""
     global _lib
     if _lib is not None:
         return _lib
-    p = path or _LIB_PATH
+    p = path or os.environ.get("INFLLMV2_LIB") or _LIB_PATH
     if not os.path.exists(p):
         raise RuntimeError(f"CUDA library not built: {p} (run __graft_entry__.build())")
     lib = ctypes.CDLL(p)
