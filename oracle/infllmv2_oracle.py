@@ -294,6 +294,85 @@ def sparse_attention(Q, K, V, idx, p: Params, rows=None):
     return O, L
 
 
+def attend_backward(q_group, K_g, V_g, keys, scale, dO_group):
+    """Gradients of attend() for one row: the softmax attention of the group's
+    heads q_group [G, d] over the listed keys, given dO [G, d].
+
+    With s = scale q.k, P = softmax(s), o = P V:
+      dV[keys] += P^T dO,  dP = dO V^T,  dS = P * (dP - rowsum(dO * o)),
+      dq = scale dS K[keys],  dK[keys] += scale dS^T q.
+    Returns (dq [G, d], dK_rows [n, d], dV_rows [n, d]) for the listed keys.
+    """
+    Kk, Vk = K_g[keys], V_g[keys]
+    s = scale * (q_group @ Kk.T)                          # [G, n]
+    P = np.exp(s - s.max(axis=1, keepdims=True))
+    P /= P.sum(axis=1, keepdims=True)
+    o = P @ Vk                                            # [G, d]
+    dV = P.T @ dO_group                                   # [n, d]
+    dP = dO_group @ Vk.T                                  # [G, n]
+    dS = P * (dP - (dO_group * o).sum(axis=1, keepdims=True))
+    dq = scale * dS @ Kk
+    dK = scale * dS.T @ q_group
+    return dq, dK, dV
+
+
+def sparse_attention_backward(Q, K, V, idx, dO, p: Params):
+    """Gradients (dQ, dK, dV) of sparse_attention's O with the selection idx
+    held fixed (the selection is a discrete choice; training propagates
+    through the attention over the chosen blocks), given dO [B, T, Hq, d].
+    Keys shared by several rows accumulate their contributions."""
+    B, T, Hq, d = Q.shape
+    Hkv = K.shape[2]
+    G = Hq // Hkv
+    sc = p.sm_scale(d)
+    dQ = np.zeros_like(Q)
+    dK = np.zeros_like(K)
+    dV = np.zeros_like(V)
+    for b in range(B):
+        for g in range(Hkv):
+            hs = slice(g * G, (g + 1) * G)
+            for t in range(T):
+                keys = selected_keys(idx[b, g, t], t, p)
+                dq, dk, dv = attend_backward(Q[b, t, hs], K[b, :, g], V[b, :, g], keys, sc,
+                                             dO[b, t, hs])
+                dQ[b, t, hs] = dq
+                np.add.at(dK[b, :, g], keys, dk)
+                np.add.at(dV[b, :, g], keys, dv)
+    return dQ, dK, dV
+
+
+def compressed_attention(Q, K, V, p: Params, rows=None):
+    """The compressed-attention branch (skill write-up, Core Concept: the
+    compressed pattern aggregates tokens hierarchically): each query row
+    attends over the compressed windows it can see, with keys Kc[j] and values
+    Vc[j] the means of K and V over window j.  Visibility follows the
+    selection's rule (window j visible to t iff 16j+31 <= t); a row with no
+    visible window gets O = 0 and LSE = -inf.
+
+    Returns (O [B, T, Hq, d], LSE [B, Hq, T]); ``rows`` as in sparse_attention.
+    """
+    B, T, Hq, d = Q.shape
+    Hkv = K.shape[2]
+    G = Hq // Hkv
+    Kc, Vc = compress_keys(K, p), compress_keys(V, p)   # the same window means
+    O = np.full((B, T, Hq, d), np.nan)
+    L = np.full((B, Hq, T), np.nan)
+    if rows is None:
+        rows = [(b, g, t) for b in range(B) for g in range(Hkv) for t in range(T)]
+    sc = p.sm_scale(d)
+    for (b, g, t) in rows:
+        hs = slice(g * G, (g + 1) * G)
+        v = min(visible_windows(t, p), Kc.shape[1])
+        if v == 0:
+            O[b, t, hs] = 0.0
+            L[b, hs, t] = -np.inf
+            continue
+        o, lse = attend(Q[b, t, hs], Kc[b, :, g], Vc[b, :, g], np.arange(v), sc)
+        O[b, t, hs] = o
+        L[b, hs, t] = lse
+    return O, L
+
+
 def dense_attention(Q, K, V, p: Params, rows=None):
     """Exact causal softmax attention (every key 0..t)."""
     B, T, Hq, d = Q.shape

@@ -419,3 +419,113 @@ def test_chunk_forward_equals_the_whole_sequence_rows(q0, Tq, threshold):
     assert np.array_equal(Oc, O[:, q0:]) and np.array_equal(Lc, L[:, :, q0:])
     if idx is not None:
         assert np.array_equal(idx_c, idx[:, :, q0:])
+
+
+def _tiny_sparse_case(seed=41, T=200, Hq=4, Hkv=2, d=16, topk=3):
+    rng = np.random.default_rng(seed)
+    Q = rng.standard_normal((1, T, Hq, d))
+    K = rng.standard_normal((1, T, Hkv, d))
+    V = rng.standard_normal((1, T, Hkv, d))
+    p = orc.Params(topk=topk, n_init=1, n_local=1, threshold=0)
+    idx, _ = orc.select_blocks(Q, K, p)
+    return Q, K, V, idx, p
+
+
+def test_sparse_backward_matches_finite_differences():
+    """Central differences of L = sum(dO * O) with the selection held fixed."""
+    Q, K, V, idx, p = _tiny_sparse_case()
+    rng = np.random.default_rng(5)
+    dO = rng.standard_normal(Q.shape)
+    loss = lambda Q_, K_, V_: float((orc.sparse_attention(Q_, K_, V_, idx, p)[0] * dO).sum())  # noqa: E731
+    dQ, dK, dV = orc.sparse_attention_backward(Q, K, V, idx, dO, p)
+    eps = 1e-6
+    picks = [(0, 150, 1, 3), (0, 70, 0, 0), (0, 199, 3, 15)]
+    for (b, t, h, c) in picks:
+        Qp, Qm = Q.copy(), Q.copy()
+        Qp[b, t, h, c] += eps
+        Qm[b, t, h, c] -= eps
+        num = (loss(Qp, K, V) - loss(Qm, K, V)) / (2 * eps)
+        assert abs(num - dQ[b, t, h, c]) <= 1e-6 * max(1.0, abs(num))
+    for (b, t, g, c) in [(0, 3, 0, 2), (0, 130, 1, 7), (0, 64, 1, 0)]:
+        for X, dX in ((K, dK), (V, dV)):
+            Xp, Xm = X.copy(), X.copy()
+            Xp[b, t, g, c] += eps
+            Xm[b, t, g, c] -= eps
+            args_p = (Q, Xp, V) if X is K else (Q, K, Xp)
+            args_m = (Q, Xm, V) if X is K else (Q, K, Xm)
+            num = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+            assert abs(num - dX[b, t, g, c]) <= 1e-6 * max(1.0, abs(num))
+
+
+def test_sparse_backward_with_every_block_equals_dense_autograd():
+    """top-k covering every block: the gradients equal torch autograd (fp64)
+    of exact causal softmax attention."""
+    import torch
+    Q, K, V, _, _ = _tiny_sparse_case(T=190, topk=3)
+    p = orc.Params(topk=8, n_init=1, n_local=1, threshold=0)
+    idx, _ = orc.select_blocks(Q, K, p)
+    dO = np.random.default_rng(6).standard_normal(Q.shape)
+    dQ, dK, dV = orc.sparse_attention_backward(Q, K, V, idx, dO, p)
+    G = Q.shape[2] // K.shape[2]
+    q = torch.tensor(Q, requires_grad=True)
+    k = torch.tensor(K, requires_grad=True)
+    v = torch.tensor(V, requires_grad=True)
+    kk = k.repeat_interleave(G, dim=2)
+    vv = v.repeat_interleave(G, dim=2)
+    out = torch.nn.functional.scaled_dot_product_attention(
+        q.transpose(1, 2), kk.transpose(1, 2), vv.transpose(1, 2), is_causal=True,
+        scale=p.sm_scale(Q.shape[-1])).transpose(1, 2)
+    (out * torch.tensor(dO)).sum().backward()
+    assert np.allclose(dQ, q.grad.numpy(), atol=1e-10)
+    assert np.allclose(dK, k.grad.numpy(), atol=1e-10)
+    assert np.allclose(dV, v.grad.numpy(), atol=1e-10)
+
+
+def test_compressed_attention_with_equal_keys_averages_the_window_values():
+    """Closed form: with every key equal, all visible windows score alike and
+    the output is the plain mean of the visible windows' mean values."""
+    rng = np.random.default_rng(12)
+    T, d = 300, 16
+    Q = rng.standard_normal((1, T, 4, d))
+    K = np.broadcast_to(rng.standard_normal((1, 1, 2, d)), (1, T, 2, d)).copy()
+    V = rng.standard_normal((1, T, 2, d))
+    p = orc.Params()
+    O, L = orc.compressed_attention(Q, K, V, p)
+    for t in (0, 30, 31, 46, 47, 299):
+        v = 0 if t < 31 else (t - 31) // 16 + 1
+        for h in range(4):
+            g = h // 2
+            if v == 0:
+                assert np.all(O[0, t, h] == 0) and L[0, h, t] == -np.inf
+                continue
+            win_means = [V[0, 16 * j:16 * j + 32, g].mean(axis=0) for j in range(v)]
+            assert np.allclose(O[0, t, h], np.mean(win_means, axis=0), atol=1e-12)
+            s = (Q[0, t, h] @ K[0, 0, g]) / np.sqrt(d)
+            assert np.isclose(L[0, h, t], s + np.log(v))
+
+
+def test_compressed_attention_equals_masked_sdpa():
+    """Against torch's fp64 scaled_dot_product_attention over the window
+    means with an explicit visibility mask."""
+    import torch
+    rng = np.random.default_rng(13)
+    T, d, Hq, Hkv = 260, 16, 4, 2
+    Q = rng.standard_normal((1, T, Hq, d))
+    K = rng.standard_normal((1, T, Hkv, d))
+    V = rng.standard_normal((1, T, Hkv, d))
+    p = orc.Params()
+    O, _ = orc.compressed_attention(Q, K, V, p)
+    n = (T - 32) // 16 + 1
+    Kc = np.stack([K[:, 16 * j:16 * j + 32].mean(axis=1) for j in range(n)], axis=1)
+    Vc = np.stack([V[:, 16 * j:16 * j + 32].mean(axis=1) for j in range(n)], axis=1)
+    t = np.arange(T)[:, None]
+    j = np.arange(n)[None, :]
+    mask = torch.tensor(16 * j + 31 <= t)                        # [T, n]
+    rows = mask.any(dim=1).numpy()
+    q = torch.tensor(Q).transpose(1, 2)
+    kk = torch.tensor(Kc).repeat_interleave(Hq // Hkv, dim=2).transpose(1, 2)
+    vv = torch.tensor(Vc).repeat_interleave(Hq // Hkv, dim=2).transpose(1, 2)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q[:, :, rows], kk, vv, attn_mask=mask[rows]).transpose(1, 2).numpy()
+    assert np.allclose(O[:, rows], ref, atol=1e-12)
+    assert np.all(O[:, ~rows] == 0)
