@@ -37,6 +37,8 @@ sys.path.insert(0, ROOT)
 METRIC = "sparse-attn prefill tokens/s + TFLOP/s at 32k/128k; decode tok/s, HBM GB/s"
 MAIN = "sparse_prefill_T131072_Hq32_Hkv2"
 SIDE = "sparse_prefill_T32768_Hq32_Hkv2"
+SMALL = "sparse_prefill_T2048_Hq8_Hkv2"
+DENSE = "dense_switch_B2_T4096_Hq32_Hkv2"
 DECODE = "sparse_decode_B16_L131072_Hq32_Hkv2"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -187,7 +189,7 @@ def attended_keys(idx_np, T):
 # our implementation
 # ---------------------------------------------------------------------------
 def run_prefill(api, wl, w, steps, warmup, dist, flush, time_e2e=True, clocks=None,
-                chunk_len=0):
+                chunk_len=0, measure_gather=False):
     import numpy as np
     import torch
     data = wl.make_prefill(w)
@@ -250,7 +252,8 @@ def run_prefill(api, wl, w, steps, warmup, dist, flush, time_e2e=True, clocks=No
         tl = min(t0 + tpt - 1, T - 1)
         vt = 0 if tl < 31 else min(n_c, (tl - 31) // 16 + 1)
         nt = (vt + 127) // 128
-        executed_score_flops += 2 * 2 * (2 * 128 * 128 * 256) * nt  # 2 passes, hi+lo
+        # pass 1 multiplies the hi plane only (K = 128), pass 2 hi and lo (K = 256)
+        executed_score_flops += (2 * 128 * 128 * 128 + 2 * 128 * 128 * 256) * nt
     executed_score_flops *= B * Hkv
     idx_np = idx.cpu().numpy()
     cur = (np.arange(T) // 64)[None, None, :, None]
@@ -258,7 +261,10 @@ def run_prefill(api, wl, w, steps, warmup, dist, flush, time_e2e=True, clocks=No
     pairs = int(((n_valid + 1) // 2).sum())
     # per gathered pair: S^T (128 keys x 16 heads x 128) and P V, 2 FLOP per MAC
     executed_attn_flops = float(pairs) * 2 * (2 * 128 * 16 * 128)
-    out = dict(ms=ms, step_ms=step_ms, kernels=kern, tokens=B * T,
+    gather = None
+    if measure_gather:
+        gather = gather_roofline(api, aws, pairs, kern["sparse_attn"])
+    out = dict(ms=ms, step_ms=step_ms, kernels=kern, tokens=B * T, gather=gather,
                useful_attn_flops=useful_attn_flops, useful_score_flops=useful_score_flops,
                executed_score_flops=executed_score_flops, executed_attn_flops=executed_attn_flops,
                clocks=clk, launches_per_step=5)
@@ -269,6 +275,34 @@ def run_prefill(api, wl, w, steps, warmup, dist, flush, time_e2e=True, clocks=No
     del Q, K, V, Kc, idx, ws, O, lse
     torch.cuda.empty_cache()
     return out
+
+
+def gather_roofline(api, tiles, pairs, attn_ms, rounds=2000, reps=5):
+    """The attention's L2 -> shared-memory gather against this GPU's ceiling
+    for that movement, measured now by the library's gather kernel over the
+    attention's own packed K/V tiles (L2-resident)."""
+    import torch
+    stream = torch.cuda.current_stream()
+    for _ in range(2):
+        api.gather_peak(tiles, rounds)
+    torch.cuda.synchronize()
+    rates = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        moved = api.gather_peak(tiles, rounds)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        rates.append(moved / (e0.elapsed_time(e1) / 1e3) / 1e9)
+    assert api.get_status() == 0
+    peak = statistics.median(rates)
+    per_launch = pairs * 65536  # K and V of two 64-key blocks per gathered pair
+    achieved = per_launch / (attn_ms / 1e3) / 1e9
+    return {"bound": "l2_gather", "kernel": "sparse_attn", "achieved": achieved, "peak": peak,
+            "unit": "GB/s", "frac": achieved / peak, "bytes_per_launch": per_launch,
+            "peak_source": "measured in this run: infllmv2_gather_peak, 16 KB bulk copies "
+                           "from the attention's packed K/V tiles into a 3 x 64 KB ring, "
+                           "one CTA per SM, median of 5"}
 
 
 def time_chunk(api, p, Q, K, V, Kc, n, steps, warmup, flush):
@@ -418,18 +452,110 @@ def run_decode(api, wl, w, steps, warmup, flush):
     assert api.get_status() == 0
     assert int(seqlens[0]) == L0 + total
     per_step = ms / steps
-    # algorithmic HBM bytes per step: every visible compressed key (hi+lo) of
-    # every sequence and kv head, the K and V rows of the selected blocks, the
-    # appended K/V rows, q and the outputs
+    # algorithmic HBM bytes per step: every visible compressed key of every
+    # sequence and kv head as one bf16 row, the K and V rows of the selected
+    # blocks, the appended K/V rows, q and the outputs.  The library also
+    # reads the low bf16 plane of each compressed key (its precision choice,
+    # not the method's work): listed apart, not counted.
     nc_vis = (L0 + warmup + steps // 2 - 31) // 16 + 1
-    kc_bytes = B * Hkv * nc_vis * 2 * 128 * 2
+    kc_bytes = B * Hkv * nc_vis * 128 * 2
     kv_bytes = B * Hkv * w.topk * 64 * 128 * 2 * 2
     small = B * (Hq * 128 * 2 * 2 + Hkv * 128 * 2 * 2 + Hq * 4)
     bytes_step = kc_bytes + kv_bytes + small
     del g
     return dict(ms_per_step=per_step, tokens_per_s=B / (per_step / 1e3),
                 hbm_gbs=bytes_step / (per_step / 1e3) / 1e9, bytes_per_step=bytes_step,
-                steps=steps, launches_per_step=6)
+                lo_plane_bytes_per_step=kc_bytes, steps=steps, launches_per_step=6)
+
+
+def run_dense(api, wl, w, steps, warmup, flush):
+    """The dense-switch workload through infllmv2_forward (T <= threshold, so
+    the switch takes exact dense causal attention), inputs resident."""
+    import torch
+    data = wl.make_prefill(w)
+    Q, K, V = (wl.to_torch_bf16(data[x]).cuda() for x in "QKV")
+    B, T, Hq, Hkv = w.B, w.T, w.Hq, w.Hkv
+    p = api.make_params(B, T, Hq, Hkv, topk=w.topk, n_init=w.n_init, n_local=w.n_local,
+                        switch_threshold=w.threshold)
+    O = torch.empty_like(Q)
+    lse = torch.empty((B, Hq, T), dtype=torch.float32, device="cuda")
+    ws = api.alloc_workspace(p, api.OP_FORWARD)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        flush()
+        assert api.forward(p, Q, K, V, O, lse, ws=ws) == api.PATH_DENSE
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(steps):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        api.forward(p, Q, K, V, O, lse, ws=ws)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    assert api.get_status() == 0
+    # causal attention: row t attends t + 1 keys; QK^T and PV, 2 FLOP per MAC
+    flops = 4.0 * 128 * Hq * B * (T * (T + 1) / 2)
+    m = sum(ms) / len(ms)
+    del Q, K, V, O, lse, ws
+    torch.cuda.empty_cache()
+    return dict(ms=m, tokens=B * T, flops=flops)
+
+
+def profile_case(api, wl, name: str, iters: int, decode_steps: int, decode_len: int):
+    """A few passes of the path for profilers (kernel filters pick what to
+    capture): the prefill stages on one workload, or decode steps over a
+    cache of decode_len tokens.  Seeded inputs, copied to the GPU once."""
+    import torch
+    if decode_steps:
+        w = wl.WORKLOADS[DECODE]
+        B, L = w.B, decode_len
+        d = wl.make_decode(w, L=L, steps=decode_steps, B=B)
+        Lmax = L + decode_steps
+        p = api.make_params(B, Lmax, w.Hq, w.Hkv, topk=w.topk)
+        Kc = torch.zeros((B, Lmax, w.Hkv, 128), dtype=torch.bfloat16, device="cuda")
+        Vc = torch.zeros_like(Kc)
+        Kc[:, :L] = wl.to_torch_bf16(d["K0"]).cuda()
+        Vc[:, :L] = wl.to_torch_bf16(d["V0"]).cuda()
+        Kcmp = torch.zeros((B, api.num_compressed(Lmax), w.Hkv, 2, 128), dtype=torch.bfloat16,
+                           device="cuda")
+        n0 = api.num_compressed(L)
+        tmp = torch.empty((B, n0, w.Hkv, 2, 128), dtype=torch.bfloat16, device="cuda")
+        api.compress_keys(api.make_params(B, L, w.Hq, w.Hkv), Kc[:, :L].contiguous(), tmp)
+        Kcmp[:, :n0] = tmp
+        seqlens = torch.full((B,), L, dtype=torch.int32, device="cuda")
+        O = torch.empty((B, w.Hq, 128), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((B, w.Hq), dtype=torch.float32, device="cuda")
+        ws = api.alloc_workspace(p, api.OP_DECODE)
+        q, kn, vn = (wl.to_torch_bf16(d[x]).cuda() for x in ("q", "k_new", "v_new"))
+        for s in range(decode_steps):
+            api.decode_step(p, q[s], kn[s], vn[s], Kc, Vc, Kcmp, seqlens, O, lse, None, ws)
+    else:
+        w = wl.WORKLOADS[name]
+        d = wl.make_prefill(w)
+        Q, K, V = (wl.to_torch_bf16(d[x]).cuda() for x in "QKV")
+        p = api.make_params(w.B, w.T, w.Hq, w.Hkv, topk=w.topk, n_init=w.n_init,
+                            n_local=w.n_local, switch_threshold=w.threshold)
+        O = torch.empty_like(Q)
+        lse = torch.empty((w.B, w.Hq, w.T), dtype=torch.float32, device="cuda")
+        if w.T <= w.threshold:
+            ws = api.alloc_workspace(p, api.OP_FORWARD)
+            for _ in range(iters):
+                api.forward(p, Q, K, V, O, lse, ws=ws)
+        else:
+            Kc = torch.empty((w.B, api.num_compressed(w.T), w.Hkv, 2, 128), dtype=torch.bfloat16,
+                             device="cuda")
+            idx = torch.empty((w.B, w.Hkv, w.T, w.topk), dtype=torch.int32, device="cuda")
+            ws = api.alloc_workspace(p, api.OP_SELECT)
+            aws = api.alloc_workspace(p, api.OP_ATTN)
+            for _ in range(iters):
+                api.compress_keys(p, K, Kc)
+                api.select_blocks(p, Q, Kc, idx, ws)
+                api.sparse_attn(p, Q, K, V, idx, O, lse, aws)
+    torch.cuda.synchronize()
+    assert api.get_status() == 0
+    print("profile case done", flush=True)
 
 
 def cpu_oracle_sample(w, seconds=15.0):
@@ -475,8 +601,22 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extras", action="store_true", help="skip the 32k and decode extras")
     ap.add_argument("--baseline-seconds", type=float, default=15.0)
+    ap.add_argument("--profile-case", metavar="WORKLOAD",
+                    help="run the path a few times on one workload for a profiler, then exit")
+    ap.add_argument("--iters", type=int, default=2, help="--profile-case: passes of the path")
+    ap.add_argument("--decode-steps", type=int, default=0,
+                    help="--profile-case: decode steps instead of prefill")
+    ap.add_argument("--decode-len", type=int, default=131072,
+                    help="--profile-case: cached tokens per sequence for the decode steps")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+
+    if args.profile_case:
+        from trainable_block_sparse_compressed_b200 import infllmv2 as api
+        from trainable_block_sparse_compressed_b200 import workloads as wl
+        api.load()
+        profile_case(api, wl, args.profile_case, args.iters, args.decode_steps, args.decode_len)
+        return
 
     from trainable_block_sparse_compressed_b200 import workloads as wl
     w = wl.WORKLOADS[MAIN]
@@ -517,7 +657,7 @@ def main():
 
     clocks = ClockSampler(dist.local)
     main_r = run_prefill(api, wl, w, args.steps, args.warmup, dist, flush, True, clocks,
-                         chunk_len=0 if args.no_extras else 8192)
+                         chunk_len=0 if args.no_extras else 8192, measure_gather=True)
     ms = dist.max(main_r["ms"])
     e2e_ms = dist.max(main_r["e2e_ms"])
     value = whole_job_rate(main_r["tokens"], dist.world, ms)
@@ -538,6 +678,22 @@ def main():
             "tokens_per_s": whole_job_rate(side["tokens"], dist.world, sms), "ms_per_step": sms,
             "useful_tflops": (side["useful_attn_flops"] + side["useful_score_flops"]) / (sms / 1e3) / 1e12,
             "kernels_ms": side["kernels"]}
+        small = run_prefill(api, wl, wl.WORKLOADS[SMALL], args.steps, args.warmup, dist, flush,
+                            False, None)
+        s1 = dist.max(small["ms"])
+        a1 = small["kernels"]["sparse_attn"]
+        extras["prefill_T2048_Hq8_Hkv2"] = {
+            "tokens_per_s": whole_job_rate(small["tokens"], dist.world, s1), "ms_per_step": s1,
+            "useful_tflops": (small["useful_attn_flops"] + small["useful_score_flops"]) / (s1 / 1e3) / 1e12,
+            "attn_tensor_frac_of_burst": small["useful_attn_flops"] / (a1 / 1e3) / 1e12 / peaks["bf16_tflops"],
+            "kernels_ms": small["kernels"], "switch_threshold": 0}
+        dn = run_dense(api, wl, wl.WORKLOADS[DENSE], args.steps, args.warmup, flush)
+        d1 = dist.max(dn["ms"])
+        extras["dense_switch_B2_T4096"] = {
+            "path": "dense", "tokens_per_s": whole_job_rate(dn["tokens"], dist.world, d1),
+            "ms_per_step": d1, "tflops": dn["flops"] / (d1 / 1e3) / 1e12,
+            "tensor_frac_of_burst": dn["flops"] / (d1 / 1e3) / 1e12 / peaks["bf16_tflops"],
+            "flops_per_step": dn["flops"]}
         wd = wl.WORKLOADS[DECODE]
         dec = run_decode(api, wl, wd, 256, 8, flush)
         dms = dist.max(dec["ms_per_step"])
@@ -545,7 +701,10 @@ def main():
             "tokens_per_s": whole_job_rate(wd.B, dist.world, dms), "ms_per_step": dms,
             "hbm_gbs": dec["bytes_per_step"] / (dms / 1e3) / 1e9,
             "hbm_frac_of_measured": dec["bytes_per_step"] / (dms / 1e3) / 1e9 / peaks["hbm_gbs"],
-            "algorithmic_bytes_per_step": dec["bytes_per_step"], "steps": 256,
+            "hbm_frac_of_nominal_8tbs": dec["bytes_per_step"] / (dms / 1e3) / 1e9 / 8000.0,
+            "algorithmic_bytes_per_step": dec["bytes_per_step"],
+            "not_counted_lo_plane_bytes_per_step": dec["lo_plane_bytes_per_step"],
+            "steps": 256,
             "timing": "256 steps in one CUDA graph, L2 flushed before the replay"}
 
     # roofline of the dominant kernel (the block-sparse attention)
@@ -562,6 +721,8 @@ def main():
                 "unit": "TFLOP/s", "frac": achieved / sustained,
                 "peak_source": f"{peak_src} bf16 sustained",
                 "traffic": profiled_traffic(kfile, MAIN)}
+    if main_r["gather"] and dom == "sparse_attn":
+        roofline["gather_frac"] = main_r["gather"]["frac"]
     useful = main_r["useful_attn_flops"] + main_r["useful_score_flops"]
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": dist.world,
@@ -574,6 +735,7 @@ def main():
             main_r["executed_attn_flops"] + main_r["executed_score_flops"], dist.world, ms) / 1e12,
         "kernels_ms": kern,
         "roofline": roofline,
+        "gather_roofline": main_r["gather"],
         "e2e": {"value": whole_job_rate(main_r["tokens"], dist.world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": main_r["h2d"], "d2h_bytes_per_step": main_r["d2h"]},
         "gpu_launches": main_r["launches_per_step"] * args.steps,

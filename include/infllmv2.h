@@ -34,8 +34,11 @@
  *   a decode sequence at capacity) set bits in the device status word, read
  *   with infllmv2_get_status.
  * - Built and supported: head_dim == 128, block_size == 64, cmp_kernel == 32,
- *   cmp_stride == 16, causal == 1, Hq/Hkv in {1,2,4,8,16}.  Other values
- *   return INFLLMV2_ERR_UNSUPPORTED.
+ *   cmp_stride == 16, causal == 1, Hq/Hkv in {1,2,4,8,16}, T <= 2^22 tokens;
+ *   block selection (select_blocks and the sparse branches of forward and
+ *   prefill_chunk) up to INFLLMV2_MAX_SELECT_T tokens per sequence, decode up
+ *   to INFLLMV2_MAX_DECODE_T.  Other values return INFLLMV2_ERR_UNSUPPORTED
+ *   before anything is enqueued.
  */
 #ifndef INFLLMV2_H_
 #define INFLLMV2_H_
@@ -46,6 +49,9 @@
 #ifdef __cplusplus
 extern "C" {
 #endif
+
+#define INFLLMV2_MAX_SELECT_T   262144  /* 4096 key blocks */
+#define INFLLMV2_MAX_DECODE_T   524288  /* 8192 key blocks */
 
 #define INFLLMV2_OK                    0
 #define INFLLMV2_ERR_INVALID_ARG      -1  /* null pointer, bad shape, topk < forced count */
@@ -283,6 +289,22 @@ void infllmv2_set_wait_limit(int64_t ns);
  * the bit and the context stays usable.
  */
 int infllmv2_selftest_timeout(void* stream);
+
+/*
+ * Measuring aid for the block-sparse attention's roofline: the rate at which
+ * this GPU moves 16 KB key/value tiles from L2 into shared memory, the
+ * movement that bounds the attention when tokens share few blocks
+ * (reportify digest, Model Advantages: the method's kernels are designed to
+ * cut HBM traffic, so the gathered blocks are served from L2).  One CTA per
+ * SM issues `rounds` x 12 bulk copies of 16 KB (three 64 KB stages per round)
+ * from pseudo-random 16 KB-aligned offsets of `src` (a device buffer of
+ * src_bytes >= 16 KB; keep it smaller than L2 so that the copies hit L2)
+ * into shared memory, and nothing else.  The caller times the launch on
+ * `stream`; it moves *ctas_out x rounds x 196608 bytes.  *ctas_out (host
+ * pointer, may be NULL) receives the number of CTAs.
+ */
+int infllmv2_gather_peak(const void* src, size_t src_bytes, int32_t rounds, int32_t* ctas_out,
+                         void* stream);
 
 /* Human-readable text of an error code. */
 const char* infllmv2_strerror(int code);

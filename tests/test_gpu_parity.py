@@ -274,9 +274,11 @@ def _full_prefill_check(api, name, n_rows, seed):
         hs = slice(g * G, (g + 1) * G)
         assert np.abs(Og[b, t, hs] - O_ref[b, t, hs]).max() <= O_ATOL
         assert np.abs(Lg[b, hs, t] - L_ref[b, hs, t]).max() <= LSE_ATOL
-        if np.array_equal(gidx[b, g, t], oidx[b, g, t]):   # forward() output too
-            assert np.abs(Of[b, t, hs] - O_ref[b, t, hs]).max() <= O_ATOL
-            assert np.abs(Lf[b, hs, t] - L_ref[b, hs, t]).max() <= LSE_ATOL
+        # forward()'s own output, over its own selection (band-checked above)
+        keys = orc.selected_keys(gidx[b, g, t], t, op)
+        o, l = orc.attend(Q[b, t, hs], K[b, :, g], V[b, :, g], keys, op.sm_scale(128))
+        assert np.abs(Of[b, t, hs] - o).max() <= O_ATOL
+        assert np.abs(Lf[b, hs, t] - l).max() <= LSE_ATOL
 
 
 def test_prefill_32k_sampled(cuda_lib):
@@ -314,6 +316,29 @@ def _decode_setup(api, w, L0, steps, B, mutate=None):
     return data, p, Kc, Vc, Kcmp, seqlens, ws
 
 
+
+def _check_decode_row(K_seq, V_seq, Kc_seq, q, t, gi, Og, Lg, op, O_ref=None, L_ref=None,
+                      i_ref=None):
+    """One sequence's decode step, every kv group: the GPU's selection by the
+    band rule; its O and LSE against the oracle's attention over the GPU's own
+    selection (so rows whose selection differs inside the band are compared
+    too), and against the oracle's own result where the selections agree."""
+    Hq = q.shape[0]
+    Hkv = K_seq.shape[1]
+    G = Hq // Hkv
+    sc = op.sm_scale(128)
+    for g in range(Hkv):
+        hs = slice(g * G, (g + 1) * G)
+        r = orc.select_query(q[hs], Kc_seq[:, g], t, op)
+        check_selection_row(r, gi[g], op.topk)
+        keys = orc.selected_keys(gi[g], t, op)
+        o, lse = orc.attend(q[hs], K_seq[:, g], V_seq[:, g], keys, sc)
+        assert np.abs(Og[hs] - o).max() <= O_ATOL
+        assert np.abs(Lg[hs] - lse).max() <= LSE_ATOL
+        if i_ref is not None and np.array_equal(gi[g], i_ref[g]):
+            assert np.abs(Og[hs] - O_ref[hs]).max() <= O_ATOL
+            assert np.abs(Lg[hs] - L_ref[hs]).max() <= LSE_ATOL
+
 def test_decode_steps_small(cuda_lib):
     import torch
     api = cuda_lib
@@ -335,16 +360,10 @@ def test_decode_steps_small(cuda_lib):
                                               wl.bf16_to_f64(data["v_new"][s]), op)
         gi = idx.cpu().numpy()
         Og, Lg = f64(O), f64(lse)
-        G = w.Hq // w.Hkv
         t = L0 + s
         for b in range(B):
-            for g in range(w.Hkv):
-                r = orc.select_query(qf[b, g * G:(g + 1) * G], st.Kc[b][:, g], t, op)
-                check_selection_row(r, gi[b, g], w.topk)
-                if np.array_equal(gi[b, g], i_ref[b, g]):
-                    hs = slice(g * G, (g + 1) * G)
-                    assert np.abs(Og[b, hs] - O_ref[b, hs]).max() <= O_ATOL
-                    assert np.abs(Lg[b, hs] - L_ref[b, hs]).max() <= LSE_ATOL
+            _check_decode_row(st.K[b], st.V[b], st.Kc[b], qf[b], t, gi[b], Og[b], Lg[b], op,
+                              O_ref[b], L_ref[b], i_ref[b])
     assert api.get_status() == 0
     assert seqlens.cpu().tolist() == [L0 + steps] * B
     # incremental compressed keys == batch compression of the final cache
@@ -356,41 +375,50 @@ def test_decode_steps_small(cuda_lib):
     assert torch.equal(batch, Kcmp[:, :nf])
 
 
-def test_decode_full_cache_sampled(cuda_lib):
-    """B=16 sequences over a 131072-token cache: one step, two sequences
-    checked against the oracle (selection by the band rule, output exact)."""
+def test_decode_workload_at_length(cuda_lib):
+    """The decode workload at its size: B=16 sequences over 131072-token
+    caches, 16 consecutive steps.  Afterwards the incrementally built
+    compressed-key cache must equal a batch compression of the final K cache
+    bit for bit, and on six sequences the first and the last step must match
+    the oracle (selection by the band rule; O and LSE of every kv group against
+    the oracle's attention over the GPU's own selection)."""
     import torch
     api = cuda_lib
     w = wl.WORKLOADS["sparse_decode_B16_L131072_Hq32_Hkv2"]
-    B, L0, steps = 16, w.T, 2
+    B, L0, steps = w.B, w.T, 16
     data, p, Kc, Vc, Kcmp, seqlens, ws = _decode_setup(api, w, L0, steps, B)
     O = torch.empty((B, w.Hq, 128), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((B, w.Hq), dtype=torch.float32, device="cuda")
     idx = torch.empty((B, w.Hkv, w.topk), dtype=torch.int32, device="cuda")
-    api.decode_step(p, gpu_bf16(data["q"][0]), gpu_bf16(data["k_new"][0]), gpu_bf16(data["v_new"][0]),
-                    Kc, Vc, Kcmp, seqlens, O, lse, idx, ws)
+    kept = {}
+    for s in range(steps):
+        api.decode_step(p, gpu_bf16(data["q"][s]), gpu_bf16(data["k_new"][s]),
+                        gpu_bf16(data["v_new"][s]), Kc, Vc, Kcmp, seqlens, O, lse, idx, ws)
+        if s in (0, steps - 1):
+            torch.cuda.synchronize()
+            kept[s] = (idx.cpu().numpy(), f64(O), f64(lse))
     torch.cuda.synchronize()
     assert api.get_status() == 0
-    op = orc.Params(topk=w.topk)
-    gi = idx.cpu().numpy()
-    Og, Lg = f64(O), f64(lse)
-    for b in (0, 11):
-        K0 = wl.bf16_to_f64(data["K0"][b])
-        V0 = wl.bf16_to_f64(data["V0"][b])
-        Kseq = np.concatenate([K0, wl.bf16_to_f64(data["k_new"][0][b])[None]], axis=0)
-        Vseq = np.concatenate([V0, wl.bf16_to_f64(data["v_new"][0][b])[None]], axis=0)
+    assert seqlens.cpu().tolist() == [L0 + steps] * B
+    Lf = L0 + steps
+    nf = api.num_compressed(Lf)
+    batch = torch.empty((B, nf, w.Hkv, 2, 128), dtype=torch.bfloat16, device="cuda")
+    api.compress_keys(api.make_params(B, Lf, w.Hq, w.Hkv), Kc[:, :Lf].contiguous(), batch)
+    torch.cuda.synchronize()
+    assert torch.equal(batch, Kcmp[:, :nf])
+    op = orc.Params(topk=w.topk, n_init=w.n_init, n_local=w.n_local)
+    for b in (0, 3, 7, 11, 14, 15):
+        Kseq = np.concatenate([wl.bf16_to_f64(data["K0"][b]),
+                               wl.bf16_to_f64(data["k_new"][:steps, b])], axis=0)
+        Vseq = np.concatenate([wl.bf16_to_f64(data["V0"][b]),
+                               wl.bf16_to_f64(data["v_new"][:steps, b])], axis=0)
         Kc_seq = orc.compress_keys(Kseq[None], op)[0]
-        qf = wl.bf16_to_f64(data["q"][0][b])
-        t = L0
-        G = w.Hq // w.Hkv
-        O_ref, L_ref, i_ref = orc.decode_query(Kseq, Vseq, Kc_seq, qf, t, op)
-        for g in range(w.Hkv):
-            r = orc.select_query(qf[g * G:(g + 1) * G], Kc_seq[:, g], t, op)
-            check_selection_row(r, gi[b, g], w.topk)
-            if np.array_equal(gi[b, g], i_ref[g]):
-                hs = slice(g * G, (g + 1) * G)
-                assert np.abs(Og[b, hs] - O_ref[hs]).max() <= O_ATOL
-                assert np.abs(Lg[b, hs] - L_ref[hs]).max() <= LSE_ATOL
+        for s, (gi, Og, Lg) in kept.items():
+            t = L0 + s
+            qf = wl.bf16_to_f64(data["q"][s][b])
+            O_ref, L_ref, i_ref = orc.decode_query(Kseq[:t + 1], Vseq[:t + 1], Kc_seq, qf, t, op)
+            _check_decode_row(Kseq[:t + 1], Vseq[:t + 1], Kc_seq, qf, t, gi[b], Og[b], Lg[b], op,
+                              O_ref, L_ref, i_ref)
 
 
 def test_decode_full_sequence_is_reported(cuda_lib):
@@ -484,13 +512,8 @@ def test_decode_small_groups(cuda_lib, G):
                                               wl.bf16_to_f64(data["v_new"][s]), op)
         gi, Og, Lg = idx.cpu().numpy(), f64(O), f64(lse)
         for b in range(B):
-            for g in range(Hkv):
-                r = orc.select_query(qf[b, g * G:(g + 1) * G], st.Kc[b][:, g], L0 + s, op)
-                check_selection_row(r, gi[b, g], w.topk)
-                if np.array_equal(gi[b, g], i_ref[b, g]):
-                    hs = slice(g * G, (g + 1) * G)
-                    assert np.abs(Og[b, hs] - O_ref[b, hs]).max() <= O_ATOL
-                    assert np.abs(Lg[b, hs] - L_ref[b, hs]).max() <= LSE_ATOL
+            _check_decode_row(st.K[b], st.V[b], st.Kc[b], qf[b], L0 + s, gi[b], Og[b], Lg[b], op,
+                              O_ref[b], L_ref[b], i_ref[b])
     assert api.get_status() == 0
 
 

@@ -52,6 +52,7 @@ cudaError_t get_dev_ctx(DevCtx* ctx) {
 int sm_count() {
   const int d = current_device();
   if (d < 0 || d >= kMaxDevices) return 148;
+  std::lock_guard<std::mutex> lk(g_mu);
   if (!g_sm_count[d]) {
     int n = 0;
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d);
@@ -127,6 +128,12 @@ size_t select_ws_bytes(const Geometry& g) {
          sizeof(float);
 }
 
+// Block selection holds a row's block scores in registers: sequences of at
+// most INFLLMV2_MAX_SELECT_T tokens (4096 blocks); checked before any launch.
+int check_select_size(const Geometry& g) {
+  return g.T > INFLLMV2_MAX_SELECT_T ? INFLLMV2_ERR_UNSUPPORTED : INFLLMV2_OK;
+}
+
 // validate() plus the query range of a prefill chunk.
 int validate_chunk(const infllmv2_params* p, int32_t q_offset, int32_t q_len, Geometry* g) {
   if (int e = validate(p, true, g)) return e;
@@ -171,13 +178,19 @@ void infllmv2_set_wait_limit(int64_t ns) {
 
 size_t infllmv2_workspace_bytes(const infllmv2_params* p, int32_t op) {
   Geometry g;
-  if (validate(p, op != 0, &g) != INFLLMV2_OK) return SIZE_MAX;
+  // the dense operations take no top-k parameters (as infllmv2_dense_attn)
+  const bool dense_only = op == INFLLMV2_OP_ATTN ||
+                          (op == INFLLMV2_OP_FORWARD && p && p->T <= p->switch_threshold);
+  if (validate(p, !dense_only, &g) != INFLLMV2_OK) return SIZE_MAX;
   switch (op) {
-    case INFLLMV2_OP_SELECT: return select_ws_bytes(g);
+    case INFLLMV2_OP_SELECT:
+      return check_select_size(g) ? SIZE_MAX : select_ws_bytes(g);
     case INFLLMV2_OP_FORWARD:
-      return p->T <= p->switch_threshold ? packed_kv_bytes(g)
-                                         : align256(select_ws_bytes(g)) + packed_kv_bytes(g);
-    case INFLLMV2_OP_DECODE: return decode_ws_bytes(g);
+      if (p->T <= p->switch_threshold) return packed_kv_bytes(g);
+      return check_select_size(g) ? SIZE_MAX
+                                  : align256(select_ws_bytes(g)) + packed_kv_bytes(g);
+    case INFLLMV2_OP_DECODE:
+      return g.T > INFLLMV2_MAX_DECODE_T ? SIZE_MAX : decode_ws_bytes(g);
     case INFLLMV2_OP_ATTN: return packed_kv_bytes(g);
     default: return SIZE_MAX;
   }
@@ -195,6 +208,7 @@ int infllmv2_select_blocks(const infllmv2_params* p, const void* Q, const void* 
                            void* ws, size_t ws_bytes, void* stream) {
   Geometry g;
   if (int e = validate(p, true, &g)) return e;
+  if (int e = check_select_size(g)) return e;
   if (empty(g)) return INFLLMV2_OK;
   if (int e = check_ptrs({Q, idx, ws})) return e;
   if (g.n_c > 0)
@@ -250,6 +264,7 @@ int infllmv2_forward(const infllmv2_params* p, const void* Q, const void* K, con
   if (dense) return infllmv2_dense_attn(p, Q, K, V, O, lse, ws, ws_bytes, stream);
   Geometry g;
   if (int e = validate(p, true, &g)) return e;
+  if (int e = check_select_size(g)) return e;
   if (empty(g)) return INFLLMV2_OK;
   // workspace: block scores of the selection, then the packed K/V tiles
   const size_t sel = align256(select_ws_bytes(g));
@@ -265,8 +280,8 @@ size_t infllmv2_prefill_chunk_workspace_bytes(const infllmv2_params* p, int32_t 
                                               int32_t q_len) {
   Geometry g;
   if (validate_chunk(p, q_offset, q_len, &g) != INFLLMV2_OK) return SIZE_MAX;
-  return p->T <= p->switch_threshold ? packed_kv_bytes(g)
-                                     : align256(select_ws_bytes(g)) + packed_kv_bytes(g);
+  if (p->T <= p->switch_threshold) return packed_kv_bytes(g);
+  return check_select_size(g) ? SIZE_MAX : align256(select_ws_bytes(g)) + packed_kv_bytes(g);
 }
 
 int infllmv2_prefill_chunk(const infllmv2_params* p, int32_t q_offset, int32_t q_len,
@@ -276,6 +291,8 @@ int infllmv2_prefill_chunk(const infllmv2_params* p, int32_t q_offset, int32_t q
   Geometry g;
   if (int e = validate_chunk(p, q_offset, q_len, &g)) return e;
   const bool dense = p->T <= p->switch_threshold;
+  if (!dense)
+    if (int e = check_select_size(g)) return e;
   if (path_used) *path_used = dense ? INFLLMV2_PATH_DENSE : INFLLMV2_PATH_SPARSE;
   if (g.B == 0 || g.Tq == 0) return INFLLMV2_OK;
   if (int e = check_ptrs({Q, K, V, O, lse})) return e;
@@ -307,6 +324,7 @@ int infllmv2_decode_step(const infllmv2_params* p, const void* q, const void* k_
                          size_t ws_bytes, void* stream) {
   Geometry g;
   if (int e = validate(p, true, &g)) return e;
+  if (g.T > INFLLMV2_MAX_DECODE_T) return INFLLMV2_ERR_UNSUPPORTED;
   if (g.B == 0) return INFLLMV2_OK;
   if (g.T < 1) return INFLLMV2_ERR_INVALID_ARG;
   if (int e = check_ptrs({q, k_new, v_new, K_cache, V_cache, seqlens, O, lse, ws})) return e;
@@ -359,6 +377,7 @@ int infllmv2_decode_step_noalloc(const infllmv2_params* p, const void* q, const 
                                  int32_t* idx_out, void* stream) {
   Geometry g;
   if (int e = validate(p, true, &g)) return e;
+  if (g.T > INFLLMV2_MAX_DECODE_T) return INFLLMV2_ERR_UNSUPPORTED;
   if (g.B == 0) return INFLLMV2_OK;
   if (g.T < 1) return INFLLMV2_ERR_INVALID_ARG;
   if (int e = check_ptrs({q, k_new, v_new, K_cache, V_cache, seqlens, O, lse})) return e;

@@ -124,21 +124,8 @@ __device__ __forceinline__ int count_valid(const int32_t* __restrict__ row, int 
   return n;
 }
 
-// The same count by one thread alone.
-__device__ __forceinline__ int count_valid_1(const int32_t* __restrict__ row, int topk, int cur) {
-  int n = 0;
-  while (n < topk) {
-    const int v = __ldg(row + n);
-    if (v < 0 || v > cur) break;
-    ++n;
-  }
-  return n;
-}
-
-// Resolves work item `it`.  collective: called by a whole warp (every lane
-// gets the same answer); otherwise by a single thread.
-__device__ __forceinline__ Item resolve_item(int64_t it, const AttnArgs& a, int lane,
-                                             bool collective) {
+// Resolves work item `it` (warp-collective: every lane gets the same answer).
+__device__ __forceinline__ Item resolve_item(int64_t it, const AttnArgs& a, int lane) {
   Item r;
   if (a.mode == 2) {
     const int c = static_cast<int>(it % a.n_chunks);
@@ -150,9 +137,7 @@ __device__ __forceinline__ Item resolve_item(int64_t it, const AttnArgs& a, int 
     r.cur = r.t / kBlock;
     r.row = a.idx + bg * a.topk;
     int nv = 0;
-    if (r.t >= 0 && r.t < a.T)
-      nv = collective ? count_valid(r.row, a.topk, r.cur, lane)
-                      : count_valid_1(r.row, a.topk, r.cur);
+    if (r.t >= 0 && r.t < a.T) nv = count_valid(r.row, a.topk, r.cur, lane);
     r.e0 = c * a.chunk_blocks;
     r.n = max(0, min(a.chunk_blocks, nv - r.e0));
   } else {
@@ -169,8 +154,7 @@ __device__ __forceinline__ Item resolve_item(int64_t it, const AttnArgs& a, int 
       r.n = r.cur + 1;
     } else {
       r.row = a.idx + ((static_cast<int64_t>(r.b) * a.Hkv + r.g) * a.Tq + r.qtok) * a.topk;
-      r.n = collective ? count_valid(r.row, a.topk, r.cur, lane)
-                       : count_valid_1(r.row, a.topk, r.cur);
+      r.n = count_valid(r.row, a.topk, r.cur, lane);
     }
   }
   r.n_pairs = (r.n + 1) >> 1;
@@ -323,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int qk = 0;           // Q loads issued
     bool ok = true;
     for (int64_t k = 0, it; ok && (it = item_of(k, n_items)) < n_items; ++k) {
-      const Item item = resolve_item(it, args, lane, true);
+      const Item item = resolve_item(it, args, lane);
       if (item.n_pairs == 0) continue;
       if (lane == 0) {
         const int qb = qk & 1;
@@ -378,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int qk = 0;      // items whose Q has been used (S issuer)
     bool ok = true;
     for (int64_t k = 0, it; ok && (it = item_of(k, n_items)) < n_items; ++k) {
-      const Item item = resolve_item(it, args, lane, true);
+      const Item item = resolve_item(it, args, lane);
       if (item.n_pairs == 0) continue;
       if (lane == 0 && pv_role) {
         for (int p = 0; ok && p < item.n_pairs; ++p, ++gp) {
@@ -467,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int64_t gp = 0;
     bool ok = true;
     for (int64_t k = 0, it; ok && (it = item_of(k, n_items)) < n_items; ++k) {
-      const Item item = resolve_item(it, args, lane, true);
+      const Item item = resolve_item(it, args, lane);
       // the item's blocks, staged once in shared memory by all 256 threads
       if (item.row)
         for (int e = gt; e < item.n; e += kSoftmaxThreads)

@@ -36,7 +36,7 @@ EXPORTS = (
     "infllmv2_workspace_bytes", "infllmv2_num_compressed", "infllmv2_get_status",
     "infllmv2_set_wait_limit", "infllmv2_selftest_timeout", "infllmv2_strerror",
     "infllmv2_version", "infllmv2_decode_step_noalloc", "infllmv2_prefill_chunk",
-    "infllmv2_prefill_chunk_workspace_bytes",
+    "infllmv2_prefill_chunk_workspace_bytes", "infllmv2_gather_peak",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -100,6 +100,7 @@ def load(path: Optional[str] = None):
         "infllmv2_selftest_timeout": (ctypes.c_int, [vp]),
         "infllmv2_strerror": (ctypes.c_char_p, [ctypes.c_int]),
         "infllmv2_version": (ctypes.c_int, []),
+        "infllmv2_gather_peak": (ctypes.c_int, [vp, sz, i32, ctypes.POINTER(i32), vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -150,6 +151,16 @@ def set_wait_limit(ns: int):
 
 def selftest_timeout(stream=None):
     _check("infllmv2_selftest_timeout", load().infllmv2_selftest_timeout(_stream(stream)))
+
+
+def gather_peak(src, rounds: int, stream=None) -> int:
+    """Enqueues the L2 -> shared-memory gather measurement over the device
+    buffer ``src``; returns the bytes it moves (the caller times it)."""
+    ctas = ctypes.c_int32(0)
+    _check("infllmv2_gather_peak",
+           load().infllmv2_gather_peak(_ptr(src), src.numel() * src.element_size(), int(rounds),
+                                       ctypes.byref(ctas), _stream(stream)))
+    return int(ctas.value) * int(rounds) * 3 * 65536
 
 
 # --------------------------------------------------------------------------
