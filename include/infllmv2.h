@@ -94,7 +94,8 @@ typedef struct infllmv2_params {
 #define INFLLMV2_OP_SELECT   1
 #define INFLLMV2_OP_FORWARD  2
 #define INFLLMV2_OP_DECODE   3
-#define INFLLMV2_OP_ATTN     4  /* sparse_attn / dense_attn: packed K and V */
+#define INFLLMV2_OP_ATTN     4  /* sparse_attn: union lists (groups of 8 or 16 heads) or packed K/V */
+#define INFLLMV2_OP_ATTN_PER_TOKEN 5  /* sparse_attn_per_token: packed K and V */
 
 /* Path reported by infllmv2_forward. */
 #define INFLLMV2_PATH_DENSE  1
@@ -143,25 +144,60 @@ int infllmv2_select_blocks(const infllmv2_params* p, const void* Q, const void* 
  *   lse[b,h,t] = log sum_{i in keys(t)} exp(scale * q.K_i).
  *   idx rows must be ascending with valid entries first (as select_blocks
  *   writes them); entries > t/64 are ignored.
- *   ws: optional device workspace of infllmv2_workspace_bytes(p,
- *   INFLLMV2_OP_ATTN) bytes.  With it, K and V are first repacked into
- *   block-contiguous tiles (one 16 KB chunk per 64-key block and kv head) so
- *   that every selected block is gathered by one bulk copy; with ws == NULL
- *   (or ws_bytes too small for it) blocks are gathered from K and V directly
- *   by tensor-map copies, which is slower.  Results are identical.
+ * Schedule: with Hq/Hkv in {8, 16} and ws of at least
+ * infllmv2_workspace_bytes(p, INFLLMV2_OP_ATTN) bytes, query tiles of 128
+ * rows (128/G tokens x G heads) run over the union of their tokens' selected
+ * blocks, each row masked to its own token's blocks, so a block that several
+ * tokens of a tile selected is loaded and multiplied once (ws holds the
+ * union lists; contents on return unspecified).  Otherwise (smaller groups, or
+ * ws NULL / too small) the call runs infllmv2_sparse_attn_per_token's
+ * schedule.  Results agree within rounding.
  */
 int infllmv2_sparse_attn(const infllmv2_params* p, const void* Q, const void* K,
                          const void* V, const int32_t* idx, void* O, float* lse, void* ws,
                          size_t ws_bytes, void* stream);
 
 /*
+ * infllmv2_sparse_attn with one work item per query token: the token's G
+ * heads against its own selected blocks only, two blocks per tensor-core
+ * product with keys on the 128-row side.  ws: optional, at least
+ * infllmv2_workspace_bytes(p, INFLLMV2_OP_ATTN_PER_TOKEN) bytes: K and V are
+ * first repacked into block-contiguous tiles (one 16 KB chunk per 64-key
+ * block and kv head) so that every selected block is gathered by one bulk
+ * copy; with ws NULL (or too small) blocks are gathered from K and V by
+ * tensor-map copies.  Same arguments and results as infllmv2_sparse_attn.
+ */
+int infllmv2_sparse_attn_per_token(const infllmv2_params* p, const void* Q, const void* K,
+                                   const void* V, const int32_t* idx, void* O, float* lse,
+                                   void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Exact dense causal attention (skill write-up, Architecture Overview, the
- * dense pathway bullet): keys(t) = [0, t], same O and lse
- * definitions as infllmv2_sparse_attn; ws as for infllmv2_sparse_attn.
+ * dense pathway bullet): keys(t) = [0, t], same O and lse definitions as
+ * infllmv2_sparse_attn.  Query tiles of 128 rows against 128-key tiles on the
+ * tensor cores.  ws and ws_bytes are unused (may be NULL / 0).
  */
 int infllmv2_dense_attn(const infllmv2_params* p, const void* Q, const void* K,
                         const void* V, void* O, float* lse, void* ws, size_t ws_bytes,
                         void* stream);
+
+/*
+ * The compressed-attention branch (skill write-up, Core Concept: the
+ * compressed pattern aggregates tokens hierarchically into representatives
+ * that every query can attend to): each query row attends over the compressed
+ * windows it can see,
+ *   keys(t) = { j : 16 j + 31 <= t, j < n_c },
+ *   O[b,t,h,:] = sum_{j in keys(t)} softmax_j(scale * q . Kc[j]) Vc[j],
+ *   lse[b,h,t] = log sum_{j in keys(t)} exp(scale * q . Kc[j]);
+ * a row with no visible window (t < 31) gets O = 0 and lse = -inf.
+ *   Q [B, T, Hq, d] bf16 (in);
+ *   Kc = infllmv2_compress_keys of K, Vc = infllmv2_compress_keys of V
+ *     ([B, n_c, Hkv, 2, d] bf16, in; scores use both planes of Kc, the values
+ *     the high plane of Vc);
+ *   O [B, T, Hq, d] bf16, lse [B, Hq, T] fp32 (out).
+ */
+int infllmv2_compressed_attn(const infllmv2_params* p, const void* Q, const void* Kc,
+                             const void* Vc, void* O, float* lse, void* stream);
 
 /*
  * The switchable attention (skill write-up, Implementation Step 3: dense when
@@ -170,7 +206,8 @@ int infllmv2_dense_attn(const infllmv2_params* p, const void* Q, const void* K,
  * idx_ws may be NULL.  *path_used (host pointer, may be NULL) receives
  * INFLLMV2_PATH_DENSE or INFLLMV2_PATH_SPARSE.
  *   Kc_ws: [B, n_c, Hkv, 2, d] bf16; idx_ws: [B, Hkv, T, topk] int32 (both out);
- *   ws: at least infllmv2_workspace_bytes(p, INFLLMV2_OP_FORWARD) bytes.
+ *   ws: at least infllmv2_workspace_bytes(p, INFLLMV2_OP_FORWARD) bytes (0 when
+ *   dense): the selection's block scores, then infllmv2_sparse_attn's.
  */
 int infllmv2_forward(const infllmv2_params* p, const void* Q, const void* K,
                      const void* V, void* O, float* lse, void* Kc_ws, int32_t* idx_ws,
@@ -193,8 +230,7 @@ int infllmv2_forward(const infllmv2_params* p, const void* Q, const void* K,
  *   idx [B, Hkv, q_len, topk] int32 (out; unused and may be NULL when dense);
  *   path_used: host int32 (may be NULL);
  *   ws: at least infllmv2_prefill_chunk_workspace_bytes(p, q_offset, q_len)
- *     bytes (dense: may be smaller, down to 0; the K/V gather then uses
- *     tensor-map boxes instead of packed tiles).
+ *     bytes (0 when dense).
  */
 size_t infllmv2_prefill_chunk_workspace_bytes(const infllmv2_params* p, int32_t q_offset,
                                               int32_t q_len);

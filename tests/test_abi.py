@@ -56,23 +56,58 @@ def test_host_helpers(lib):
         assert lib.infllmv2_strerror(code)
 
 
+def _union_bytes(B, T, Hkv, G, topk):
+    """Union lists of the query-tile schedule: per tile of 128/G tokens, room
+    for every token's topk entries (256-byte aligned), then one count per tile."""
+    tpt = 128 // G
+    tiles = B * Hkv * (-(-T // tpt))
+    return (-(-(tiles * tpt * topk * 4) // 256) * 256) + tiles * 4
+
+
+def _packed_bytes(B, T, Hkv):
+    return 2 * B * Hkv * (-(-T // 64)) * 16384
+
+
 def test_workspace_sizes(lib):
     p = api.make_params(1, 131072, 32, 2, topk=64)
     # causally packed block scores: sum_t (t//64 + 1) floats per (b, kv head)
     T = 131072
     per = sum((t // 64 + 1) for t in range(0, T, 64)) * 64
     assert api.workspace_bytes(p, api.OP_SELECT) == 2 * per * 4
+    # groups of 16 heads: the query-tile schedule's union lists
+    assert api.workspace_bytes(p, api.OP_ATTN) == _union_bytes(1, T, 2, 16, 64)
+    assert api.workspace_bytes(p, api.OP_ATTN_PER_TOKEN) == _packed_bytes(1, T, 2)
+    # smaller groups: the per-token schedule's packed K/V tiles
+    p4 = api.make_params(1, 2048, 8, 2, topk=8)
+    assert api.workspace_bytes(p4, api.OP_ATTN) == _packed_bytes(1, 2048, 2)
+    p8 = api.make_params(1, 2000, 16, 2, topk=8)
+    assert api.workspace_bytes(p8, api.OP_ATTN) == _union_bytes(1, 2000, 2, 8, 8)
+    # the dense forward needs no workspace
     dense = api.make_params(2, 4096, 32, 2, switch_threshold=8192)
-    # dense forward: only the packed K/V tiles (2 tensors x B x Hkv x blocks x 16 KB)
-    assert api.workspace_bytes(dense, api.OP_FORWARD) == 2 * 2 * 2 * 64 * 16384
-    assert api.workspace_bytes(dense, api.OP_ATTN) == 2 * 2 * 2 * 64 * 16384
-    # sparse forward: block scores (256-byte aligned) then the tiles
+    assert api.workspace_bytes(dense, api.OP_FORWARD) == 0
+    # sparse forward: block scores (256-byte aligned) then the attention's
     assert api.workspace_bytes(p, api.OP_FORWARD) == \
         (-(-api.workspace_bytes(p, api.OP_SELECT) // 256) * 256) + api.workspace_bytes(p, api.OP_ATTN)
     assert api.workspace_bytes(api.make_params(16, 131328, 32, 2), api.OP_DECODE) > 0
     bad = api.make_params(1, 100, 32, 2, head_dim=64)
     with pytest.raises(api.InfLLMV2Error):
         api.workspace_bytes(bad, api.OP_SELECT)
+    # sizes beyond the selection / decode limits are refused before any launch
+    with pytest.raises(api.InfLLMV2Error):
+        api.workspace_bytes(api.make_params(1, 262144 + 64, 32, 2), api.OP_SELECT)
+    with pytest.raises(api.InfLLMV2Error):
+        api.workspace_bytes(api.make_params(1, 524288 + 64, 32, 2), api.OP_DECODE)
+
+
+def test_size_limits_rejected_before_any_launch(lib):
+    big = api.make_params(1, 262144 + 64, 32, 2, topk=64, switch_threshold=0)
+    P = ctypes.byref(big)
+    assert lib.infllmv2_select_blocks(P, FAKE, FAKE, FAKE, FAKE, 1 << 40, None) == api.ERR_UNSUPPORTED
+    assert lib.infllmv2_forward(P, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 40,
+                                None) == api.ERR_UNSUPPORTED
+    dec = api.make_params(1, 524288 + 64, 32, 2, topk=64)
+    assert lib.infllmv2_decode_step(ctypes.byref(dec), *([FAKE] * 11), 1 << 40, None) == \
+        api.ERR_UNSUPPORTED
 
 
 FAKE = 0x10000  # never dereferenced: validation fails first
@@ -134,11 +169,11 @@ def test_prefill_chunk_workspace_sizes(lib):
     p = api.make_params(1, 131072, 32, 2, topk=64, switch_threshold=8192)
     # the whole sequence as one chunk needs what forward needs
     assert api.prefill_chunk_workspace_bytes(p, 0, 131072) == api.workspace_bytes(p, api.OP_FORWARD)
-    # a tail chunk: the block scores of its rows only, then the packed K/V of all tokens
+    # a tail chunk: the block scores of its rows only, then the union lists of its tiles
     q0, n = 131072 - 4096, 4096
     rows = sum(t // 64 + 1 for t in range(q0, q0 + n))
     sel = 2 * rows * 4
     assert api.prefill_chunk_workspace_bytes(p, q0, n) == \
-        (-(-sel // 256) * 256) + api.workspace_bytes(p, api.OP_ATTN)
+        (-(-sel // 256) * 256) + _union_bytes(1, n, 2, 16, 64)
     d = api.make_params(1, 4096, 32, 2, switch_threshold=8192)
-    assert api.prefill_chunk_workspace_bytes(d, 1000, 3096) == api.workspace_bytes(d, api.OP_ATTN)
+    assert api.prefill_chunk_workspace_bytes(d, 1000, 3096) == 0

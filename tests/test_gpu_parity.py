@@ -128,9 +128,27 @@ def test_select_exact_ties_go_to_lower_blocks(cuda_lib, case):
 # ---------------------------------------------------------------------------
 # attention with the oracle's selection
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("packed", [True, False], ids=["packed_kv", "tensor_map_gather"])
+SCHEDULES = ["query_tiles", "per_token_packed", "per_token_tensor_map"]
+
+
+def _run_sparse(api, p, schedule, Q, K, V, idx, O, lse):
+    """The block-sparse attention under one of its schedules: query tiles over
+    each tile's union of blocks (sparse_attn with its workspace; groups of 8
+    or 16 heads, smaller groups fall back to the per-token schedule), one item
+    per token gathering packed tiles, or one item per token gathering from K
+    and V by tensor maps (no workspace)."""
+    if schedule == "query_tiles":
+        api.sparse_attn(p, Q, K, V, idx, O, lse, api.alloc_workspace(p, api.OP_ATTN))
+    elif schedule == "per_token_packed":
+        api.sparse_attn_per_token(p, Q, K, V, idx, O, lse,
+                                  api.alloc_workspace(p, api.OP_ATTN_PER_TOKEN))
+    else:
+        api.sparse_attn_per_token(p, Q, K, V, idx, O, lse, None)
+
+
+@pytest.mark.parametrize("schedule", SCHEDULES)
 @pytest.mark.parametrize("case", SMALL, ids=[f"B{c[0]}_T{c[1]}_Hq{c[2]}_Hkv{c[3]}_k{c[4]}" for c in SMALL])
-def test_sparse_attn_all_rows(cuda_lib, case, packed):
+def test_sparse_attn_all_rows(cuda_lib, case, schedule):
     import torch
     api = cuda_lib
     B, T, Hq, Hkv, topk, needles, seed = case
@@ -143,9 +161,46 @@ def test_sparse_attn_all_rows(cuda_lib, case, packed):
     O = torch.empty((B, T, Hq, 128), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((B, Hq, T), dtype=torch.float32, device="cuda")
     p = _params(api, w)
-    ws = api.alloc_workspace(p, api.OP_ATTN) if packed else None
-    api.sparse_attn(p, gpu_bf16(data["Q"]), gpu_bf16(data["K"]), gpu_bf16(data["V"]),
-                    torch.from_numpy(idx).cuda(), O, lse, ws)
+    _run_sparse(api, p, schedule, gpu_bf16(data["Q"]), gpu_bf16(data["K"]), gpu_bf16(data["V"]),
+                torch.from_numpy(idx).cuda(), O, lse)
+    torch.cuda.synchronize()
+    assert api.get_status() == 0
+    assert np.abs(f64(O) - O_ref).max() <= O_ATOL
+    assert np.abs(f64(lse) - L_ref).max() <= LSE_ATOL
+
+
+@pytest.mark.parametrize("shared", [True, False], ids=["tokens_share_blocks", "tokens_disjoint"])
+def test_query_tile_union_extremes(cuda_lib, shared):
+    """The query-tile schedule at the two ends of block sharing: every token
+    of a tile selecting the same blocks (union = one token's set), and
+    neighbouring tokens selecting disjoint blocks (union = 8 x topk)."""
+    import torch
+    api = cuda_lib
+    B, T, Hq, Hkv, topk = 1, 2500, 32, 2, 6
+    w = wl.small_workload(B=B, T=T, Hq=Hq, Hkv=Hkv, topk=topk, needles=0, seed=31)
+    data = wl.make_prefill(w)
+    Q, K, V = (wl.bf16_to_f64(data[x]) for x in "QKV")
+    rng = np.random.default_rng(5)
+    idx = np.full((B, Hkv, T, topk), -1, dtype=np.int32)
+    for g in range(Hkv):
+        for t in range(T):
+            cur = t // 64
+            free = [b for b in range(1, cur - 1)]
+            if shared:
+                r = np.random.default_rng(1000 * g + t // 8)   # one choice per 8-token tile
+            else:
+                r = rng
+            k = min(topk - 3, len(free))
+            pick = sorted(set([0, max(cur - 1, 0), cur] + list(r.choice(free, size=k, replace=False)))) \
+                if free else sorted(set([0, max(cur - 1, 0), cur]))
+            idx[0, g, t, :len(pick)] = pick
+    op = orc.Params(topk=topk)
+    O_ref, L_ref = orc.sparse_attention(Q, K, V, idx, op)
+    O = torch.empty((B, T, Hq, 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, Hq, T), dtype=torch.float32, device="cuda")
+    p = _params(api, w)
+    _run_sparse(api, p, "query_tiles", gpu_bf16(data["Q"]), gpu_bf16(data["K"]), gpu_bf16(data["V"]),
+                torch.from_numpy(idx).cuda(), O, lse)
     torch.cuda.synchronize()
     assert api.get_status() == 0
     assert np.abs(f64(O) - O_ref).max() <= O_ATOL
@@ -183,9 +238,12 @@ def test_sparse_attn_unsorted_padding_and_ignored_entries(cuda_lib):
 # ---------------------------------------------------------------------------
 # dense path and the switch
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("packed", [True, False], ids=["packed_kv", "tensor_map_gather"])
-@pytest.mark.parametrize("B,T,Hq,Hkv", [(1, 300, 32, 2), (2, 130, 8, 2), (1, 1, 16, 1)])
-def test_dense_attn_all_rows(cuda_lib, B, T, Hq, Hkv, packed):
+DENSE = [(1, 300, 32, 2), (2, 130, 8, 2), (1, 1, 16, 1), (1, 1000, 16, 1), (1, 700, 2, 2),
+         (2, 333, 16, 2), (1, 517, 4, 2)]
+
+
+@pytest.mark.parametrize("B,T,Hq,Hkv", DENSE, ids=[f"B{c[0]}_T{c[1]}_Hq{c[2]}_Hkv{c[3]}" for c in DENSE])
+def test_dense_attn_all_rows(cuda_lib, B, T, Hq, Hkv):
     import torch
     api = cuda_lib
     w = wl.small_workload(B=B, T=T, Hq=Hq, Hkv=Hkv, needles=0, seed=T + Hq)
@@ -195,11 +253,67 @@ def test_dense_attn_all_rows(cuda_lib, B, T, Hq, Hkv, packed):
     O = torch.empty((B, T, Hq, 128), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((B, Hq, T), dtype=torch.float32, device="cuda")
     p = _params(api, w)
-    ws = api.alloc_workspace(p, api.OP_ATTN) if packed else None
-    api.dense_attn(p, gpu_bf16(data["Q"]), gpu_bf16(data["K"]), gpu_bf16(data["V"]), O, lse, ws)
+    api.dense_attn(p, gpu_bf16(data["Q"]), gpu_bf16(data["K"]), gpu_bf16(data["V"]), O, lse)
     torch.cuda.synchronize()
+    assert api.get_status() == 0
     assert np.abs(f64(O) - O_ref).max() <= O_ATOL
     assert np.abs(f64(lse) - L_ref).max() <= LSE_ATOL
+
+
+# ---------------------------------------------------------------------------
+# the compressed-attention branch
+# ---------------------------------------------------------------------------
+CMP = [(1, 700, 32, 2), (1, 1000, 8, 2), (2, 300, 16, 1), (1, 31, 32, 2), (1, 47, 16, 2),
+       (1, 1500, 2, 2)]
+
+
+def _run_compressed(api, w, data):
+    import torch
+    p = _params(api, w)
+    n_c = api.num_compressed(w.T)
+    K, V = gpu_bf16(data["K"]), gpu_bf16(data["V"])
+    Kc = torch.empty((w.B, max(n_c, 1), w.Hkv, 2, 128), dtype=torch.bfloat16, device="cuda")
+    Vc = torch.empty_like(Kc)
+    if n_c:
+        api.compress_keys(p, K, Kc)
+        api.compress_keys(p, V, Vc)
+    O = torch.full((w.B, w.T, w.Hq, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((w.B, w.Hq, w.T), float("nan"), dtype=torch.float32, device="cuda")
+    api.compressed_attn(p, gpu_bf16(data["Q"]), Kc, Vc, O, lse)
+    torch.cuda.synchronize()
+    assert api.get_status() == 0
+    return f64(O), f64(lse)
+
+
+@pytest.mark.parametrize("B,T,Hq,Hkv", CMP, ids=[f"B{c[0]}_T{c[1]}_Hq{c[2]}_Hkv{c[3]}" for c in CMP])
+def test_compressed_attn_all_rows(cuda_lib, B, T, Hq, Hkv):
+    w = wl.small_workload(B=B, T=T, Hq=Hq, Hkv=Hkv, needles=2, seed=T + 3 * Hq)
+    data = wl.make_prefill(w)
+    Og, Lg = _run_compressed(cuda_lib, w, data)
+    Q, K, V = (wl.bf16_to_f64(data[x]) for x in "QKV")
+    O_ref, L_ref = orc.compressed_attention(Q, K, V, orc.Params())
+    none = np.isneginf(L_ref)            # rows that see no window: O = 0, lse = -inf
+    assert np.array_equal(np.isneginf(Lg), none)
+    assert np.abs(Og - O_ref).max() <= O_ATOL
+    assert np.abs(Lg[~none] - L_ref[~none]).max() <= LSE_ATOL
+
+
+def test_compressed_attn_32k_sampled(cuda_lib):
+    w = wl.WORKLOADS["sparse_prefill_T32768_Hq32_Hkv2"]
+    data = wl.make_prefill(w)
+    Og, Lg = _run_compressed(cuda_lib, w, data)
+    Q, K, V = (wl.bf16_to_f64(data[x]) for x in "QKV")
+    needle_rows = [nd.query_block * 64 + 5 for nd in data["needles"][:8]]
+    rows = [(0, g, t) for g in range(w.Hkv) for t in sample_rows(w.T, 40, 9, needle_rows)]
+    O_ref, L_ref = orc.compressed_attention(Q, K, V, orc.Params(), rows)
+    G = w.Hq // w.Hkv
+    for (b, g, t) in rows:
+        hs = slice(g * G, (g + 1) * G)
+        assert np.abs(Og[b, t, hs] - O_ref[b, t, hs]).max() <= O_ATOL
+        if t >= 31:
+            assert np.abs(Lg[b, hs, t] - L_ref[b, hs, t]).max() <= LSE_ATOL
+        else:
+            assert np.all(np.isneginf(Lg[b, hs, t]))
 
 
 def test_dense_switch_workload_sampled(cuda_lib):

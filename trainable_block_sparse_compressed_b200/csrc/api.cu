@@ -134,6 +134,28 @@ int check_select_size(const Geometry& g) {
   return g.T > INFLLMV2_MAX_SELECT_T ? INFLLMV2_ERR_UNSUPPORTED : INFLLMV2_OK;
 }
 
+// Workspace of the block-sparse attention: the union lists of the query-tile
+// schedule (groups of 8 or 16 heads), else the packed K/V tiles of the
+// per-token schedule.
+size_t attn_ws_bytes(const Geometry& g) {
+  return union_supported(g) ? union_ws_bytes(g) : packed_kv_bytes(g);
+}
+
+// Enqueues the block-sparse attention: the query-tile schedule over each
+// tile's union of selected blocks when the group allows it and the workspace
+// holds its lists; else one work item per query token, gathering from packed
+// K/V tiles when the workspace holds them, from K and V directly otherwise.
+int enqueue_sparse(const Geometry& g, const void* Q, const void* K, const void* V,
+                   const int32_t* idx, void* O, float* lse, void* ws, size_t ws_bytes,
+                   bool per_token, const DevCtx& ctx, cudaStream_t st) {
+  if (!per_token && union_supported(g) && ws && ws_bytes >= union_ws_bytes(g))
+    return launch_union_tile(g, Q, K, V, idx, O, lse, ws, ctx, st);
+  const bool pack = ws && ws_bytes >= packed_kv_bytes(g);
+  if (pack)
+    if (int e = launch_pack_kv(g, K, V, ws, st)) return e;
+  return launch_sparse_attn(g, Q, K, V, idx, O, lse, pack ? ws : nullptr, ctx, st);
+}
+
 // validate() plus the query range of a prefill chunk.
 int validate_chunk(const infllmv2_params* p, int32_t q_offset, int32_t q_len, Geometry* g) {
   if (int e = validate(p, true, g)) return e;
@@ -178,20 +200,19 @@ void infllmv2_set_wait_limit(int64_t ns) {
 
 size_t infllmv2_workspace_bytes(const infllmv2_params* p, int32_t op) {
   Geometry g;
-  // the dense operations take no top-k parameters (as infllmv2_dense_attn)
-  const bool dense_only = op == INFLLMV2_OP_ATTN ||
-                          (op == INFLLMV2_OP_FORWARD && p && p->T <= p->switch_threshold);
-  if (validate(p, !dense_only, &g) != INFLLMV2_OK) return SIZE_MAX;
+  // the dense forward takes no top-k parameters (as infllmv2_dense_attn)
+  const bool dense_fwd = op == INFLLMV2_OP_FORWARD && p && p->T <= p->switch_threshold;
+  if (validate(p, !dense_fwd, &g) != INFLLMV2_OK) return SIZE_MAX;
   switch (op) {
     case INFLLMV2_OP_SELECT:
       return check_select_size(g) ? SIZE_MAX : select_ws_bytes(g);
     case INFLLMV2_OP_FORWARD:
-      if (p->T <= p->switch_threshold) return packed_kv_bytes(g);
-      return check_select_size(g) ? SIZE_MAX
-                                  : align256(select_ws_bytes(g)) + packed_kv_bytes(g);
+      if (dense_fwd) return 0;
+      return check_select_size(g) ? SIZE_MAX : align256(select_ws_bytes(g)) + attn_ws_bytes(g);
     case INFLLMV2_OP_DECODE:
       return g.T > INFLLMV2_MAX_DECODE_T ? SIZE_MAX : decode_ws_bytes(g);
-    case INFLLMV2_OP_ATTN: return packed_kv_bytes(g);
+    case INFLLMV2_OP_ATTN: return attn_ws_bytes(g);
+    case INFLLMV2_OP_ATTN_PER_TOKEN: return packed_kv_bytes(g);
     default: return SIZE_MAX;
   }
 }
@@ -232,27 +253,48 @@ int infllmv2_sparse_attn(const infllmv2_params* p, const void* Q, const void* K,
   if (ws && !aligned16(ws)) return INFLLMV2_ERR_UNSUPPORTED;
   DevCtx ctx;
   if (int e = ctx_or_error(&ctx)) return e;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const bool pack = ws && ws_bytes >= packed_kv_bytes(g);
-  if (pack)
-    if (int e = launch_pack_kv(g, K, V, ws, st)) return e;
-  return launch_sparse_attn(g, Q, K, V, idx, O, lse, 0, pack ? ws : nullptr, ctx, st);
+  return enqueue_sparse(g, Q, K, V, idx, O, lse, ws, ws_bytes, false, ctx,
+                        static_cast<cudaStream_t>(stream));
+}
+
+int infllmv2_sparse_attn_per_token(const infllmv2_params* p, const void* Q, const void* K,
+                                   const void* V, const int32_t* idx, void* O, float* lse,
+                                   void* ws, size_t ws_bytes, void* stream) {
+  Geometry g;
+  if (int e = validate(p, true, &g)) return e;
+  if (empty(g)) return INFLLMV2_OK;
+  if (int e = check_ptrs({Q, K, V, idx, O, lse})) return e;
+  if (ws && !aligned16(ws)) return INFLLMV2_ERR_UNSUPPORTED;
+  DevCtx ctx;
+  if (int e = ctx_or_error(&ctx)) return e;
+  return enqueue_sparse(g, Q, K, V, idx, O, lse, ws, ws_bytes, true, ctx,
+                        static_cast<cudaStream_t>(stream));
 }
 
 int infllmv2_dense_attn(const infllmv2_params* p, const void* Q, const void* K, const void* V,
                         void* O, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
   Geometry g;
   if (int e = validate(p, false, &g)) return e;
   if (empty(g)) return INFLLMV2_OK;
   if (int e = check_ptrs({Q, K, V, O, lse})) return e;
-  if (ws && !aligned16(ws)) return INFLLMV2_ERR_UNSUPPORTED;
   DevCtx ctx;
   if (int e = ctx_or_error(&ctx)) return e;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const bool pack = ws && ws_bytes >= packed_kv_bytes(g);
-  if (pack)
-    if (int e = launch_pack_kv(g, K, V, ws, st)) return e;
-  return launch_sparse_attn(g, Q, K, V, nullptr, O, lse, 1, pack ? ws : nullptr, ctx, st);
+  return launch_dense_tile(g, Q, K, V, O, lse, ctx, static_cast<cudaStream_t>(stream));
+}
+
+int infllmv2_compressed_attn(const infllmv2_params* p, const void* Q, const void* Kc,
+                             const void* Vc, void* O, float* lse, void* stream) {
+  Geometry g;
+  if (int e = validate(p, false, &g)) return e;
+  if (empty(g)) return INFLLMV2_OK;
+  if (int e = check_ptrs({Q, O, lse})) return e;
+  if (g.n_c > 0)
+    if (int e = check_ptrs({Kc, Vc})) return e;
+  DevCtx ctx;
+  if (int e = ctx_or_error(&ctx)) return e;
+  return launch_compressed_tile(g, Q, Kc, Vc, O, lse, ctx, static_cast<cudaStream_t>(stream));
 }
 
 int infllmv2_forward(const infllmv2_params* p, const void* Q, const void* K, const void* V,
@@ -266,7 +308,7 @@ int infllmv2_forward(const infllmv2_params* p, const void* Q, const void* K, con
   if (int e = validate(p, true, &g)) return e;
   if (int e = check_select_size(g)) return e;
   if (empty(g)) return INFLLMV2_OK;
-  // workspace: block scores of the selection, then the packed K/V tiles
+  // workspace: block scores of the selection, then the attention's
   const size_t sel = align256(select_ws_bytes(g));
   if (ws_bytes < sel) return INFLLMV2_ERR_WORKSPACE;
   if (g.n_c > 0)
@@ -280,8 +322,8 @@ size_t infllmv2_prefill_chunk_workspace_bytes(const infllmv2_params* p, int32_t 
                                               int32_t q_len) {
   Geometry g;
   if (validate_chunk(p, q_offset, q_len, &g) != INFLLMV2_OK) return SIZE_MAX;
-  if (p->T <= p->switch_threshold) return packed_kv_bytes(g);
-  return check_select_size(g) ? SIZE_MAX : align256(select_ws_bytes(g)) + packed_kv_bytes(g);
+  if (p->T <= p->switch_threshold) return 0;
+  return check_select_size(g) ? SIZE_MAX : align256(select_ws_bytes(g)) + attn_ws_bytes(g);
 }
 
 int infllmv2_prefill_chunk(const infllmv2_params* p, int32_t q_offset, int32_t q_len,
@@ -306,16 +348,11 @@ int infllmv2_prefill_chunk(const infllmv2_params* p, int32_t q_offset, int32_t q
   DevCtx ctx;
   if (int e = ctx_or_error(&ctx)) return e;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (!dense) {
-    if (int e = launch_score_blocks(g, Q, Kc, static_cast<float*>(ws), ctx, st)) return e;
-    if (int e = launch_topk(g, static_cast<float*>(ws), idx, st)) return e;
-  }
-  uint8_t* rest = ws ? static_cast<uint8_t*>(ws) + sel : nullptr;
-  const bool pack = rest && ws_bytes - sel >= packed_kv_bytes(g);
-  if (pack)
-    if (int e = launch_pack_kv(g, K, V, rest, st)) return e;
-  return launch_sparse_attn(g, Q, K, V, dense ? nullptr : idx, O, lse, dense ? 1 : 0,
-                            pack ? rest : nullptr, ctx, st);
+  if (dense) return launch_dense_tile(g, Q, K, V, O, lse, ctx, st);
+  if (int e = launch_score_blocks(g, Q, Kc, static_cast<float*>(ws), ctx, st)) return e;
+  if (int e = launch_topk(g, static_cast<float*>(ws), idx, st)) return e;
+  return enqueue_sparse(g, Q, K, V, idx, O, lse, static_cast<uint8_t*>(ws) + sel, ws_bytes - sel,
+                        false, ctx, st);
 }
 
 int infllmv2_decode_step(const infllmv2_params* p, const void* q, const void* k_new,

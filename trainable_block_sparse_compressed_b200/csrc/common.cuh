@@ -125,11 +125,22 @@ int launch_topk(const Geometry& g, const float* scores, int32_t* idx, cudaStream
 size_t packed_kv_bytes(const Geometry& g);
 int launch_pack_kv(const Geometry& g, const void* K, const void* V, void* packed,
                    cudaStream_t st);
-// Sparse attention over selected blocks; dense == 1 attends to every block <= t/64.
+// Sparse attention over selected blocks, one work item per query token.
 // packed: K/V tiles from launch_pack_kv, or null to gather from K and V.
 int launch_sparse_attn(const Geometry& g, const void* Q, const void* K, const void* V,
-                       const int32_t* idx, void* O, float* lse, int dense, const void* packed,
+                       const int32_t* idx, void* O, float* lse, const void* packed,
                        const DevCtx& ctx, cudaStream_t st);
+// Query-tile attention (tile_attn.cu): dense causal, the union of the tile's
+// selected blocks, or the compressed windows.
+bool union_supported(const Geometry& g);
+size_t union_ws_bytes(const Geometry& g);
+int launch_dense_tile(const Geometry& g, const void* Q, const void* K, const void* V, void* O,
+                      float* lse, const DevCtx& ctx, cudaStream_t st);
+int launch_union_tile(const Geometry& g, const void* Q, const void* K, const void* V,
+                      const int32_t* idx, void* O, float* lse, void* ws, const DevCtx& ctx,
+                      cudaStream_t st);
+int launch_compressed_tile(const Geometry& g, const void* Q, const void* Kc, const void* Vc,
+                           void* O, float* lse, const DevCtx& ctx, cudaStream_t st);
 // Decode (decode.cu); g.T is the cache capacity.
 size_t decode_ws_bytes(const Geometry& g);
 int launch_decode_step(const Geometry& g, const void* q, const void* k_new, const void* v_new,

@@ -1,8 +1,8 @@
 // sparse_attn.cu -- block-sparse causal attention over selected key blocks
 // (reportify digest, Technical Mechanism: after block selection, attention is
-// computed only over the selected key/value subsets), and the dense causal
-// path (every block <= t/64; InfLLM-V2 skill write-up, Architecture
-// Overview, dense pathway bullet).
+// computed only over the selected key/value subsets), one work item per query
+// token: the per-token schedule of the prefill, and the decode step's
+// attention.
 //
 // Work item = one query token t of one (batch, kv head): its G query heads
 // share the item's selected blocks.  On i.i.d. data neighbouring tokens share
@@ -92,21 +92,21 @@ struct AttnArgs {
   const uint8_t* Kp;        // packed K / V tiles (pack.cu), or null: tensor-map gather
   const uint8_t* Vp;
   int nb;                   // blocks per (batch, kv head) of the packed tiles
-  const int32_t* idx;       // selected blocks (null when dense)
-  __nv_bfloat16* O;         // final output (prefill / dense)
+  const int32_t* idx;       // selected blocks
+  __nv_bfloat16* O;         // final output (prefill)
   float* lse;
   float* part;              // decode partials: [items][G][128] o, then [items][G][2] (m, l)
   const int32_t* seqlens;   // decode: query position of each sequence
   int B, T, Hq, Hkv, topk;  // T: key tokens (prefill) or cache capacity (decode)
   int q0, Tq;               // prefill: the queries are tokens q0 .. q0+Tq-1
-  int mode;                 // 0 sparse prefill, 1 dense prefill, 2 decode
+  int mode;                 // 0 sparse prefill, 2 decode
   int n_chunks, chunk_blocks;
   float scale_log2;
 };
 
 struct Item {
   int b, g, t, qtok, cur, e0, n, n_pairs;
-  const int32_t* row;  // index row (null when dense)
+  const int32_t* row;  // index row
 };
 
 // Length of the prefix of entries in [0, cur] (warp-collective).
@@ -149,13 +149,8 @@ __device__ __forceinline__ Item resolve_item(int64_t it, const AttnArgs& a, int 
     r.t = a.q0 + r.qtok;                    // its token position
     r.cur = r.t / kBlock;
     r.e0 = 0;
-    if (a.mode == 1) {
-      r.row = nullptr;
-      r.n = r.cur + 1;
-    } else {
-      r.row = a.idx + ((static_cast<int64_t>(r.b) * a.Hkv + r.g) * a.Tq + r.qtok) * a.topk;
-      r.n = count_valid(r.row, a.topk, r.cur, lane);
-    }
+    r.row = a.idx + ((static_cast<int64_t>(r.b) * a.Hkv + r.g) * a.Tq + r.qtok) * a.topk;
+    r.n = count_valid(r.row, a.topk, r.cur, lane);
   }
   r.n_pairs = (r.n + 1) >> 1;
   return r;
@@ -179,7 +174,7 @@ __device__ __forceinline__ int64_t item_of(int64_t k, int64_t n_items) {
 
 // Block of entry e (0 <= e < n) of an item, from global memory.
 __device__ __forceinline__ int item_block(const Item& it, int e) {
-  return it.row ? __ldg(it.row + it.e0 + e) : it.e0 + e;
+  return __ldg(it.row + it.e0 + e);
 }
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, const DevCtx& ctx,
@@ -453,9 +448,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int64_t k = 0, it; ok && (it = item_of(k, n_items)) < n_items; ++k) {
       const Item item = resolve_item(it, args, lane);
       // the item's blocks, staged once in shared memory by all 256 threads
-      if (item.row)
-        for (int e = gt; e < item.n; e += kSoftmaxThreads)
-          sm.blocks[e] = __ldg(item.row + item.e0 + e);
+      for (int e = gt; e < item.n; e += kSoftmaxThreads)
+        sm.blocks[e] = __ldg(item.row + item.e0 + e);
       named_bar_sync(bar_sync_id, kSoftmaxThreads);
       float m[kHH], l[kHH], o[kHH], alpha_prev[kHH];
 #pragma unroll
@@ -480,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_wait();
           tc_fence_before();
           const int e = 2 * p + slot;
-          const int blk = e < item.n ? (item.row ? sm.blocks[e] : item.e0 + e) : -1;
+          const int blk = e < item.n ? sm.blocks[e] : -1;
           const bool valid = blk >= 0 && blk * kBlock + krow <= item.t;
           float s[kHH];
           bool exceed = false;
@@ -672,7 +666,7 @@ int launch_attn(const Geometry& g, const void* Q, int q_tokens, const void* K, c
 }  // namespace
 
 int launch_sparse_attn(const Geometry& g, const void* Q, const void* K, const void* V,
-                       const int32_t* idx, void* O, float* lse, int dense, const void* packed,
+                       const int32_t* idx, void* O, float* lse, const void* packed,
                        const DevCtx& ctx, cudaStream_t st) {
   if (g.B == 0 || g.Tq == 0) return INFLLMV2_OK;
   AttnArgs a{};
@@ -691,7 +685,7 @@ int launch_sparse_attn(const Geometry& g, const void* Q, const void* K, const vo
   a.topk = g.topk;
   a.q0 = g.q0;
   a.Tq = g.Tq;
-  a.mode = dense ? 1 : 0;
+  a.mode = 0;
   a.scale_log2 = g.scale_log2;
   const int64_t n_items = static_cast<int64_t>(g.B) * g.Hkv * g.Tq;
   return launch_attn(g, Q, g.Tq, K, V, g.T, a, n_items, ctx, st);

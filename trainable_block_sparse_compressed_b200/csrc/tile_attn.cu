@@ -1,0 +1,718 @@
+// tile_attn.cu -- causal softmax attention over query tiles.
+//
+// A query tile is 128 rows: the 128/G consecutive tokens x the G query heads
+// of one GQA group, the rows that one TMA box of the BSHD query tensor holds.
+// Every row of the tile runs over the same stream of key tiles, so each key
+// tile is loaded once for 128 rows and both products are full tensor-core
+// tiles (tcgen05.mma, M = 128):
+//
+//   S[128 rows x KT keys] = Q (K-major, 128-byte swizzle) x K_tile^T
+//   O[128 rows x 128 d ] += P (K-major, no swizzle)      x V_tile (MN-major)
+//
+// with S double-buffered and O accumulated in tensor memory.  Three key
+// streams share the kernel:
+//
+//   dense      every key 0 .. t: exact dense causal attention (InfLLM-V2 skill
+//              write-up, Architecture Overview, the dense pathway bullet);
+//              key tiles of 128 keys, the blocks past the tile's last token
+//              are not loaded.
+//   union      the union of the 64-key blocks the tile's tokens selected, two
+//              blocks per key tile, each row masked to its own token's
+//              blocks (block-sparse attention over the selected blocks:
+//              reportify digest, Technical Mechanism).  A block that several
+//              tokens of the tile selected is loaded and multiplied once.
+//   compressed the window means Kc, Vc (skill write-up, Core Concept: the
+//              compressed pattern aggregates tokens hierarchically); window
+//              j is visible to token t iff 16 j + 31 <= t.  Key tiles of 64
+//              windows; q . Kc takes both bf16 planes of the compressed key
+//              (K = 2 x 128), Vc its high plane.
+//
+// Warp roles: warp 0 loads Q (double-buffered) and the key tiles (K and V of
+// a tile in one ring stage) by TMA; warp 1 owns tensor memory and one thread
+// issues the MMAs; warps 2-5 are the softmax, one thread per query row (TMEM
+// lane), so a row's maximum and sum need no cross-thread reduction.  Each row
+// keeps a reference maximum m that moves only when a score exceeds it by more
+// than 8 (log2 units), so P = exp2(s - m) <= 256 is exact enough in bf16 and
+// the O accumulator is rescaled in tensor memory only on those (rare) moves.
+// Persistent CTAs, one per SM, take the query tiles heaviest first.
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace infllmv2 {
+
+constexpr int kTileDense = 0, kTileUnion = 1, kTileCompressed = 2;
+
+// Union lists (tile_attn.cu and its builder): entry = block | token mask << 16.
+struct TileArgs {
+  __nv_bfloat16* O;         // [B, Tq, Hq, 128]
+  float* lse;               // [B, Hq, Tq]
+  const uint32_t* ulist;    // union: per query tile, its blocks ascending
+  const int32_t* ucount;    // union: entries per query tile
+  int ustride;              // union: list capacity per query tile
+  int B, Hq, Hkv, q0, Tq;   // queries are tokens q0 .. q0+Tq-1
+  int n_c;                  // compressed: windows in Kc / Vc
+  float scale_log2;
+};
+
+namespace {
+
+template <int MODE>
+struct TileCfg {
+  static constexpr int KT = MODE == kTileCompressed ? 64 : 128;  // keys per tile
+  static constexpr int KP = MODE == kTileCompressed ? 2 : 1;     // bf16 planes of K
+  static constexpr int kStages = MODE == kTileCompressed ? 3 : 2;
+  static constexpr int kBox = 64 * 128;                          // 64 rows x 64 channels
+  static constexpr int kKBytes = KP * KT * 256;
+  static constexpr int kVBytes = KT * 256;
+  static constexpr int kStageBytes = kKBytes + kVBytes;
+  static constexpr int kQBytes = 128 * 256;
+  static constexpr int kPBytes = 128 * KT * 2;
+  static constexpr uint32_t kOCol = 2 * KT;                      // S0, S1, then O
+  static constexpr uint32_t kTmemCols = MODE == kTileCompressed ? 256 : 512;
+  static constexpr int kThreads = 64 + 128;
+};
+
+struct TileSmem {
+  uint64_t q_full[2], q_empty[2];
+  uint64_t kv_full[3], kv_empty[3];
+  uint64_t s_full[2];
+  uint64_t p_full, pv_done, o_free, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+constexpr float kTileSlack = 8.0f;   // log2 units
+constexpr float kLn2f = 0.6931471805599453f;
+
+struct TileItem {
+  int b, g, qt, qtok0, t_last, n_kt, n_u;
+  int64_t list;  // union: index of the tile's list
+};
+
+template <int G, int MODE>
+__device__ __forceinline__ TileItem tile_item(int64_t k, const TileArgs& a, int n_qt) {
+  constexpr int TPT = 128 / G;
+  using C = TileCfg<MODE>;
+  TileItem r;
+  const int bgn = a.B * a.Hkv;
+  r.qt = n_qt - 1 - static_cast<int>(k / bgn);  // heaviest (latest) tiles first
+  const int bg = static_cast<int>(k % bgn);
+  r.b = bg / a.Hkv;
+  r.g = bg % a.Hkv;
+  r.qtok0 = r.qt * TPT;
+  r.t_last = a.q0 + min(r.qtok0 + TPT, a.Tq) - 1;
+  r.list = static_cast<int64_t>(bg) * n_qt + r.qt;
+  r.n_u = 0;
+  if (MODE == kTileDense) {
+    r.n_kt = r.t_last / C::KT + 1;
+  } else if (MODE == kTileUnion) {
+    r.n_u = a.ucount[r.list];
+    r.n_kt = (r.n_u + 1) >> 1;
+  } else {
+    const int v = min(a.n_c, visible_windows(r.t_last));
+    r.n_kt = (v + C::KT - 1) / C::KT;
+  }
+  return r;
+}
+
+__device__ __forceinline__ bool tile_wait(uint64_t* bar, uint32_t parity, const DevCtx& ctx,
+                                          volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  if (*abort_flag) return false;
+  if (mbar_wait(bar, parity, ctx.wait_ns)) return true;
+  report_status(ctx.status, INFLLMV2_STATUS_TIMEOUT);
+  *abort_flag = 1;
+  return false;
+}
+
+template <int G, int MODE>
+__global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
+    tile_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
+                     const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const TileArgs args, DevCtx ctx) {
+  using C = TileCfg<MODE>;
+  constexpr int TPT = 128 / G;
+  constexpr int KT = C::KT;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* sQ = base;                                   // 2 x 32 KB
+  uint8_t* sKV = sQ + 2 * C::kQBytes;                   // stages: K planes, then V
+  uint8_t* sP = sKV + C::kStages * C::kStageBytes;      // P, 128 rows x KT keys
+  TileSmem& sm = *reinterpret_cast<TileSmem*>(sP + C::kPBytes);
+
+  const int warp = warp_id(), lane = lane_id();
+  const int n_qt = (args.Tq + TPT - 1) / TPT;
+  const int64_t n_items = static_cast<int64_t>(args.B) * args.Hkv * n_qt;
+
+  // A key tile may fill only its first block (dense past the last token,
+  // union with an odd count): the stale rows of the other block are masked
+  // in S, and their V rows meet P = 0, so V must hold finite values: zero
+  // every stage's V area once.
+  for (int i = threadIdx.x; i < C::kStages * C::kVBytes / 16; i += blockDim.x) {
+    const int st = i / (C::kVBytes / 16), k = i % (C::kVBytes / 16);
+    reinterpret_cast<uint4*>(sKV + st * C::kStageBytes + C::kKBytes)[k] = make_uint4(0, 0, 0, 0);
+  }
+  fence_proxy_async_smem();
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.q_full[i], 1);
+      mbar_init(&sm.q_empty[i], 1);
+      mbar_init(&sm.s_full[i], 1);
+    }
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&sm.kv_full[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
+    }
+    mbar_init(&sm.p_full, 4);   // one arrival per softmax warp
+    mbar_init(&sm.pv_done, 1);
+    mbar_init(&sm.o_free, 4);
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort_flag = &sm.abort_flag;
+
+  if (warp == 0) {
+    // ------------------------------ producer ------------------------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      int qk = 0;
+      int64_t gt = 0;
+      bool ok = true;
+      for (int64_t k = blockIdx.x; ok && k < n_items; k += gridDim.x) {
+        const TileItem it = tile_item<G, MODE>(k, args, n_qt);
+        if (it.n_kt == 0) continue;
+        const int qb = qk & 1;
+        if (qk >= 2 && !(ok = tile_wait(&sm.q_empty[qb], ((qk >> 1) & 1) ^ 1, ctx, abort_flag)))
+          break;
+        mbar_arrive_expect_tx(&sm.q_full[qb], C::kQBytes);
+        uint8_t* q = sQ + qb * C::kQBytes;
+        tma_load_4d(q, &tmQ, &sm.q_full[qb], 0, it.g * G, it.qtok0, it.b);
+        tma_load_4d(q + C::kQBytes / 2, &tmQ, &sm.q_full[qb], 64, it.g * G, it.qtok0, it.b);
+        ++qk;
+        for (int i = 0; i < it.n_kt; ++i, ++gt) {
+          const int s = static_cast<int>(gt % C::kStages);
+          if (gt >= C::kStages &&
+              !(ok = tile_wait(&sm.kv_empty[s], ((gt / C::kStages) & 1) ^ 1, ctx, abort_flag)))
+            break;
+          uint8_t* stK = sKV + s * C::kStageBytes;
+          uint8_t* stV = stK + C::kKBytes;
+          uint64_t* full = &sm.kv_full[s];
+          if (MODE == kTileCompressed) {
+            // 64 windows: K hi / lo planes x 2 channel halves, V hi x 2 halves
+            mbar_arrive_expect_tx(full, C::kStageBytes);
+            const int j0 = i * KT;
+            for (int x = 0; x < 4; ++x)
+              tma_load_4d(stK + x * C::kBox, &tmK, full, 64 * x, it.g, j0, it.b);
+            for (int x = 0; x < 2; ++x)
+              tma_load_4d(stV + x * C::kBox, &tmV, full, 64 * x, it.g, j0, it.b);
+          } else {
+            int blk[2];
+            int nblk;
+            if (MODE == kTileDense) {
+              blk[0] = 2 * i;
+              blk[1] = 2 * i + 1;
+              nblk = blk[1] * kBlock <= it.t_last ? 2 : 1;
+            } else {
+              const uint32_t* L = args.ulist + it.list * args.ustride;
+              blk[0] = static_cast<int>(__ldg(L + 2 * i) & 0xFFFFu);
+              nblk = 2 * i + 1 < it.n_u ? 2 : 1;
+              blk[1] = nblk == 2 ? static_cast<int>(__ldg(L + 2 * i + 1) & 0xFFFFu) : 0;
+            }
+            mbar_arrive_expect_tx(full, nblk * 4 * C::kBox);
+            for (int e = 0; e < nblk; ++e) {
+              // half h of block e at h * (KT rows) + e * 64 rows
+              for (int h = 0; h < 2; ++h) {
+                tma_load_4d(stK + h * KT * 128 + e * C::kBox, &tmK, full, 64 * h, it.g,
+                            blk[e] * kBlock, it.b);
+                tma_load_4d(stV + h * KT * 128 + e * C::kBox, &tmV, full, 64 * h, it.g,
+                            blk[e] * kBlock, it.b);
+              }
+            }
+          }
+        }
+      }
+      // drain: never leave with copies of this CTA in flight
+      for (int x = 0; x < 2 && x < qk; ++x)
+        mbar_wait(&sm.q_full[(qk - 1 - x) & 1], ((qk - 1 - x) >> 1) & 1, ctx.wait_ns);
+      for (int64_t q = gt - 1; q >= 0 && q >= gt - C::kStages; --q)
+        mbar_wait(&sm.kv_full[q % C::kStages], (q / C::kStages) & 1, ctx.wait_ns);
+    }
+  } else if (warp == 1) {
+    // ----------------------------- MMA issuer -----------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = instr_desc_bf16(128, KT, 0, 0);
+      constexpr uint32_t idesc_pv = instr_desc_bf16(128, 128, 0, 1);
+      const uint32_t p_addr = smem_u32(sP);
+      int qk = 0, ik = 0;
+      int64_t gt = 0;
+      bool ok = true;
+      // P V of tile q (its P written by the softmax); `first` starts the
+      // item's O accumulator, after the previous item's epilogue read O out
+      auto issue_pv = [&](int64_t q, bool first) -> bool {
+        if (!tile_wait(&sm.p_full, static_cast<uint32_t>(q & 1), ctx, abort_flag)) return false;
+        if (first && ik > 0 && !tile_wait(&sm.o_free, (ik - 1) & 1, ctx, abort_flag)) return false;
+        tc_fence_after();
+        const int s = static_cast<int>(q % C::kStages);
+        const uint32_t v_addr = smem_u32(sKV + s * C::kStageBytes + C::kKBytes);
+#pragma unroll
+        for (int kk = 0; kk < KT / 16; ++kk) {
+          // A = P: K-major, no swizzle: 8-key core-matrix columns 2 KB apart
+          // (LBO), 8-row groups 128 B apart (SBO).  B = V: MN-major, 128-byte
+          // swizzle: 16 keys = 2 KB, the two 64-channel halves KT rows apart.
+          const uint64_t ad = smem_desc(p_addr + kk * 4096, 2048, 128, 0);
+          const uint64_t bd = smem_desc(v_addr + kk * 2048, KT * 128, 1024, 2);
+          umma_bf16(tmem + C::kOCol, ad, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
+        }
+        umma_commit(&sm.kv_empty[s]);
+        umma_commit(&sm.pv_done);
+        return true;
+      };
+      for (int64_t k = blockIdx.x; ok && k < n_items; k += gridDim.x) {
+        const TileItem it = tile_item<G, MODE>(k, args, n_qt);
+        if (it.n_kt == 0) continue;
+        const int qb = qk & 1;
+        if (!(ok = tile_wait(&sm.q_full[qb], (qk >> 1) & 1, ctx, abort_flag))) break;
+        const uint32_t q_addr = smem_u32(sQ + qb * C::kQBytes);
+        for (int i = 0; ok && i < it.n_kt; ++i, ++gt) {
+          const int s = static_cast<int>(gt % C::kStages);
+          if (!(ok = tile_wait(&sm.kv_full[s], (gt / C::kStages) & 1, ctx, abort_flag))) break;
+          tc_fence_after();
+          // S(gt) overwrites the buffer of S(gt-2), read by the softmax
+          // before it wrote P(gt-2), which P V(gt-2) waited for
+          const uint32_t k_addr = smem_u32(sKV + s * C::kStageBytes);
+#pragma unroll
+          for (int kk = 0; kk < 8 * C::KP; ++kk) {
+            // K-major, 128-byte swizzle: 16 channels = 32 B inside a
+            // 64-channel half; plane p, half h at (2p + h) * KT rows
+            const uint32_t off = ((kk >> 2) & 1) * (KT * 128) + (kk & 3) * 32;
+            const uint64_t qd = smem_desc(q_addr + ((kk >> 2) & 1) * (C::kQBytes / 2) + (kk & 3) * 32,
+                                          16, 1024, 2);
+            const uint64_t kd = smem_desc(k_addr + (kk >> 3) * (2 * KT * 128) + off, 16, 1024, 2);
+            umma_bf16(tmem + static_cast<uint32_t>(gt & 1) * KT, qd, kd, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&sm.s_full[gt & 1]);
+          if (i == it.n_kt - 1) umma_commit(&sm.q_empty[qb]);
+          if (i > 0) ok = issue_pv(gt - 1, i == 1);
+        }
+        if (ok) ok = issue_pv(gt - 1, it.n_kt == 1);
+        ++qk;
+        ++ik;
+      }
+      // drain: every MMA of this CTA completes before TMEM is released
+      umma_commit(&sm.drain);
+      mbar_wait(&sm.drain, 0, ctx.wait_ns);
+    }
+  } else {
+    // ------------------------------ softmax ------------------------------
+    const int quad = warp & 3;          // TMEM lane quadrant of this warp
+    const int r = quad * 32 + lane;     // query row of the tile
+    const int tok = r / G, h = r % G;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const float sl2 = args.scale_log2;
+    // P: K-major no-swizzle image, row r's 8-key chunk c at c*2048 + (r/8)*128 + (r%8)*16
+    uint8_t* p_row = sP + (r >> 3) * 128 + (r & 7) * 16;
+    int64_t gt = 0;
+    bool ok = true;
+    for (int64_t k = blockIdx.x; ok && k < n_items; k += gridDim.x) {
+      const TileItem it = tile_item<G, MODE>(k, args, n_qt);
+      const int qtok = it.qtok0 + tok;
+      const bool row_ok = qtok < args.Tq;
+      const int t = args.q0 + qtok;
+      const int64_t orow = (static_cast<int64_t>(it.b) * args.Tq + qtok) * args.Hq + it.g * G + h;
+      const int64_t lrow = (static_cast<int64_t>(it.b) * args.Hq + it.g * G + h) * args.Tq + qtok;
+      if (it.n_kt == 0) {
+        // no visible key for any row of the tile (compressed, t < 31)
+        if (row_ok) {
+          uint4* o = reinterpret_cast<uint4*>(args.O + orow * kHeadDim);
+          for (int c = 0; c < 16; ++c) o[c] = make_uint4(0, 0, 0, 0);
+          args.lse[lrow] = -INFINITY;
+        }
+        continue;
+      }
+      const int v_row = MODE == kTileCompressed ? min(args.n_c, visible_windows(t)) : 0;
+      float m = -INFINITY, l = 0.f;
+      for (int i = 0; i < it.n_kt; ++i, ++gt) {
+        ok = __all_sync(0xffffffffu, tile_wait(&sm.s_full[gt & 1], (gt >> 1) & 1, ctx, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        float x[KT];
+#pragma unroll
+        for (int c = 0; c < KT / 32; ++c)
+          tmem_ld32(lane_addr + static_cast<uint32_t>(gt & 1) * KT + 32 * c,
+                    *reinterpret_cast<float(*)[32]>(x + 32 * c));
+        tmem_ld_wait();
+        // the row's keys in this tile, masked and scaled to log2 units
+        uint32_t sel[2] = {1u, 1u};
+        int kbase[2] = {i * KT, i * KT + 64};
+        if (MODE == kTileUnion) {
+          const uint32_t* L = args.ulist + it.list * args.ustride;
+          const uint32_t e0 = __ldg(L + 2 * i);
+          const uint32_t e1 = 2 * i + 1 < it.n_u ? __ldg(L + 2 * i + 1) : 0u;
+          sel[0] = (e0 >> (16 + tok)) & 1u;
+          sel[1] = (e1 >> (16 + tok)) & 1u;
+          kbase[0] = static_cast<int>(e0 & 0xFFFFu) * kBlock;
+          kbase[1] = static_cast<int>(e1 & 0xFFFFu) * kBlock;
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < KT; ++c) {
+          bool valid;
+          if (MODE == kTileCompressed) {
+            valid = i * KT + c < v_row;
+          } else {
+            const int e = c >> 6;
+            valid = sel[e] != 0u && kbase[e] + (c & 63) <= t;
+          }
+          valid = valid && row_ok;
+          x[c] = valid ? x[c] * sl2 : -INFINITY;
+          mx = fmaxf(mx, x[c]);
+        }
+        float alpha = 1.f;
+        if (mx > m + kTileSlack) {
+          alpha = fast_exp2(m - mx);  // 0 while the row had no key
+          m = mx;
+        }
+        float psum = 0.f;
+        uint32_t pk[KT / 2];
+#pragma unroll
+        for (int c = 0; c < KT; c += 2) {
+          const float p0 = fast_exp2(x[c] - m);       // exp2(-inf) = 0 for masked keys
+          const float p1 = fast_exp2(x[c + 1] - m);
+          psum += p0 + p1;
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+          pk[c >> 1] = *reinterpret_cast<uint32_t*>(&b2);
+        }
+        if (m == -INFINITY) {  // no key of the row so far: nothing to add
+          psum = 0.f;
+#pragma unroll
+          for (int c = 0; c < KT / 2; ++c) pk[c] = 0u;
+        }
+        l = l * alpha + psum;
+        // P and O are free once P V of the previous tile has completed
+        if (i > 0) {
+          ok = __all_sync(0xffffffffu,
+                          tile_wait(&sm.pv_done, static_cast<uint32_t>((gt - 1) & 1), ctx, abort_flag));
+          if (!ok) break;
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, alpha != 1.f)) {
+            // move this row's accumulator to the new reference maximum
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              float o[32];
+              tmem_ld32(lane_addr + C::kOCol + 32 * c, o);
+              tmem_ld_wait();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) o[j] *= alpha;
+              tmem_st32(lane_addr + C::kOCol + 32 * c, o);
+            }
+            tmem_st_wait();
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < KT / 8; ++c)
+          *reinterpret_cast<uint4*>(p_row + c * 2048) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.p_full);
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l and the row's log-sum-exp ----
+      ok = __all_sync(0xffffffffu,
+                      tile_wait(&sm.pv_done, static_cast<uint32_t>((gt - 1) & 1), ctx, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float o[32];
+        tmem_ld32(lane_addr + C::kOCol + 32 * c, o);
+        tmem_ld_wait();
+        if (row_ok && INFLLMV2_CHECK(ctx.status, it.b < args.B && it.g < args.Hkv)) {
+          uint4* dst = reinterpret_cast<uint4*>(args.O + orow * kHeadDim + 32 * c);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(o[8 * j + 2 * e] * inv,
+                                                        o[8 * j + 2 * e + 1] * inv);
+              w[e] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+            dst[j] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+      if (row_ok) args.lse[lrow] = l > 0.f ? (m + __log2f(l)) * kLn2f : -INFINITY;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.o_free);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// union lists: for every query tile (b, g, qt), the blocks its TPT tokens
+// selected, ascending, each with the mask of the tokens that selected it.
+// One CTA per tile: the (block, token) keys of the tile's index rows are
+// sorted (bitonic, in shared memory), equal blocks merged.
+// ---------------------------------------------------------------------------
+constexpr int kUnionThreads = 256;
+
+template <int TPT>
+__global__ void __launch_bounds__(kUnionThreads) union_build_kernel(
+    const int32_t* __restrict__ idx, uint32_t* __restrict__ ulist, int32_t* __restrict__ ucount,
+    int Hkv, int q0, int Tq, int topk, int n_qt, int cap) {
+  extern __shared__ uint32_t keys[];  // cap entries (a power of two)
+  __shared__ int scan[kUnionThreads / 32 + 1];
+  const int64_t tile = blockIdx.x;
+  const int64_t bg = tile / n_qt;
+  const int qt = static_cast<int>(tile % n_qt);
+  const int n = TPT * topk;
+  for (int e = threadIdx.x; e < cap; e += blockDim.x) {
+    uint32_t key = 0xFFFFFFFFu;
+    if (e < n) {
+      const int tk = e / topk, j = e % topk;
+      const int qtok = qt * TPT + tk;
+      if (qtok < Tq) {
+        const int v = __ldg(idx + ((bg * Tq + qtok) * topk + j));
+        const int t = q0 + qtok;
+        if (v >= 0 && v <= t / kBlock) key = (static_cast<uint32_t>(v) << 4) | static_cast<uint32_t>(tk);
+      }
+    }
+    keys[e] = key;
+  }
+  __syncthreads();
+  for (int size = 2; size <= cap; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < cap / 2; i += blockDim.x) {
+        const int lo = 2 * i - (i & (stride - 1));
+        const int hi = lo + stride;
+        const bool up = (lo & size) == 0;
+        const uint32_t a = keys[lo], b = keys[hi];
+        if ((a > b) == up) {
+          keys[lo] = b;
+          keys[hi] = a;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // merge equal blocks: the first key of each block emits (block, token mask)
+  constexpr int PER = 16;  // keys per thread (cap <= 4096)
+  const int base = threadIdx.x * PER;
+  uint32_t ent[PER];
+  int nh = 0;
+#pragma unroll
+  for (int s = 0; s < PER; ++s) {
+    const int p = base + s;
+    ent[s] = 0xFFFFFFFFu;
+    if (p < cap && keys[p] != 0xFFFFFFFFu && (p == 0 || (keys[p] >> 4) != (keys[p - 1] >> 4))) {
+      const uint32_t blk = keys[p] >> 4;
+      uint32_t mask = 0u;
+      for (int q = p; q < cap && (keys[q] >> 4) == blk && keys[q] != 0xFFFFFFFFu; ++q)
+        mask |= 1u << (keys[q] & 15u);
+      ent[s] = blk | (mask << 16);
+      ++nh;
+    }
+  }
+  // exclusive scan of the head counts over threads
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int x = nh;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) scan[wid] = x;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int w = 0; w < kUnionThreads / 32; ++w) {
+      const int v = scan[w];
+      scan[w] = acc;
+      acc += v;
+    }
+    scan[kUnionThreads / 32] = acc;
+  }
+  __syncthreads();
+  int pos = scan[wid] + x - nh;
+  uint32_t* L = ulist + tile * static_cast<int64_t>(n);
+#pragma unroll
+  for (int s = 0; s < PER; ++s)
+    if (ent[s] != 0xFFFFFFFFu) L[pos++] = ent[s];
+  if (threadIdx.x == 0) ucount[tile] = scan[kUnionThreads / 32];
+}
+
+int next_pow2(int x) {
+  int p = 1;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+template <int G, int MODE>
+int launch_tile_g(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                  const TileArgs& a, const DevCtx& ctx, cudaStream_t st) {
+  using C = TileCfg<MODE>;
+  constexpr int TPT = 128 / G;
+  const size_t smem = 1024 + 2 * C::kQBytes + C::kStages * C::kStageBytes + C::kPBytes +
+                      sizeof(TileSmem);
+  static std::atomic<uint64_t> smem_set{0};
+  if (int e = set_smem_limit(tile_attn_kernel<G, MODE>, smem, smem_set)) return e;
+  const int64_t n_items = static_cast<int64_t>(a.B) * a.Hkv * ((a.Tq + TPT - 1) / TPT);
+  const int64_t grid = n_items < sm_count() ? n_items : sm_count();
+  tile_attn_kernel<G, MODE><<<static_cast<unsigned>(grid), C::kThreads, smem, st>>>(tq, tk, tv, a,
+                                                                                  ctx);
+  return cudaGetLastError() == cudaSuccess ? INFLLMV2_OK : INFLLMV2_ERR_CUDA;
+}
+
+template <int MODE>
+int launch_tile(const Geometry& g, const CUtensorMap& tq, const CUtensorMap& tk,
+                const CUtensorMap& tv, const TileArgs& a, const DevCtx& ctx, cudaStream_t st) {
+  switch (g.G) {
+    case 8: return launch_tile_g<8, MODE>(tq, tk, tv, a, ctx, st);
+    case 16: return launch_tile_g<16, MODE>(tq, tk, tv, a, ctx, st);
+    default: break;
+  }
+  if constexpr (MODE != kTileUnion) {  // the union lists' token masks hold 16 tokens
+    switch (g.G) {
+      case 1: return launch_tile_g<1, MODE>(tq, tk, tv, a, ctx, st);
+      case 2: return launch_tile_g<2, MODE>(tq, tk, tv, a, ctx, st);
+      case 4: return launch_tile_g<4, MODE>(tq, tk, tv, a, ctx, st);
+      default: break;
+    }
+  }
+  return INFLLMV2_ERR_UNSUPPORTED;
+}
+
+// Q box: 64 channels x G heads x 128/G tokens.
+int q_map(const Geometry& g, const void* Q, CUtensorMap* tq) {
+  const uint64_t dims[4] = {static_cast<uint64_t>(kHeadDim), static_cast<uint64_t>(g.Hq),
+                            static_cast<uint64_t>(g.Tq), static_cast<uint64_t>(g.B)};
+  const uint64_t strides[3] = {static_cast<uint64_t>(kHeadDim) * 2,
+                               static_cast<uint64_t>(g.Hq) * kHeadDim * 2,
+                               static_cast<uint64_t>(g.Tq) * g.Hq * kHeadDim * 2};
+  const uint32_t box[4] = {64u, static_cast<uint32_t>(g.G), static_cast<uint32_t>(128 / g.G), 1u};
+  return make_tmap_bf16_4d(tq, Q, dims, strides, box);
+}
+
+// K / V box: 64 channels x 64 tokens of one kv head.
+int kv_map(const Geometry& g, const void* X, CUtensorMap* tm) {
+  const uint64_t dims[4] = {static_cast<uint64_t>(kHeadDim), static_cast<uint64_t>(g.Hkv),
+                            static_cast<uint64_t>(g.T), static_cast<uint64_t>(g.B)};
+  const uint64_t strides[3] = {static_cast<uint64_t>(kHeadDim) * 2,
+                               static_cast<uint64_t>(g.Hkv) * kHeadDim * 2,
+                               static_cast<uint64_t>(g.T) * g.Hkv * kHeadDim * 2};
+  const uint32_t box[4] = {64u, 1u, static_cast<uint32_t>(kBlock), 1u};
+  return make_tmap_bf16_4d(tm, X, dims, strides, box);
+}
+
+TileArgs tile_args(const Geometry& g, void* O, float* lse) {
+  TileArgs a{};
+  a.O = static_cast<__nv_bfloat16*>(O);
+  a.lse = lse;
+  a.B = g.B;
+  a.Hq = g.Hq;
+  a.Hkv = g.Hkv;
+  a.q0 = g.q0;
+  a.Tq = g.Tq;
+  a.n_c = g.n_c;
+  a.scale_log2 = g.scale_log2;
+  return a;
+}
+
+}  // namespace
+
+bool union_supported(const Geometry& g) { return g.G >= 8; }
+
+size_t union_ws_bytes(const Geometry& g) {
+  if (!union_supported(g) || g.B == 0 || g.Tq == 0) return 0;
+  const int TPT = 128 / g.G;
+  const int64_t tiles = static_cast<int64_t>(g.B) * g.Hkv * ((g.Tq + TPT - 1) / TPT);
+  const size_t lists = static_cast<size_t>(tiles) * TPT * g.topk * sizeof(uint32_t);
+  return ((lists + 255) & ~static_cast<size_t>(255)) + static_cast<size_t>(tiles) * sizeof(int32_t);
+}
+
+int launch_dense_tile(const Geometry& g, const void* Q, const void* K, const void* V, void* O,
+                      float* lse, const DevCtx& ctx, cudaStream_t st) {
+  if (g.B == 0 || g.Tq == 0) return INFLLMV2_OK;
+  CUtensorMap tq, tk, tv;
+  if (int e = q_map(g, Q, &tq)) return e;
+  if (int e = kv_map(g, K, &tk)) return e;
+  if (int e = kv_map(g, V, &tv)) return e;
+  return launch_tile<kTileDense>(g, tq, tk, tv, tile_args(g, O, lse), ctx, st);
+}
+
+int launch_union_tile(const Geometry& g, const void* Q, const void* K, const void* V,
+                      const int32_t* idx, void* O, float* lse, void* ws, const DevCtx& ctx,
+                      cudaStream_t st) {
+  if (g.B == 0 || g.Tq == 0) return INFLLMV2_OK;
+  if (!union_supported(g)) return INFLLMV2_ERR_UNSUPPORTED;
+  const int TPT = 128 / g.G;
+  const int n_qt = (g.Tq + TPT - 1) / TPT;
+  const int64_t tiles = static_cast<int64_t>(g.B) * g.Hkv * n_qt;
+  const int n = TPT * g.topk;
+  const int cap = next_pow2(n);
+  if (cap > 16 * kUnionThreads) return INFLLMV2_ERR_UNSUPPORTED;
+  uint32_t* ulist = static_cast<uint32_t*>(ws);
+  const size_t lists = static_cast<size_t>(tiles) * n * sizeof(uint32_t);
+  int32_t* ucount = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) +
+                                               ((lists + 255) & ~static_cast<size_t>(255)));
+  const size_t ush = static_cast<size_t>(cap) * sizeof(uint32_t);
+  if (TPT == 8)
+    union_build_kernel<8><<<static_cast<unsigned>(tiles), kUnionThreads, ush, st>>>(
+        idx, ulist, ucount, g.Hkv, g.q0, g.Tq, g.topk, n_qt, cap);
+  else
+    union_build_kernel<16><<<static_cast<unsigned>(tiles), kUnionThreads, ush, st>>>(
+        idx, ulist, ucount, g.Hkv, g.q0, g.Tq, g.topk, n_qt, cap);
+  if (cudaGetLastError() != cudaSuccess) return INFLLMV2_ERR_CUDA;
+  CUtensorMap tq, tk, tv;
+  if (int e = q_map(g, Q, &tq)) return e;
+  if (int e = kv_map(g, K, &tk)) return e;
+  if (int e = kv_map(g, V, &tv)) return e;
+  TileArgs a = tile_args(g, O, lse);
+  a.ulist = ulist;
+  a.ucount = ucount;
+  a.ustride = n;
+  return launch_tile<kTileUnion>(g, tq, tk, tv, a, ctx, st);
+}
+
+int launch_compressed_tile(const Geometry& g, const void* Q, const void* Kc, const void* Vc,
+                           void* O, float* lse, const DevCtx& ctx, cudaStream_t st) {
+  if (g.B == 0 || g.Tq == 0) return INFLLMV2_OK;
+  CUtensorMap tq, tk, tv;
+  if (int e = q_map(g, Q, &tq)) return e;
+  // compressed rows [B, n_c, Hkv, 2 planes x 128]; box 64 channels x 64 windows
+  const uint64_t rows = g.n_c > 0 ? static_cast<uint64_t>(g.n_c) : 1u;
+  const uint64_t dims[4] = {static_cast<uint64_t>(kKcRow), static_cast<uint64_t>(g.Hkv), rows,
+                            static_cast<uint64_t>(g.B)};
+  const uint64_t strides[3] = {static_cast<uint64_t>(kKcRow) * 2,
+                               static_cast<uint64_t>(g.Hkv) * kKcRow * 2,
+                               rows * g.Hkv * kKcRow * 2};
+  const uint32_t box[4] = {64u, 1u, 64u, 1u};
+  if (int e = make_tmap_bf16_4d(&tk, g.n_c > 0 ? Kc : Q, dims, strides, box)) return e;
+  if (int e = make_tmap_bf16_4d(&tv, g.n_c > 0 ? Vc : Q, dims, strides, box)) return e;
+  return launch_tile<kTileCompressed>(g, tq, tk, tv, tile_args(g, O, lse), ctx, st);
+}
+
+}  // namespace infllmv2

@@ -26,7 +26,7 @@ ERR_WORKSPACE = -5
 ERR_DEVICE_CHECK = -6
 STATUS_TIMEOUT = 0x1
 STATUS_SEQ_FULL = 0x2
-OP_SELECT, OP_FORWARD, OP_DECODE, OP_ATTN = 1, 2, 3, 4
+OP_SELECT, OP_FORWARD, OP_DECODE, OP_ATTN, OP_ATTN_PER_TOKEN = 1, 2, 3, 4, 5
 PATH_DENSE, PATH_SPARSE = 1, 2
 
 # every symbol include/infllmv2.h declares
@@ -37,6 +37,7 @@ EXPORTS = (
     "infllmv2_set_wait_limit", "infllmv2_selftest_timeout", "infllmv2_strerror",
     "infllmv2_version", "infllmv2_decode_step_noalloc", "infllmv2_prefill_chunk",
     "infllmv2_prefill_chunk_workspace_bytes", "infllmv2_gather_peak",
+    "infllmv2_sparse_attn_per_token", "infllmv2_compressed_attn",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -84,7 +85,9 @@ def load(path: Optional[str] = None):
         "infllmv2_compress_keys": (ctypes.c_int, [P, vp, vp, vp]),
         "infllmv2_select_blocks": (ctypes.c_int, [P, vp, vp, vp, vp, sz, vp]),
         "infllmv2_sparse_attn": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "infllmv2_sparse_attn_per_token": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "infllmv2_dense_attn": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "infllmv2_compressed_attn": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp]),
         "infllmv2_forward": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "infllmv2_decode_step": (ctypes.c_int,
                                  [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
@@ -184,11 +187,28 @@ def _nbytes(ws) -> int:
 
 
 def sparse_attn(p: Params, Q, K, V, idx, O, lse, ws=None, stream=None):
-    """Block-sparse attention; ws (OP_ATTN bytes) enables the packed K/V gather."""
+    """Block-sparse attention; ws (OP_ATTN bytes) enables the query-tile
+    schedule (groups of 8 or 16 heads) or the packed K/V gather."""
     _check("infllmv2_sparse_attn",
            load().infllmv2_sparse_attn(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx),
                                        _ptr(O), _ptr(lse), _ptr(ws), _nbytes(ws),
                                        _stream(stream)))
+
+
+def sparse_attn_per_token(p: Params, Q, K, V, idx, O, lse, ws=None, stream=None):
+    """Block-sparse attention, one work item per query token; ws
+    (OP_ATTN_PER_TOKEN bytes) enables the packed K/V gather."""
+    _check("infllmv2_sparse_attn_per_token",
+           load().infllmv2_sparse_attn_per_token(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V),
+                                                 _ptr(idx), _ptr(O), _ptr(lse), _ptr(ws),
+                                                 _nbytes(ws), _stream(stream)))
+
+
+def compressed_attn(p: Params, Q, Kc, Vc, O, lse, stream=None):
+    """Attention over the compressed windows (Kc, Vc from compress_keys of K, V)."""
+    _check("infllmv2_compressed_attn",
+           load().infllmv2_compressed_attn(ctypes.byref(p), _ptr(Q), _ptr(Kc), _ptr(Vc), _ptr(O),
+                                           _ptr(lse), _stream(stream)))
 
 
 def dense_attn(p: Params, Q, K, V, O, lse, ws=None, stream=None):
