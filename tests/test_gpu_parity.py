@@ -295,7 +295,8 @@ def test_compressed_attn_all_rows(cuda_lib, B, T, Hq, Hkv):
     none = np.isneginf(L_ref)            # rows that see no window: O = 0, lse = -inf
     assert np.array_equal(np.isneginf(Lg), none)
     assert np.abs(Og - O_ref).max() <= O_ATOL
-    assert np.abs(Lg[~none] - L_ref[~none]).max() <= LSE_ATOL
+    if (~none).any():
+        assert np.abs(Lg[~none] - L_ref[~none]).max() <= LSE_ATOL
 
 
 def test_compressed_attn_32k_sampled(cuda_lib):
