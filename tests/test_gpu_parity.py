@@ -700,13 +700,17 @@ def test_prefill_chunk_against_the_oracle(cuda_lib, case):
                 assert np.abs(Lg[b, hs, i] - l).max() <= LSE_ATOL
 
 
-def test_prefill_chunk_equals_the_whole_sequence_rows(cuda_lib):
-    """The chunk's rows are bit-identical to the same rows of a whole-sequence
-    forward on the GPU: every row's arithmetic is independent of how the
-    queries are grouped into tiles."""
+@pytest.mark.parametrize("q0", [1336, 1337], ids=["tile_aligned", "unaligned"])
+def test_prefill_chunk_equals_the_whole_sequence_rows(cuda_lib, q0):
+    """The chunk's selection is bit-identical to the same rows of a
+    whole-sequence forward on the GPU.  Its outputs are too when the chunk
+    starts on a query-tile boundary (8 tokens for 16-head groups: the tiles,
+    their block unions and so every row's arithmetic are the same); from an
+    unaligned start the tiles group other tokens, and the rows agree within
+    rounding."""
     import torch
     api = cuda_lib
-    B, T, Hq, Hkv, topk, q0 = 1, 3000, 32, 2, 16, 1337
+    B, T, Hq, Hkv, topk = 1, 3000, 32, 2, 16
     w, data, (Q, K, V, Kc), path, Og, Lg, ig = _run_chunk(api, B, T, Hq, Hkv, topk, q0, 0, 77)
     p = _params(api, w)
     O = torch.empty_like(Q)
@@ -717,5 +721,9 @@ def test_prefill_chunk_equals_the_whole_sequence_rows(cuda_lib):
     assert api.forward(p, Q, K, V, O, lse, Kc2, idx, ws) == api.PATH_SPARSE
     torch.cuda.synchronize()
     assert np.array_equal(idx.cpu().numpy()[:, :, q0:], ig)
-    assert np.array_equal(f64(O)[:, q0:], Og)
-    assert np.array_equal(f64(lse)[:, :, q0:], Lg)
+    if q0 % 8 == 0:
+        assert np.array_equal(f64(O)[:, q0:], Og)
+        assert np.array_equal(f64(lse)[:, :, q0:], Lg)
+    else:
+        assert np.abs(f64(O)[:, q0:] - Og).max() <= O_ATOL
+        assert np.abs(f64(lse)[:, :, q0:] - Lg).max() <= LSE_ATOL
