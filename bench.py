@@ -257,13 +257,32 @@ def run_prefill(api, wl, w, steps, warmup, dist, flush, time_e2e=True, clocks=No
     executed_score_flops *= B * Hkv
     idx_np = idx.cpu().numpy()
     cur = (np.arange(T) // 64)[None, None, :, None]
-    n_valid = ((idx_np >= 0) & (idx_np <= cur)).sum(axis=-1)
-    pairs = int(((n_valid + 1) // 2).sum())
-    # per gathered pair: S^T (128 keys x 16 heads x 128) and P V, 2 FLOP per MAC
-    executed_attn_flops = float(pairs) * 2 * (2 * 128 * 16 * 128)
+    valid = (idx_np >= 0) & (idx_np <= cur)
+    if G >= 8:
+        # query-tile schedule: each tile of 128/G tokens loads the union of its
+        # tokens' blocks once (K and V, 32 KB per block) and runs 128-key
+        # tiles of 128 rows (S and P V, 2 FLOP per MAC)
+        tpt = 128 // G
+        n_t = -(-T // tpt)
+        pad = n_t * tpt - T
+        u = np.where(valid, idx_np, -1)
+        if pad:
+            u = np.concatenate([u, np.full(u.shape[:2] + (pad, u.shape[3]), -1, u.dtype)], axis=2)
+        u = np.sort(u.reshape(B, Hkv, n_t, tpt * w.topk), axis=-1)
+        heads = (u >= 0) & np.concatenate([np.ones(u.shape[:3] + (1,), bool),
+                                           u[..., 1:] != u[..., :-1]], axis=-1)
+        n_u = heads.sum(axis=-1)
+        gathered_bytes = float(n_u.sum()) * 32768
+        executed_attn_flops = float(((n_u + 1) // 2).sum()) * 2 * (2 * 128 * 128 * 128)
+    else:
+        n_valid = valid.sum(axis=-1)
+        pairs = int(((n_valid + 1) // 2).sum())
+        gathered_bytes = float(pairs) * 65536
+        # per gathered pair: S^T (128 keys x 16 heads x 128) and P V, 2 FLOP per MAC
+        executed_attn_flops = float(pairs) * 2 * (2 * 128 * 16 * 128)
     gather = None
     if measure_gather:
-        gather = gather_roofline(api, aws, pairs, kern["sparse_attn"])
+        gather = gather_roofline(api, aws, gathered_bytes, kern["sparse_attn"])
     out = dict(ms=ms, step_ms=step_ms, kernels=kern, tokens=B * T, gather=gather,
                useful_attn_flops=useful_attn_flops, useful_score_flops=useful_score_flops,
                executed_score_flops=executed_score_flops, executed_attn_flops=executed_attn_flops,
@@ -277,10 +296,10 @@ def run_prefill(api, wl, w, steps, warmup, dist, flush, time_e2e=True, clocks=No
     return out
 
 
-def gather_roofline(api, tiles, pairs, attn_ms, rounds=2000, reps=5):
-    """The attention's L2 -> shared-memory gather against this GPU's ceiling
-    for that movement, measured now by the library's gather kernel over the
-    attention's own packed K/V tiles (L2-resident)."""
+def gather_roofline(api, tiles, per_launch, attn_ms, rounds=2000, reps=5):
+    """The attention's L2 -> shared-memory gather (per_launch bytes of K and V
+    blocks) against this GPU's ceiling for that movement, measured now by the
+    library's gather kernel over the attention's workspace (L2-resident)."""
     import torch
     stream = torch.cuda.current_stream()
     for _ in range(2):
@@ -296,13 +315,12 @@ def gather_roofline(api, tiles, pairs, attn_ms, rounds=2000, reps=5):
         rates.append(moved / (e0.elapsed_time(e1) / 1e3) / 1e9)
     assert api.get_status() == 0
     peak = statistics.median(rates)
-    per_launch = pairs * 65536  # K and V of two 64-key blocks per gathered pair
     achieved = per_launch / (attn_ms / 1e3) / 1e9
     return {"bound": "l2_gather", "kernel": "sparse_attn", "achieved": achieved, "peak": peak,
             "unit": "GB/s", "frac": achieved / peak, "bytes_per_launch": per_launch,
             "peak_source": "measured in this run: infllmv2_gather_peak, 16 KB bulk copies "
-                           "from the attention's packed K/V tiles into a 3 x 64 KB ring, "
-                           "one CTA per SM, median of 5"}
+                           "from an L2-resident buffer into a 3 x 64 KB ring, one CTA "
+                           "per SM, median of 5"}
 
 
 def time_chunk(api, p, Q, K, V, Kc, n, steps, warmup, flush):
@@ -466,6 +484,48 @@ def run_decode(api, wl, w, steps, warmup, flush):
     return dict(ms_per_step=per_step, tokens_per_s=B / (per_step / 1e3),
                 hbm_gbs=bytes_step / (per_step / 1e3) / 1e9, bytes_per_step=bytes_step,
                 lo_plane_bytes_per_step=kc_bytes, steps=steps, launches_per_step=6)
+
+
+def run_compressed(api, wl, w, steps, warmup, flush):
+    """The compressed-attention branch on a prefill workload: compress V (the
+    keys' compression is the selection's), then every query row over its
+    visible window means.  Inputs resident; the compressed keys precomputed."""
+    import torch
+    data = wl.make_prefill(w)
+    Q, K, V = (wl.to_torch_bf16(data[x]).cuda() for x in "QKV")
+    B, T, Hq, Hkv = w.B, w.T, w.Hq, w.Hkv
+    p = api.make_params(B, T, Hq, Hkv, topk=w.topk, n_init=w.n_init, n_local=w.n_local,
+                        switch_threshold=w.threshold)
+    n_c = api.num_compressed(T)
+    Kc = torch.empty((B, n_c, Hkv, 2, 128), dtype=torch.bfloat16, device="cuda")
+    Vc = torch.empty_like(Kc)
+    api.compress_keys(p, K, Kc)
+    O = torch.empty_like(Q)
+    lse = torch.empty((B, Hq, T), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        flush()
+        api.compress_keys(p, V, Vc)
+        api.compressed_attn(p, Q, Kc, Vc, O, lse)
+    torch.cuda.synchronize()
+    ms, ams = [], []
+    for _ in range(steps):
+        flush()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record(stream)
+        api.compress_keys(p, V, Vc)
+        e[1].record(stream)
+        api.compressed_attn(p, Q, Kc, Vc, O, lse)
+        e[2].record(stream)
+        torch.cuda.synchronize()
+        ms.append(e[0].elapsed_time(e[2]))
+        ams.append(e[1].elapsed_time(e[2]))
+    assert api.get_status() == 0
+    v = [0 if t < 31 else min(n_c, (t - 31) // 16 + 1) for t in range(T)]
+    flops = 4.0 * 128 * Hq * B * float(sum(v))  # q.Kc and P Vc over the visible windows
+    del Q, K, V, Kc, Vc, O, lse
+    torch.cuda.empty_cache()
+    return dict(ms=sum(ms) / len(ms), attn_ms=sum(ams) / len(ams), tokens=B * T, flops=flops)
 
 
 def run_dense(api, wl, w, steps, warmup, flush):
@@ -694,6 +754,14 @@ def main():
             "ms_per_step": d1, "tflops": dn["flops"] / (d1 / 1e3) / 1e12,
             "tensor_frac_of_burst": dn["flops"] / (d1 / 1e3) / 1e12 / peaks["bf16_tflops"],
             "flops_per_step": dn["flops"]}
+        cm = run_compressed(api, wl, w, args.steps, args.warmup, flush)
+        c1 = dist.max(cm["ms"])
+        extras["compressed_branch_T131072"] = {
+            "tokens_per_s": whole_job_rate(cm["tokens"], dist.world, c1), "ms_per_step": c1,
+            "attn_ms": cm["attn_ms"], "tflops": cm["flops"] / (cm["attn_ms"] / 1e3) / 1e12,
+            "tensor_frac_of_burst": cm["flops"] / (cm["attn_ms"] / 1e3) / 1e12 / peaks["bf16_tflops"],
+            "flops_per_step": cm["flops"],
+            "timing": "compress V + attention over the visible window means; L2 flushed"}
         wd = wl.WORKLOADS[DECODE]
         dec = run_decode(api, wl, wd, 256, 8, flush)
         dms = dist.max(dec["ms_per_step"])
