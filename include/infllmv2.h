@@ -96,6 +96,7 @@ typedef struct infllmv2_params {
 #define INFLLMV2_OP_DECODE   3
 #define INFLLMV2_OP_ATTN     4  /* sparse_attn: union lists (groups of 8 or 16 heads) or packed K/V */
 #define INFLLMV2_OP_ATTN_PER_TOKEN 5  /* sparse_attn_per_token: packed K and V */
+#define INFLLMV2_OP_FORWARD_FP32   6  /* forward_fp32: block scores (0 when dense) */
 
 /* Path reported by infllmv2_forward. */
 #define INFLLMV2_PATH_DENSE  1
@@ -214,6 +215,24 @@ int infllmv2_forward(const infllmv2_params* p, const void* Q, const void* K,
                      int32_t* path_used, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * The fp32 validation build of infllmv2_forward: the same switch and the same
+ * steps (compressed keys, per-head softmax scores summed over the group and
+ * max-pooled to blocks, top-k with the forced blocks, block-sparse or dense
+ * causal attention), with every product and sum in fp32 on the CUDA cores:
+ * compressed keys stored in fp32, scores and softmax in fp32, P and O never
+ * rounded to bf16.  For checking the method's arithmetic to ~1e-6 (the
+ * tensor-core path's error is set by bf16 rounding); not tuned for speed.
+ *   Q, K, V as for infllmv2_forward (bf16, in);
+ *   O [B, T, Hq, d] fp32, lse [B, Hq, T] fp32 (out);
+ *   Kc32_ws [B, n_c, Hkv, d] fp32 and idx_ws [B, Hkv, T, topk] int32 (out;
+ *     unused and may be NULL when dense);
+ *   ws: at least infllmv2_workspace_bytes(p, INFLLMV2_OP_FORWARD_FP32) bytes.
+ */
+int infllmv2_forward_fp32(const infllmv2_params* p, const void* Q, const void* K,
+                          const void* V, float* O, float* lse, float* Kc32_ws, int32_t* idx_ws,
+                          int32_t* path_used, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Chunked prefill: queries for the tokens q_offset .. q_offset+q_len-1 of a
  * sequence whose keys, values and compressed keys are already in the caches
  * (the chunk's own tokens included).  Each query row t gets exactly what
@@ -238,6 +257,36 @@ int infllmv2_prefill_chunk(const infllmv2_params* p, int32_t q_offset, int32_t q
                            const void* Q, const void* K, const void* V, const void* Kc,
                            void* O, float* lse, int32_t* idx, int32_t* path_used, void* ws,
                            size_t ws_bytes, void* stream);
+
+/*
+ * Variable-length prefill: n_seqs sequences of different lengths packed
+ * together, each a query chunk over its own caches (the last q_len_i of its
+ * k_len_i tokens: q_len_i = k_len_i is an ordinary prefill), so that serving
+ * can prefill a batch of ragged prompts with one call (reportify digest,
+ * Performance Evaluation: prefill speed-up on long inputs).  Every row gets
+ * exactly what infllmv2_prefill_chunk gives it, with the switch taken per
+ * sequence (dense iff k_len_i <= p->switch_threshold).  p->B and p->T are
+ * ignored.  The sequences run one after another on `stream` and share ws.
+ *   cu_seqlens_q, cu_seqlens_k: HOST int32 arrays of n_seqs + 1 ascending
+ *     offsets from 0; q_len_i = cu_seqlens_q[i+1] - cu_seqlens_q[i] <= k_len_i;
+ *   Q, O [total_q, Hq, d] bf16; K, V [total_k, Hkv, d] bf16;
+ *   Kc: the sequences' compressed keys one after another, sequence i's
+ *     n_c(k_len_i) rows [n_c_i, Hkv, 2, d] (as infllmv2_compress_keys writes
+ *     them for B = 1); unused and may be NULL when no sequence is sparse;
+ *   lse: sequence i's [Hq, q_len_i] fp32 block at element Hq * cu_seqlens_q[i];
+ *   idx: sequence i's [Hkv, q_len_i, topk] int32 block at element
+ *     Hkv * topk * cu_seqlens_q[i] (unused, may be NULL, when all are dense);
+ *   path_used: host int32[n_seqs] (may be NULL);
+ *   ws: at least infllmv2_prefill_varlen_workspace_bytes(...) bytes.
+ */
+size_t infllmv2_prefill_varlen_workspace_bytes(const infllmv2_params* p, int32_t n_seqs,
+                                               const int32_t* cu_seqlens_q,
+                                               const int32_t* cu_seqlens_k);
+int infllmv2_prefill_varlen(const infllmv2_params* p, int32_t n_seqs,
+                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                            const void* Q, const void* K, const void* V, const void* Kc,
+                            void* O, float* lse, int32_t* idx, int32_t* path_used, void* ws,
+                            size_t ws_bytes, void* stream);
 
 /*
  * One decode step for B sequences (reportify digest, Performance Evaluation:

@@ -23,7 +23,7 @@ def lib():
 def declared_symbols():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(infllmv2_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(infllmv2_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_the_binding_exports():
@@ -177,3 +177,21 @@ def test_prefill_chunk_workspace_sizes(lib):
         (-(-sel // 256) * 256) + _union_bytes(1, n, 2, 16, 64)
     d = api.make_params(1, 4096, 32, 2, switch_threshold=8192)
     assert api.prefill_chunk_workspace_bytes(d, 1000, 3096) == 0
+
+
+def test_prefill_varlen_rejected_on_host(lib):
+    p = api.make_params(1, 1, 32, 2, topk=8, switch_threshold=0)
+    # a sequence with more queries than keys
+    with pytest.raises(api.InfLLMV2Error):
+        api.prefill_varlen_workspace_bytes(p, [0, 10, 30], [0, 10, 20])
+    # offsets must start at 0 and ascend
+    with pytest.raises(api.InfLLMV2Error):
+        api.prefill_varlen_workspace_bytes(p, [5, 10], [0, 10])
+    # no sequences: nothing to do
+    assert api.prefill_varlen_workspace_bytes(p, [0], [0]) == 0
+    # the workspace is the largest any one sequence needs (they share it)
+    w1 = api.prefill_chunk_workspace_bytes(api.make_params(1, 3000, 32, 2, topk=8,
+                                                           switch_threshold=0), 0, 3000)
+    w2 = api.prefill_chunk_workspace_bytes(api.make_params(1, 2000, 32, 2, topk=8,
+                                                           switch_threshold=0), 1000, 1000)
+    assert api.prefill_varlen_workspace_bytes(p, [0, 3000, 4000], [0, 3000, 5000]) == max(w1, w2)

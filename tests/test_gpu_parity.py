@@ -727,3 +727,71 @@ def test_prefill_chunk_equals_the_whole_sequence_rows(cuda_lib, q0):
     else:
         assert np.abs(f64(O)[:, q0:] - Og).max() <= O_ATOL
         assert np.abs(f64(lse)[:, :, q0:] - Lg).max() <= LSE_ATOL
+
+
+# ---------------------------------------------------------------------------
+# variable-length prefill: a packed batch of ragged sequences
+# ---------------------------------------------------------------------------
+def test_prefill_varlen_against_the_oracle(cuda_lib):
+    """Five sequences of different lengths in one call: full prefills and
+    tail chunks, sparse (longer than the threshold) and dense, one with no
+    query at all.  Each row against the oracle's chunked forward of its own
+    sequence: selection by the band rule, O and LSE over the GPU's own
+    selection (dense rows over every key)."""
+    import torch
+    api = cuda_lib
+    Hq, Hkv, topk, thr = 32, 2, 8, 1024
+    seqs = [(1500, 1500), (700, 700), (2000, 333), (64, 10), (1200, 0)]  # (k_len, q_len)
+    datas = [wl.make_prefill(wl.small_workload(B=1, T=k, Hq=Hq, Hkv=Hkv, topk=topk, needles=1,
+                                               seed=90 + i, threshold=thr))
+             for i, (k, _) in enumerate(seqs)]
+    cu_q, cu_k = [0], [0]
+    for k, q in seqs:
+        cu_q.append(cu_q[-1] + q)
+        cu_k.append(cu_k[-1] + k)
+    Qp = torch.cat([gpu_bf16(d["Q"])[0, k - q:] for d, (k, q) in zip(datas, seqs)])
+    Kp = torch.cat([gpu_bf16(d["K"])[0] for d in datas])
+    Vp = torch.cat([gpu_bf16(d["V"])[0] for d in datas])
+    kcs = []
+    for d, (k, _) in zip(datas, seqs):
+        n_c = api.num_compressed(k)
+        Kc = torch.empty((1, max(n_c, 1), Hkv, 2, 128), dtype=torch.bfloat16, device="cuda")
+        if n_c:
+            api.compress_keys(api.make_params(1, k, Hq, Hkv), gpu_bf16(d["K"]), Kc)
+        kcs.append(Kc[0, :n_c])
+    Kcp = torch.cat(kcs)
+    p = api.make_params(1, 1, Hq, Hkv, topk=topk, switch_threshold=thr)
+    O = torch.full((cu_q[-1], Hq, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((Hq * cu_q[-1],), float("nan"), dtype=torch.float32, device="cuda")
+    idx = torch.full((Hkv * topk * cu_q[-1],), -7, dtype=torch.int32, device="cuda")
+    ws = torch.empty(max(api.prefill_varlen_workspace_bytes(p, cu_q, cu_k), 16), dtype=torch.uint8,
+                     device="cuda")
+    paths = api.prefill_varlen(p, cu_q, cu_k, Qp, Kp, Vp, Kcp, O, lse, idx, ws)
+    torch.cuda.synchronize()
+    assert api.get_status() == 0
+    Og, Lg, ig = f64(O), f64(lse), idx.cpu().numpy()
+    G = Hq // Hkv
+    for i, (d, (k, q)) in enumerate(zip(datas, seqs)):
+        assert paths[i] == (api.PATH_DENSE if k <= thr else api.PATH_SPARSE)
+        if q == 0:
+            continue
+        Qf, Kf, Vf = (wl.bf16_to_f64(d[x])[0] for x in "QKV")
+        op = orc.Params(topk=topk, threshold=thr)
+        Kc = orc.compress_keys(Kf[None], op)[0]
+        q0 = k - q
+        Oi = Og[cu_q[i]:cu_q[i + 1]]
+        Li = Lg[Hq * cu_q[i]:Hq * cu_q[i + 1]].reshape(Hq, q)
+        Ii = ig[Hkv * topk * cu_q[i]:Hkv * topk * cu_q[i + 1]].reshape(Hkv, q, topk)
+        for g in range(Hkv):
+            hs = slice(g * G, (g + 1) * G)
+            for r in range(q):
+                t = q0 + r
+                if k > thr:
+                    sel = orc.select_query(Qf[t, hs], Kc[:, g], t, op)
+                    check_selection_row(sel, Ii[g, r], topk)
+                    keys = orc.selected_keys(Ii[g, r], t, op)
+                else:
+                    keys = np.arange(t + 1)
+                o, l = orc.attend(Qf[t, hs], Kf[:, g], Vf[:, g], keys, op.sm_scale(128))
+                assert np.abs(Oi[r, hs] - o).max() <= O_ATOL
+                assert np.abs(Li[hs, r] - l).max() <= LSE_ATOL

@@ -170,6 +170,53 @@ int ctx_or_error(DevCtx* ctx) {
   return get_dev_ctx(ctx) == cudaSuccess ? INFLLMV2_OK : INFLLMV2_ERR_CUDA;
 }
 
+size_t chunk_ws_bytes(const Geometry& g, bool dense) {
+  return dense ? 0 : align256(select_ws_bytes(g)) + attn_ws_bytes(g);
+}
+
+// The chunk's kernels: dense attention, or scoring -> top-k -> sparse
+// attention.  Arguments already checked.
+int enqueue_chunk(const Geometry& g, bool dense, const void* Q, const void* K, const void* V,
+                  const void* Kc, void* O, float* lse, int32_t* idx, void* ws, size_t ws_bytes,
+                  const DevCtx& ctx, cudaStream_t st) {
+  if (dense) return launch_dense_tile(g, Q, K, V, O, lse, ctx, st);
+  const size_t sel = align256(select_ws_bytes(g));
+  if (ws_bytes < sel) return INFLLMV2_ERR_WORKSPACE;
+  if (int e = launch_score_blocks(g, Q, Kc, static_cast<float*>(ws), ctx, st)) return e;
+  if (int e = launch_topk(g, static_cast<float*>(ws), idx, st)) return e;
+  return enqueue_sparse(g, Q, K, V, idx, O, lse, static_cast<uint8_t*>(ws) + sel, ws_bytes - sel,
+                        false, ctx, st);
+}
+
+// A packed batch of sequences: cu_seqlens_q / _k (host) hold n_seqs + 1
+// ascending offsets from 0; every sequence's query count is at most its key
+// count.  *need: the largest workspace any one sequence needs (they run one
+// after another on the stream and share it).
+int check_varlen(const infllmv2_params* p, int32_t n_seqs, const int32_t* cu_q,
+                 const int32_t* cu_k, size_t* need) {
+  if (!p || n_seqs < 0) return INFLLMV2_ERR_INVALID_ARG;
+  if (n_seqs > 0 && (!cu_q || !cu_k)) return INFLLMV2_ERR_INVALID_ARG;
+  if (n_seqs > 0 && (cu_q[0] != 0 || cu_k[0] != 0)) return INFLLMV2_ERR_INVALID_ARG;
+  *need = 0;
+  for (int i = 0; i < n_seqs; ++i) {
+    const int64_t ql = static_cast<int64_t>(cu_q[i + 1]) - cu_q[i];
+    const int64_t kl = static_cast<int64_t>(cu_k[i + 1]) - cu_k[i];
+    if (ql < 0 || kl < 0 || ql > kl) return INFLLMV2_ERR_INVALID_ARG;
+    infllmv2_params pi = *p;
+    pi.B = 1;
+    pi.T = static_cast<int32_t>(kl);
+    Geometry g;
+    if (int e = validate_chunk(&pi, static_cast<int32_t>(kl - ql), static_cast<int32_t>(ql), &g))
+      return e;
+    const bool dense = kl <= p->switch_threshold;
+    if (!dense && ql > 0)
+      if (int e = check_select_size(g)) return e;
+    const size_t w = ql > 0 ? chunk_ws_bytes(g, dense) : 0;
+    if (w > *need) *need = w;
+  }
+  return INFLLMV2_OK;
+}
+
 }  // namespace
 }  // namespace infllmv2
 
@@ -201,7 +248,8 @@ void infllmv2_set_wait_limit(int64_t ns) {
 size_t infllmv2_workspace_bytes(const infllmv2_params* p, int32_t op) {
   Geometry g;
   // the dense forward takes no top-k parameters (as infllmv2_dense_attn)
-  const bool dense_fwd = op == INFLLMV2_OP_FORWARD && p && p->T <= p->switch_threshold;
+  const bool dense_fwd = (op == INFLLMV2_OP_FORWARD || op == INFLLMV2_OP_FORWARD_FP32) && p &&
+                         p->T <= p->switch_threshold;
   if (validate(p, !dense_fwd, &g) != INFLLMV2_OK) return SIZE_MAX;
   switch (op) {
     case INFLLMV2_OP_SELECT:
@@ -213,6 +261,9 @@ size_t infllmv2_workspace_bytes(const infllmv2_params* p, int32_t op) {
       return g.T > INFLLMV2_MAX_DECODE_T ? SIZE_MAX : decode_ws_bytes(g);
     case INFLLMV2_OP_ATTN: return attn_ws_bytes(g);
     case INFLLMV2_OP_ATTN_PER_TOKEN: return packed_kv_bytes(g);
+    case INFLLMV2_OP_FORWARD_FP32:
+      if (dense_fwd) return 0;
+      return check_select_size(g) ? SIZE_MAX : select_ws_bytes(g);
     default: return SIZE_MAX;
   }
 }
@@ -318,12 +369,34 @@ int infllmv2_forward(const infllmv2_params* p, const void* Q, const void* K, con
                               ws_bytes - sel, stream);
 }
 
+int infllmv2_forward_fp32(const infllmv2_params* p, const void* Q, const void* K, const void* V,
+                          float* O, float* lse, float* Kc32_ws, int32_t* idx_ws,
+                          int32_t* path_used, void* ws, size_t ws_bytes, void* stream) {
+  if (!p) return INFLLMV2_ERR_INVALID_ARG;
+  const bool dense = p->T <= p->switch_threshold;
+  Geometry g;
+  if (int e = validate(p, !dense, &g)) return e;
+  if (!dense)
+    if (int e = check_select_size(g)) return e;
+  if (path_used) *path_used = dense ? INFLLMV2_PATH_DENSE : INFLLMV2_PATH_SPARSE;
+  if (empty(g)) return INFLLMV2_OK;
+  if (int e = check_ptrs({Q, K, V, O, lse})) return e;
+  if (!dense) {
+    if (int e = check_ptrs({idx_ws, ws})) return e;
+    if (g.n_c > 0)
+      if (int e = check_ptrs({Kc32_ws})) return e;
+    if (ws_bytes < select_ws_bytes(g)) return INFLLMV2_ERR_WORKSPACE;
+  }
+  return launch_forward_f32(g, Q, K, V, O, lse, Kc32_ws, idx_ws, static_cast<float*>(ws), dense,
+                            static_cast<cudaStream_t>(stream));
+}
+
 size_t infllmv2_prefill_chunk_workspace_bytes(const infllmv2_params* p, int32_t q_offset,
                                               int32_t q_len) {
   Geometry g;
   if (validate_chunk(p, q_offset, q_len, &g) != INFLLMV2_OK) return SIZE_MAX;
   if (p->T <= p->switch_threshold) return 0;
-  return check_select_size(g) ? SIZE_MAX : align256(select_ws_bytes(g)) + attn_ws_bytes(g);
+  return check_select_size(g) ? SIZE_MAX : chunk_ws_bytes(g, false);
 }
 
 int infllmv2_prefill_chunk(const infllmv2_params* p, int32_t q_offset, int32_t q_len,
@@ -343,16 +416,74 @@ int infllmv2_prefill_chunk(const infllmv2_params* p, int32_t q_offset, int32_t q
     if (g.n_c > 0)
       if (int e = check_ptrs({Kc})) return e;
   }
-  const size_t sel = dense ? 0 : align256(select_ws_bytes(g));
-  if (ws_bytes < sel) return INFLLMV2_ERR_WORKSPACE;
+  DevCtx ctx;
+  if (int e = ctx_or_error(&ctx)) return e;
+  return enqueue_chunk(g, dense, Q, K, V, Kc, O, lse, idx, ws, ws_bytes, ctx,
+                       static_cast<cudaStream_t>(stream));
+}
+
+size_t infllmv2_prefill_varlen_workspace_bytes(const infllmv2_params* p, int32_t n_seqs,
+                                               const int32_t* cu_seqlens_q,
+                                               const int32_t* cu_seqlens_k) {
+  size_t need = 0;
+  if (check_varlen(p, n_seqs, cu_seqlens_q, cu_seqlens_k, &need) != INFLLMV2_OK) return SIZE_MAX;
+  return need;
+}
+
+int infllmv2_prefill_varlen(const infllmv2_params* p, int32_t n_seqs,
+                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                            const void* Q, const void* K, const void* V, const void* Kc, void* O,
+                            float* lse, int32_t* idx, int32_t* path_used, void* ws,
+                            size_t ws_bytes, void* stream) {
+  size_t need = 0;
+  if (int e = check_varlen(p, n_seqs, cu_seqlens_q, cu_seqlens_k, &need)) return e;
+  if (n_seqs == 0 || cu_seqlens_q[n_seqs] == 0) return INFLLMV2_OK;
+  if (int e = check_ptrs({Q, K, V, O, lse})) return e;
+  bool any_sparse = false, any_cmp = false;
+  for (int i = 0; i < n_seqs; ++i) {
+    const int kl = cu_seqlens_k[i + 1] - cu_seqlens_k[i];
+    if (kl > p->switch_threshold && cu_seqlens_q[i + 1] > cu_seqlens_q[i]) {
+      any_sparse = true;
+      any_cmp |= num_compressed(kl) > 0;
+    }
+  }
+  if (any_sparse)
+    if (int e = check_ptrs({idx, ws})) return e;
+  if (any_cmp)
+    if (int e = check_ptrs({Kc})) return e;
+  if (ws_bytes < need) return INFLLMV2_ERR_WORKSPACE;
   DevCtx ctx;
   if (int e = ctx_or_error(&ctx)) return e;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dense) return launch_dense_tile(g, Q, K, V, O, lse, ctx, st);
-  if (int e = launch_score_blocks(g, Q, Kc, static_cast<float*>(ws), ctx, st)) return e;
-  if (int e = launch_topk(g, static_cast<float*>(ws), idx, st)) return e;
-  return enqueue_sparse(g, Q, K, V, idx, O, lse, static_cast<uint8_t*>(ws) + sel, ws_bytes - sel,
-                        false, ctx, st);
+  const int Hq = p->Hq, Hkv = p->Hkv;
+  int64_t cmp_off = 0;  // compressed rows before sequence i
+  for (int i = 0; i < n_seqs; ++i) {
+    const int q_start = cu_seqlens_q[i], q_len = cu_seqlens_q[i + 1] - q_start;
+    const int k_start = cu_seqlens_k[i], k_len = cu_seqlens_k[i + 1] - k_start;
+    const bool dense = k_len <= p->switch_threshold;
+    if (path_used) path_used[i] = dense ? INFLLMV2_PATH_DENSE : INFLLMV2_PATH_SPARSE;
+    infllmv2_params pi = *p;
+    pi.B = 1;
+    pi.T = k_len;
+    Geometry g;
+    if (int e = validate_chunk(&pi, k_len - q_len, q_len, &g)) return e;
+    if (q_len > 0) {
+      const size_t row = static_cast<size_t>(kHeadDim) * sizeof(__nv_bfloat16);
+      const uint8_t* Qi = static_cast<const uint8_t*>(Q) + static_cast<size_t>(q_start) * Hq * row;
+      uint8_t* Oi = static_cast<uint8_t*>(O) + static_cast<size_t>(q_start) * Hq * row;
+      const uint8_t* Ki = static_cast<const uint8_t*>(K) + static_cast<size_t>(k_start) * Hkv * row;
+      const uint8_t* Vi = static_cast<const uint8_t*>(V) + static_cast<size_t>(k_start) * Hkv * row;
+      const uint8_t* Kci =
+          Kc ? static_cast<const uint8_t*>(Kc) + static_cast<size_t>(cmp_off) * Hkv * 2 * row
+             : nullptr;
+      float* lsei = lse + static_cast<int64_t>(q_start) * Hq;
+      int32_t* idxi = idx ? idx + static_cast<int64_t>(q_start) * Hkv * p->topk : nullptr;
+      if (int e = enqueue_chunk(g, dense, Qi, Ki, Vi, Kci, Oi, lsei, idxi, ws, ws_bytes, ctx, st))
+        return e;
+    }
+    cmp_off += num_compressed(k_len);
+  }
+  return INFLLMV2_OK;
 }
 
 int infllmv2_decode_step(const infllmv2_params* p, const void* q, const void* k_new,

@@ -141,6 +141,11 @@ int launch_union_tile(const Geometry& g, const void* Q, const void* K, const voi
                       cudaStream_t st);
 int launch_compressed_tile(const Geometry& g, const void* Q, const void* Kc, const void* Vc,
                            void* O, float* lse, const DevCtx& ctx, cudaStream_t st);
+// The fp32 validation build of the forward (fp32_path.cu): dense, or compress
+// into Kc32 -> block scores into `scores` -> top-k into idx -> attention.
+int launch_forward_f32(const Geometry& g, const void* Q, const void* K, const void* V, void* O,
+                       float* lse, float* Kc32, int32_t* idx, float* scores, bool dense,
+                       cudaStream_t st);
 // Decode (decode.cu); g.T is the cache capacity.
 size_t decode_ws_bytes(const Geometry& g);
 int launch_decode_step(const Geometry& g, const void* q, const void* k_new, const void* v_new,

@@ -26,7 +26,7 @@ ERR_WORKSPACE = -5
 ERR_DEVICE_CHECK = -6
 STATUS_TIMEOUT = 0x1
 STATUS_SEQ_FULL = 0x2
-OP_SELECT, OP_FORWARD, OP_DECODE, OP_ATTN, OP_ATTN_PER_TOKEN = 1, 2, 3, 4, 5
+OP_SELECT, OP_FORWARD, OP_DECODE, OP_ATTN, OP_ATTN_PER_TOKEN, OP_FORWARD_FP32 = 1, 2, 3, 4, 5, 6
 PATH_DENSE, PATH_SPARSE = 1, 2
 
 # every symbol include/infllmv2.h declares
@@ -37,7 +37,8 @@ EXPORTS = (
     "infllmv2_set_wait_limit", "infllmv2_selftest_timeout", "infllmv2_strerror",
     "infllmv2_version", "infllmv2_decode_step_noalloc", "infllmv2_prefill_chunk",
     "infllmv2_prefill_chunk_workspace_bytes", "infllmv2_gather_peak",
-    "infllmv2_sparse_attn_per_token", "infllmv2_compressed_attn",
+    "infllmv2_sparse_attn_per_token", "infllmv2_compressed_attn", "infllmv2_forward_fp32",
+    "infllmv2_prefill_varlen", "infllmv2_prefill_varlen_workspace_bytes",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -89,6 +90,7 @@ def load(path: Optional[str] = None):
         "infllmv2_dense_attn": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
         "infllmv2_compressed_attn": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp]),
         "infllmv2_forward": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
+        "infllmv2_forward_fp32": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "infllmv2_decode_step": (ctypes.c_int,
                                  [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "infllmv2_decode_step_noalloc": (ctypes.c_int,
@@ -97,6 +99,9 @@ def load(path: Optional[str] = None):
         "infllmv2_prefill_chunk": (ctypes.c_int, [P, i32, i32, vp, vp, vp, vp, vp, vp, vp,
                                                   vp, vp, sz, vp]),
         "infllmv2_prefill_chunk_workspace_bytes": (sz, [P, i32, i32]),
+        "infllmv2_prefill_varlen": (ctypes.c_int, [P, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                                   vp, vp, sz, vp]),
+        "infllmv2_prefill_varlen_workspace_bytes": (sz, [P, i32, vp, vp]),
         "infllmv2_num_compressed": (i32, [i32]),
         "infllmv2_get_status": (ctypes.c_int, [vp, ctypes.POINTER(i32)]),
         "infllmv2_set_wait_limit": (None, [ctypes.c_int64]),
@@ -228,6 +233,17 @@ def forward(p: Params, Q, K, V, O, lse, Kc_ws=None, idx_ws=None, ws=None, stream
     return int(path.value)
 
 
+def forward_fp32(p: Params, Q, K, V, O, lse, Kc32_ws=None, idx_ws=None, ws=None,
+                 stream=None) -> int:
+    """The fp32 validation build of forward (O fp32); returns the path taken."""
+    path = ctypes.c_int32(0)
+    _check("infllmv2_forward_fp32",
+           load().infllmv2_forward_fp32(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
+                                        _ptr(lse), _ptr(Kc32_ws), _ptr(idx_ws), ctypes.byref(path),
+                                        _ptr(ws), _nbytes(ws), _stream(stream)))
+    return int(path.value)
+
+
 def prefill_chunk_workspace_bytes(p: Params, q_offset: int, q_len: int) -> int:
     n = load().infllmv2_prefill_chunk_workspace_bytes(ctypes.byref(p), q_offset, q_len)
     if n == ctypes.c_size_t(-1).value:
@@ -246,6 +262,37 @@ def prefill_chunk(p: Params, q_offset: int, q_len: int, Q, K, V, Kc, O, lse, idx
                                          _ptr(V), _ptr(Kc), _ptr(O), _ptr(lse), _ptr(idx),
                                          ctypes.byref(path), _ptr(ws), nbytes, _stream(stream)))
     return int(path.value)
+
+
+def _i32_array(xs):
+    arr = (ctypes.c_int32 * len(xs))(*[int(x) for x in xs])
+    return arr
+
+
+def prefill_varlen_workspace_bytes(p: Params, cu_q, cu_k) -> int:
+    n = len(cu_q) - 1
+    n_bytes = load().infllmv2_prefill_varlen_workspace_bytes(
+        ctypes.byref(p), n, ctypes.cast(_i32_array(cu_q), ctypes.c_void_p),
+        ctypes.cast(_i32_array(cu_k), ctypes.c_void_p))
+    if n_bytes == ctypes.c_size_t(-1).value:
+        raise InfLLMV2Error("infllmv2_prefill_varlen_workspace_bytes", ERR_INVALID_ARG)
+    return int(n_bytes)
+
+
+def prefill_varlen(p: Params, cu_q, cu_k, Q, K, V, Kc, O, lse, idx=None, ws=None,
+                   stream=None):
+    """A packed batch of ragged sequences (host offset lists cu_q, cu_k);
+    returns the path taken per sequence."""
+    n = len(cu_q) - 1
+    aq, ak = _i32_array(cu_q), _i32_array(cu_k)
+    paths = (ctypes.c_int32 * max(n, 1))()
+    _check("infllmv2_prefill_varlen",
+           load().infllmv2_prefill_varlen(ctypes.byref(p), n, ctypes.cast(aq, ctypes.c_void_p),
+                                          ctypes.cast(ak, ctypes.c_void_p), _ptr(Q), _ptr(K),
+                                          _ptr(V), _ptr(Kc), _ptr(O), _ptr(lse), _ptr(idx),
+                                          ctypes.cast(paths, ctypes.c_void_p), _ptr(ws),
+                                          _nbytes(ws), _stream(stream)))
+    return [int(paths[i]) for i in range(n)]
 
 
 def decode_step(p: Params, q, k_new, v_new, K_cache, V_cache, Kc_cache, seqlens, O, lse,
