@@ -7,10 +7,11 @@
 // tiles (tcgen05.mma, M = 128):
 //
 //   S[128 rows x KT keys] = Q (K-major, 128-byte swizzle) x K_tile^T
-//   O[128 rows x 128 d ] += P (K-major, no swizzle)      x V_tile (MN-major)
+//   O[128 rows x 128 d ] += P (tensor memory)            x V_tile (MN-major)
 //
-// with S double-buffered and O accumulated in tensor memory.  Three key
-// streams share the kernel:
+// with S and P double-buffered and O accumulated in tensor memory (P is the
+// A operand straight from tensor memory, so it never touches shared memory).
+// Three key streams share the kernel:
 //
 //   dense      every key 0 .. t: exact dense causal attention (InfLLM-V2 skill
 //              write-up, Architecture Overview, the dense pathway bullet);
@@ -29,11 +30,14 @@
 //
 // Warp roles: warp 0 loads Q (double-buffered) and the key tiles (K and V of
 // a tile in one ring stage) by TMA; warp 1 owns tensor memory and one thread
-// issues the MMAs; warps 2-5 are the softmax, one thread per query row (TMEM
-// lane), so a row's maximum and sum need no cross-thread reduction.  Each row
-// keeps a reference maximum m that moves only when a score exceeds it by more
-// than 8 (log2 units), so P = exp2(s - m) <= 256 is exact enough in bf16 and
-// the O accumulator is rescaled in tensor memory only on those (rare) moves.
+// issues the MMAs; warps 2-9 are the softmax, two warpgroups on the same 128
+// rows (thread = TMEM lane = query row), warpgroup hf taking the tile's keys
+// hf*KT/2 .. (hf+1)*KT/2 - 1 (in the union stream: one selected block each).
+// Each row keeps a reference maximum m, common to its two halves, that moves
+// only when a score exceeds it by more than 8 (log2 units): P = exp2(s - m)
+// <= 256 is exact enough in bf16, the halves exchange maxima only on those
+// (rare) moves, and only then is the O accumulator rescaled in tensor memory.
+// A half whose keys no row of its warp may see skips its exponentials.
 // Persistent CTAs, one per SM, take the query tiles heaviest first.
 #include "common.cuh"
 #include "sm100.cuh"
@@ -66,19 +70,24 @@ struct TileCfg {
   static constexpr int kVBytes = KT * 256;
   static constexpr int kStageBytes = kKBytes + kVBytes;
   static constexpr int kQBytes = 128 * 256;
-  static constexpr int kPBytes = 128 * KT * 2;
-  static constexpr uint32_t kOCol = 2 * KT;                      // S0, S1, then O
-  static constexpr uint32_t kTmemCols = MODE == kTileCompressed ? 256 : 512;
-  static constexpr int kThreads = 64 + 128;
+  static constexpr int H = KT / 2;                               // keys per softmax warpgroup
+  // tensor memory: S0, S1 (KT fp32 columns each), O (128), P0, P1 (KT/2
+  // columns of packed bf16 pairs each)
+  static constexpr uint32_t kOCol = 2 * KT;
+  static constexpr uint32_t kPCol = kOCol + 128;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr int kThreads = 64 + 256;
 };
 
 struct TileSmem {
   uint64_t q_full[2], q_empty[2];
   uint64_t kv_full[3], kv_empty[3];
-  uint64_t s_full[2];
-  uint64_t p_full, pv_done, o_free, drain;
+  uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t o_free, drain;
   uint32_t tmem_base;
   int abort_flag;
+  float xch[2][2][128];  // per tile parity and warpgroup: a row's half maximum
+  float xl[2][128];      // per warpgroup: a row's half sum, at the item's end
 };
 
 constexpr float kTileSlack = 8.0f;   // log2 units
@@ -138,8 +147,7 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint8_t* sQ = base;                                   // 2 x 32 KB
   uint8_t* sKV = sQ + 2 * C::kQBytes;                   // stages: K planes, then V
-  uint8_t* sP = sKV + C::kStages * C::kStageBytes;      // P, 128 rows x KT keys
-  TileSmem& sm = *reinterpret_cast<TileSmem*>(sP + C::kPBytes);
+  TileSmem& sm = *reinterpret_cast<TileSmem*>(sKV + C::kStages * C::kStageBytes);
 
   const int warp = warp_id(), lane = lane_id();
   const int n_qt = (args.Tq + TPT - 1) / TPT;
@@ -159,14 +167,14 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
       mbar_init(&sm.q_full[i], 1);
       mbar_init(&sm.q_empty[i], 1);
       mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.p_full[i], 8);  // one arrival per softmax warp
+      mbar_init(&sm.pv_done[i], 1);
     }
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&sm.kv_full[s], 1);
       mbar_init(&sm.kv_empty[s], 1);
     }
-    mbar_init(&sm.p_full, 4);   // one arrival per softmax warp
-    mbar_init(&sm.pv_done, 1);
-    mbar_init(&sm.o_free, 4);
+    mbar_init(&sm.o_free, 8);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     fence_mbar_init();
@@ -254,29 +262,30 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = instr_desc_bf16(128, KT, 0, 0);
       constexpr uint32_t idesc_pv = instr_desc_bf16(128, 128, 0, 1);
-      const uint32_t p_addr = smem_u32(sP);
       int qk = 0, ik = 0;
       int64_t gt = 0;
       bool ok = true;
-      // P V of tile q (its P written by the softmax); `first` starts the
-      // item's O accumulator, after the previous item's epilogue read O out
+      // P V of tile q (its P written to tensor memory by the softmax);
+      // `first` starts the item's O accumulator, after the previous item's
+      // epilogue read O out
       auto issue_pv = [&](int64_t q, bool first) -> bool {
-        if (!tile_wait(&sm.p_full, static_cast<uint32_t>(q & 1), ctx, abort_flag)) return false;
+        if (!tile_wait(&sm.p_full[q & 1], static_cast<uint32_t>((q >> 1) & 1), ctx, abort_flag))
+          return false;
         if (first && ik > 0 && !tile_wait(&sm.o_free, (ik - 1) & 1, ctx, abort_flag)) return false;
         tc_fence_after();
         const int s = static_cast<int>(q % C::kStages);
         const uint32_t v_addr = smem_u32(sKV + s * C::kStageBytes + C::kKBytes);
+        const uint32_t p_tmem = tmem + C::kPCol + static_cast<uint32_t>(q & 1) * (KT / 2);
 #pragma unroll
         for (int kk = 0; kk < KT / 16; ++kk) {
-          // A = P: K-major, no swizzle: 8-key core-matrix columns 2 KB apart
-          // (LBO), 8-row groups 128 B apart (SBO).  B = V: MN-major, 128-byte
-          // swizzle: 16 keys = 2 KB, the two 64-channel halves KT rows apart.
-          const uint64_t ad = smem_desc(p_addr + kk * 4096, 2048, 128, 0);
+          // A = P in tensor memory: 16 keys = 8 columns of bf16 pairs.  B = V:
+          // MN-major, 128-byte swizzle: 16 keys = 2 KB, the two 64-channel
+          // halves KT rows apart.
           const uint64_t bd = smem_desc(v_addr + kk * 2048, KT * 128, 1024, 2);
-          umma_bf16(tmem + C::kOCol, ad, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
+          umma_bf16_ts(tmem + C::kOCol, p_tmem + 8 * kk, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
         }
         umma_commit(&sm.kv_empty[s]);
-        umma_commit(&sm.pv_done);
+        umma_commit(&sm.pv_done[q & 1]);
         return true;
       };
       for (int64_t k = blockIdx.x; ok && k < n_items; k += gridDim.x) {
@@ -290,7 +299,7 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
           if (!(ok = tile_wait(&sm.kv_full[s], (gt / C::kStages) & 1, ctx, abort_flag))) break;
           tc_fence_after();
           // S(gt) overwrites the buffer of S(gt-2), read by the softmax
-          // before it wrote P(gt-2), which P V(gt-2) waited for
+          // before it signalled P(gt-2), which P V(gt-2) waited for
           const uint32_t k_addr = smem_u32(sKV + s * C::kStageBytes);
 #pragma unroll
           for (int kk = 0; kk < 8 * C::KP; ++kk) {
@@ -316,13 +325,17 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
     }
   } else {
     // ------------------------------ softmax ------------------------------
-    const int quad = warp & 3;          // TMEM lane quadrant of this warp
-    const int r = quad * 32 + lane;     // query row of the tile
+    constexpr int H = C::H;               // keys of this warpgroup per tile
+    const int hf = (warp - 2) >> 2;       // warpgroup: keys hf*H .. hf*H+H-1 of a tile
+    const int quad = warp & 3;            // TMEM lane quadrant of this warp
+    const int r = quad * 32 + lane;       // query row of the tile
     const int tok = r / G, h = r % G;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     const float sl2 = args.scale_log2;
-    // P: K-major no-swizzle image, row r's 8-key chunk c at c*2048 + (r/8)*128 + (r%8)*16
-    uint8_t* p_row = sP + (r >> 3) * 128 + (r & 7) * 16;
+    // named barriers over the 256 softmax threads: every decision taken at
+    // one is the same for both warpgroups, so neither leaves a loop while the
+    // other waits at a later barrier
+    constexpr uint32_t bar_sync = 1, bar_or = 2, kSm = 256;
     int64_t gt = 0;
     bool ok = true;
     for (int64_t k = blockIdx.x; ok && k < n_items; k += gridDim.x) {
@@ -335,114 +348,139 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
       if (it.n_kt == 0) {
         // no visible key for any row of the tile (compressed, t < 31)
         if (row_ok) {
-          uint4* o = reinterpret_cast<uint4*>(args.O + orow * kHeadDim);
-          for (int c = 0; c < 16; ++c) o[c] = make_uint4(0, 0, 0, 0);
-          args.lse[lrow] = -INFINITY;
+          uint4* o = reinterpret_cast<uint4*>(args.O + orow * kHeadDim + 64 * hf);
+          for (int c = 0; c < 8; ++c) o[c] = make_uint4(0, 0, 0, 0);
+          if (hf == 0) args.lse[lrow] = -INFINITY;
         }
         continue;
       }
-      const int v_row = MODE == kTileCompressed ? min(args.n_c, visible_windows(t)) : 0;
+      // the last key (or, compressed, window count) this row may see
+      const int lim = MODE == kTileCompressed ? min(args.n_c, visible_windows(t)) : t + 1;
       float m = -INFINITY, l = 0.f;
       for (int i = 0; i < it.n_kt; ++i, ++gt) {
-        ok = __all_sync(0xffffffffu, tile_wait(&sm.s_full[gt & 1], (gt >> 1) & 1, ctx, abort_flag));
-        if (!ok) break;
-        tc_fence_after();
-        float x[KT];
-#pragma unroll
-        for (int c = 0; c < KT / 32; ++c)
-          tmem_ld32(lane_addr + static_cast<uint32_t>(gt & 1) * KT + 32 * c,
-                    *reinterpret_cast<float(*)[32]>(x + 32 * c));
-        tmem_ld_wait();
-        // the row's keys in this tile, masked and scaled to log2 units
-        uint32_t sel[2] = {1u, 1u};
-        int kbase[2] = {i * KT, i * KT + 64};
+        const bool s_ok =
+            __all_sync(0xffffffffu, tile_wait(&sm.s_full[gt & 1], (gt >> 1) & 1, ctx, abort_flag));
+        // this half's keys: [lo, lo + H) of one block (dense, union) or
+        // window range (compressed); sel: the row's token selected them
+        int lo;
+        bool sel = true;
         if (MODE == kTileUnion) {
-          const uint32_t* L = args.ulist + it.list * args.ustride;
-          const uint32_t e0 = __ldg(L + 2 * i);
-          const uint32_t e1 = 2 * i + 1 < it.n_u ? __ldg(L + 2 * i + 1) : 0u;
-          sel[0] = (e0 >> (16 + tok)) & 1u;
-          sel[1] = (e1 >> (16 + tok)) & 1u;
-          kbase[0] = static_cast<int>(e0 & 0xFFFFu) * kBlock;
-          kbase[1] = static_cast<int>(e1 & 0xFFFFu) * kBlock;
+          const uint32_t e = 2 * i + hf < it.n_u
+                                 ? __ldg(args.ulist + it.list * args.ustride + 2 * i + hf)
+                                 : 0u;
+          sel = ((e >> (16 + tok)) & 1u) != 0u;
+          lo = static_cast<int>(e & 0xFFFFu) * kBlock;
+        } else {
+          lo = i * KT + hf * H;
         }
+        // none: no key of the half visible to the row; full: every key is
+        const bool none = !(row_ok && sel && lo < lim) || !s_ok;
+        const bool full = !none && lo + H <= lim;
+        float x[H];
         float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < KT; ++c) {
-          bool valid;
-          if (MODE == kTileCompressed) {
-            valid = i * KT + c < v_row;
-          } else {
-            const int e = c >> 6;
-            valid = sel[e] != 0u && kbase[e] + (c & 63) <= t;
-          }
-          valid = valid && row_ok;
-          x[c] = valid ? x[c] * sl2 : -INFINITY;
-          mx = fmaxf(mx, x[c]);
-        }
-        float alpha = 1.f;
-        if (mx > m + kTileSlack) {
-          alpha = fast_exp2(m - mx);  // 0 while the row had no key
-          m = mx;
-        }
-        float psum = 0.f;
-        uint32_t pk[KT / 2];
-#pragma unroll
-        for (int c = 0; c < KT; c += 2) {
-          const float p0 = fast_exp2(x[c] - m);       // exp2(-inf) = 0 for masked keys
-          const float p1 = fast_exp2(x[c + 1] - m);
-          psum += p0 + p1;
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-          pk[c >> 1] = *reinterpret_cast<uint32_t*>(&b2);
-        }
-        if (m == -INFINITY) {  // no key of the row so far: nothing to add
-          psum = 0.f;
-#pragma unroll
-          for (int c = 0; c < KT / 2; ++c) pk[c] = 0u;
-        }
-        l = l * alpha + psum;
-        // P and O are free once P V of the previous tile has completed
-        if (i > 0) {
-          ok = __all_sync(0xffffffffu,
-                          tile_wait(&sm.pv_done, static_cast<uint32_t>((gt - 1) & 1), ctx, abort_flag));
-          if (!ok) break;
+        if (s_ok && __any_sync(0xffffffffu, !none)) {
           tc_fence_after();
-          if (__any_sync(0xffffffffu, alpha != 1.f)) {
-            // move this row's accumulator to the new reference maximum
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+          for (int c = 0; c < H / 32; ++c)
+            tmem_ld32(lane_addr + static_cast<uint32_t>(gt & 1) * KT + hf * H + 32 * c,
+                      *reinterpret_cast<float(*)[32]>(x + 32 * c));
+          tmem_ld_wait();
+          if (!full) {
+#pragma unroll
+            for (int c = 0; c < H; ++c)
+              if (none || lo + c >= lim) x[c] = -INFINITY;
+          }
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int c = 0; c < H; ++c) m4[c & 3] = fmaxf(m4[c & 3], x[c]);
+          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+        }
+        // the row's reference maximum, common to both halves
+        float alpha = 1.f;
+        const bool ab = !s_ok || *abort_flag != 0;
+        if (named_bar_or(bar_or, kSm, mx > m + kTileSlack || ab)) {
+          if (named_bar_or(bar_or, kSm, ab)) {
+            ok = false;
+            break;
+          }
+          sm.xch[gt & 1][hf][r] = mx;
+          named_bar_sync(bar_sync, kSm);
+          const float rm = fmaxf(mx, sm.xch[gt & 1][hf ^ 1][r]);
+          if (rm > m + kTileSlack) {
+            alpha = fast_exp2(m - rm);  // 0 while the row had no key
+            m = rm;
+          }
+        }
+        // P(gt) reuses the buffer of P(gt-2): P V(gt-2) must have read it
+        bool w_ok = true;
+        if (gt >= 2)
+          w_ok = __all_sync(0xffffffffu, tile_wait(&sm.pv_done[gt & 1],
+                                                   static_cast<uint32_t>(((gt >> 1) & 1) ^ 1), ctx,
+                                                   abort_flag));
+        // P = exp2(s - m) as bf16 pairs into tensor memory, 32 keys at a time
+        const uint32_t pcol = lane_addr + C::kPCol + static_cast<uint32_t>(gt & 1) * (KT / 2) +
+                              hf * (H / 2);
+        const bool zero = none || m == -INFINITY;
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int q = 0; q < H / 32; ++q) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float p0 = zero ? 0.f : fast_exp2(fmaf(x[32 * q + 2 * c], sl2, -m));
+            const float p1 = zero ? 0.f : fast_exp2(fmaf(x[32 * q + 2 * c + 1], sl2, -m));
+            s4[c & 3] += p0 + p1;  // masked keys: exp2(-inf) = 0
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+            pk[c] = *reinterpret_cast<uint32_t*>(&b2);
+          }
+          if (w_ok) tmem_st16(pcol + 16 * q, pk);
+        }
+        l = l * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+        // move the O accumulator (this half's 64 channels) to the new
+        // reference, once P V of the previous tile has added into it
+        if (w_ok && i > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          w_ok = __all_sync(0xffffffffu,
+                            tile_wait(&sm.pv_done[(gt - 1) & 1],
+                                      static_cast<uint32_t>(((gt - 1) >> 1) & 1), ctx, abort_flag));
+          if (w_ok) {
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
               float o[32];
-              tmem_ld32(lane_addr + C::kOCol + 32 * c, o);
+              tmem_ld32(lane_addr + C::kOCol + 64 * hf + 32 * c, o);
               tmem_ld_wait();
 #pragma unroll
               for (int j = 0; j < 32; ++j) o[j] *= alpha;
-              tmem_st32(lane_addr + C::kOCol + 32 * c, o);
+              tmem_st32(lane_addr + C::kOCol + 64 * hf + 32 * c, o);
             }
-            tmem_st_wait();
           }
         }
-#pragma unroll
-        for (int c = 0; c < KT / 8; ++c)
-          *reinterpret_cast<uint4*>(p_row + c * 2048) =
-              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        fence_proxy_async_smem();
+        if (w_ok) tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.p_full);
+        if (lane == 0 && w_ok) mbar_arrive(&sm.p_full[gt & 1]);
       }
       if (!ok) break;
       // ---- epilogue: O / l and the row's log-sum-exp ----
-      ok = __all_sync(0xffffffffu,
-                      tile_wait(&sm.pv_done, static_cast<uint32_t>((gt - 1) & 1), ctx, abort_flag));
-      if (!ok) break;
+      const bool e_ok = __all_sync(0xffffffffu,
+                                   tile_wait(&sm.pv_done[(gt - 1) & 1],
+                                             static_cast<uint32_t>(((gt - 1) >> 1) & 1), ctx,
+                                             abort_flag));
+      sm.xl[hf][r] = l;
+      if (named_bar_or(bar_or, kSm, !e_ok || *abort_flag != 0)) {
+        ok = false;
+        break;
+      }
+      const float L = sm.xl[0][r] + sm.xl[1][r];
+      const float inv = L > 0.f ? 1.f / L : 0.f;
       tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         float o[32];
-        tmem_ld32(lane_addr + C::kOCol + 32 * c, o);
+        tmem_ld32(lane_addr + C::kOCol + 64 * hf + 32 * c, o);
         tmem_ld_wait();
         if (row_ok && INFLLMV2_CHECK(ctx.status, it.b < args.B && it.g < args.Hkv)) {
-          uint4* dst = reinterpret_cast<uint4*>(args.O + orow * kHeadDim + 32 * c);
+          uint4* dst = reinterpret_cast<uint4*>(args.O + orow * kHeadDim + 64 * hf + 32 * c);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             uint32_t w[4];
@@ -456,7 +494,7 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
           }
         }
       }
-      if (row_ok) args.lse[lrow] = l > 0.f ? (m + __log2f(l)) * kLn2f : -INFINITY;
+      if (row_ok && hf == 0) args.lse[lrow] = L > 0.f ? (m + __log2f(L)) * kLn2f : -INFINITY;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.o_free);
@@ -575,8 +613,7 @@ int launch_tile_g(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMa
                   const TileArgs& a, const DevCtx& ctx, cudaStream_t st) {
   using C = TileCfg<MODE>;
   constexpr int TPT = 128 / G;
-  const size_t smem = 1024 + 2 * C::kQBytes + C::kStages * C::kStageBytes + C::kPBytes +
-                      sizeof(TileSmem);
+  const size_t smem = 1024 + 2 * C::kQBytes + C::kStages * C::kStageBytes + sizeof(TileSmem);
   static std::atomic<uint64_t> smem_set{0};
   if (int e = set_smem_limit(tile_attn_kernel<G, MODE>, smem, smem_set)) return e;
   const int64_t n_items = static_cast<int64_t>(a.B) * a.Hkv * ((a.Tq + TPT - 1) / TPT);
