@@ -258,7 +258,7 @@ def run_prefill(api, wl, w, steps, warmup, dist, flush, time_e2e=True, clocks=No
     idx_np = idx.cpu().numpy()
     cur = (np.arange(T) // 64)[None, None, :, None]
     valid = (idx_np >= 0) & (idx_np <= cur)
-    if G >= 8:
+    if G >= 4:
         # query-tile schedule: each tile of 128/G tokens loads the union of its
         # tokens' blocks once (K and V, 32 KB per block) and runs 128-key
         # tiles of 128 rows (S and P V, 2 FLOP per MAC)

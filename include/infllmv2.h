@@ -94,7 +94,7 @@ typedef struct infllmv2_params {
 #define INFLLMV2_OP_SELECT   1
 #define INFLLMV2_OP_FORWARD  2
 #define INFLLMV2_OP_DECODE   3
-#define INFLLMV2_OP_ATTN     4  /* sparse_attn: union lists (groups of 8 or 16 heads) or packed K/V */
+#define INFLLMV2_OP_ATTN     4  /* sparse_attn: union lists (groups of 4+ heads) or packed K/V */
 #define INFLLMV2_OP_ATTN_PER_TOKEN 5  /* sparse_attn_per_token: packed K and V */
 #define INFLLMV2_OP_FORWARD_FP32   6  /* forward_fp32: block scores (0 when dense) */
 
@@ -145,7 +145,7 @@ int infllmv2_select_blocks(const infllmv2_params* p, const void* Q, const void* 
  *   lse[b,h,t] = log sum_{i in keys(t)} exp(scale * q.K_i).
  *   idx rows must be ascending with valid entries first (as select_blocks
  *   writes them); entries > t/64 are ignored.
- * Schedule: with Hq/Hkv in {8, 16} and ws of at least
+ * Schedule: with Hq/Hkv in {4, 8, 16} and ws of at least
  * infllmv2_workspace_bytes(p, INFLLMV2_OP_ATTN) bytes, query tiles of 128
  * rows (128/G tokens x G heads) run over the union of their tokens' selected
  * blocks, each row masked to its own token's blocks, so a block that several

@@ -58,10 +58,11 @@ def test_host_helpers(lib):
 
 def _union_bytes(B, T, Hkv, G, topk):
     """Union lists of the query-tile schedule: per tile of 128/G tokens, room
-    for every token's topk entries (256-byte aligned), then one count per tile."""
+    for every token's topk (block, token mask) entries of 8 bytes (256-byte
+    aligned), then one count per tile."""
     tpt = 128 // G
     tiles = B * Hkv * (-(-T // tpt))
-    return (-(-(tiles * tpt * topk * 4) // 256) * 256) + tiles * 4
+    return (-(-(tiles * tpt * topk * 8) // 256) * 256) + tiles * 4
 
 
 def _packed_bytes(B, T, Hkv):
@@ -77,9 +78,12 @@ def test_workspace_sizes(lib):
     # groups of 16 heads: the query-tile schedule's union lists
     assert api.workspace_bytes(p, api.OP_ATTN) == _union_bytes(1, T, 2, 16, 64)
     assert api.workspace_bytes(p, api.OP_ATTN_PER_TOKEN) == _packed_bytes(1, T, 2)
-    # smaller groups: the per-token schedule's packed K/V tiles
+    # groups of 4 heads: 32-token query tiles
     p4 = api.make_params(1, 2048, 8, 2, topk=8)
-    assert api.workspace_bytes(p4, api.OP_ATTN) == _packed_bytes(1, 2048, 2)
+    assert api.workspace_bytes(p4, api.OP_ATTN) == _union_bytes(1, 2048, 2, 4, 8)
+    # smaller groups: the per-token schedule's packed K/V tiles
+    p2 = api.make_params(1, 2048, 4, 2, topk=8)
+    assert api.workspace_bytes(p2, api.OP_ATTN) == _packed_bytes(1, 2048, 2)
     p8 = api.make_params(1, 2000, 16, 2, topk=8)
     assert api.workspace_bytes(p8, api.OP_ATTN) == _union_bytes(1, 2000, 2, 8, 8)
     # the dense forward needs no workspace

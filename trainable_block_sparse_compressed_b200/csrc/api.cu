@@ -135,7 +135,7 @@ int check_select_size(const Geometry& g) {
 }
 
 // Workspace of the block-sparse attention: the union lists of the query-tile
-// schedule (groups of 8 or 16 heads), else the packed K/V tiles of the
+// schedule (groups of 4, 8 or 16 heads), else the packed K/V tiles of the
 // per-token schedule.
 size_t attn_ws_bytes(const Geometry& g) {
   return union_supported(g) ? union_ws_bytes(g) : packed_kv_bytes(g);

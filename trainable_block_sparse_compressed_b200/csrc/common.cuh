@@ -134,6 +134,10 @@ int launch_sparse_attn(const Geometry& g, const void* Q, const void* K, const vo
 // selected blocks, or the compressed windows.
 bool union_supported(const Geometry& g);
 size_t union_ws_bytes(const Geometry& g);
+// Union lists of the query tiles of g (in ws, union_ws_bytes(g) bytes):
+// per tile, `stride` slots of (block, token mask) ascending, and the counts.
+int launch_union_build(const Geometry& g, const int32_t* idx, void* ws, const uint2** ulist,
+                       const int32_t** ucount, int* stride, cudaStream_t st);
 int launch_dense_tile(const Geometry& g, const void* Q, const void* K, const void* V, void* O,
                       float* lse, const DevCtx& ctx, cudaStream_t st);
 int launch_union_tile(const Geometry& g, const void* Q, const void* K, const void* V,

@@ -46,11 +46,12 @@ namespace infllmv2 {
 
 constexpr int kTileDense = 0, kTileUnion = 1, kTileCompressed = 2;
 
-// Union lists (tile_attn.cu and its builder): entry = block | token mask << 16.
+// Union lists (tile_attn.cu and its builder): entry = (block, mask of the
+// tile's tokens that selected it).
 struct TileArgs {
   __nv_bfloat16* O;         // [B, Tq, Hq, 128]
   float* lse;               // [B, Hq, Tq]
-  const uint32_t* ulist;    // union: per query tile, its blocks ascending
+  const uint2* ulist;       // union: per query tile, its blocks ascending
   const int32_t* ucount;    // union: entries per query tile
   int ustride;              // union: list capacity per query tile
   int B, Hq, Hkv, q0, Tq;   // queries are tokens q0 .. q0+Tq-1
@@ -233,10 +234,10 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
               blk[1] = 2 * i + 1;
               nblk = blk[1] * kBlock <= it.t_last ? 2 : 1;
             } else {
-              const uint32_t* L = args.ulist + it.list * args.ustride;
-              blk[0] = static_cast<int>(__ldg(L + 2 * i) & 0xFFFFu);
+              const uint2* L = args.ulist + it.list * args.ustride;
+              blk[0] = static_cast<int>(__ldg(L + 2 * i).x);
               nblk = 2 * i + 1 < it.n_u ? 2 : 1;
-              blk[1] = nblk == 2 ? static_cast<int>(__ldg(L + 2 * i + 1) & 0xFFFFu) : 0;
+              blk[1] = nblk == 2 ? static_cast<int>(__ldg(L + 2 * i + 1).x) : 0;
             }
             mbar_arrive_expect_tx(full, nblk * 4 * C::kBox);
             for (int e = 0; e < nblk; ++e) {
@@ -365,11 +366,11 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
         int lo;
         bool sel = true;
         if (MODE == kTileUnion) {
-          const uint32_t e = 2 * i + hf < it.n_u
-                                 ? __ldg(args.ulist + it.list * args.ustride + 2 * i + hf)
-                                 : 0u;
-          sel = ((e >> (16 + tok)) & 1u) != 0u;
-          lo = static_cast<int>(e & 0xFFFFu) * kBlock;
+          const uint2 e = 2 * i + hf < it.n_u
+                              ? __ldg(args.ulist + it.list * args.ustride + 2 * i + hf)
+                              : make_uint2(0u, 0u);
+          sel = ((e.y >> tok) & 1u) != 0u;
+          lo = static_cast<int>(e.x) * kBlock;
         } else {
           lo = i * KT + hf * H;
         }
@@ -516,11 +517,12 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
 // sorted (bitonic, in shared memory), equal blocks merged.
 // ---------------------------------------------------------------------------
 constexpr int kUnionThreads = 256;
+constexpr int kUnionPer = 32;  // sorted keys per thread when merging (cap <= 8192)
 
 template <int TPT>
 __global__ void __launch_bounds__(kUnionThreads) union_build_kernel(
-    const int32_t* __restrict__ idx, uint32_t* __restrict__ ulist, int32_t* __restrict__ ucount,
-    int Hkv, int q0, int Tq, int topk, int n_qt, int cap) {
+    const int32_t* __restrict__ idx, uint2* __restrict__ ulist, int32_t* __restrict__ ucount,
+    int q0, int Tq, int topk, int n_qt, int cap) {
   extern __shared__ uint32_t keys[];  // cap entries (a power of two)
   __shared__ int scan[kUnionThreads / 32 + 1];
   const int64_t tile = blockIdx.x;
@@ -535,7 +537,8 @@ __global__ void __launch_bounds__(kUnionThreads) union_build_kernel(
       if (qtok < Tq) {
         const int v = __ldg(idx + ((bg * Tq + qtok) * topk + j));
         const int t = q0 + qtok;
-        if (v >= 0 && v <= t / kBlock) key = (static_cast<uint32_t>(v) << 4) | static_cast<uint32_t>(tk);
+        if (v >= 0 && v <= t / kBlock)
+          key = (static_cast<uint32_t>(v) << 5) | static_cast<uint32_t>(tk);
       }
     }
     keys[e] = key;
@@ -557,20 +560,19 @@ __global__ void __launch_bounds__(kUnionThreads) union_build_kernel(
     }
   }
   // merge equal blocks: the first key of each block emits (block, token mask)
-  constexpr int PER = 16;  // keys per thread (cap <= 4096)
-  const int base = threadIdx.x * PER;
-  uint32_t ent[PER];
+  const int base = threadIdx.x * kUnionPer;
+  uint2 ent[kUnionPer];
   int nh = 0;
 #pragma unroll
-  for (int s = 0; s < PER; ++s) {
+  for (int s = 0; s < kUnionPer; ++s) {
     const int p = base + s;
-    ent[s] = 0xFFFFFFFFu;
-    if (p < cap && keys[p] != 0xFFFFFFFFu && (p == 0 || (keys[p] >> 4) != (keys[p - 1] >> 4))) {
-      const uint32_t blk = keys[p] >> 4;
+    ent[s] = make_uint2(0xFFFFFFFFu, 0u);
+    if (p < cap && keys[p] != 0xFFFFFFFFu && (p == 0 || (keys[p] >> 5) != (keys[p - 1] >> 5))) {
+      const uint32_t blk = keys[p] >> 5;
       uint32_t mask = 0u;
-      for (int q = p; q < cap && (keys[q] >> 4) == blk && keys[q] != 0xFFFFFFFFu; ++q)
-        mask |= 1u << (keys[q] & 15u);
-      ent[s] = blk | (mask << 16);
+      for (int q = p; q < cap && keys[q] != 0xFFFFFFFFu && (keys[q] >> 5) == blk; ++q)
+        mask |= 1u << (keys[q] & 31u);
+      ent[s] = make_uint2(blk, mask);
       ++nh;
     }
   }
@@ -595,10 +597,10 @@ __global__ void __launch_bounds__(kUnionThreads) union_build_kernel(
   }
   __syncthreads();
   int pos = scan[wid] + x - nh;
-  uint32_t* L = ulist + tile * static_cast<int64_t>(n);
+  uint2* L = ulist + tile * static_cast<int64_t>(n);
 #pragma unroll
-  for (int s = 0; s < PER; ++s)
-    if (ent[s] != 0xFFFFFFFFu) L[pos++] = ent[s];
+  for (int s = 0; s < kUnionPer; ++s)
+    if (ent[s].x != 0xFFFFFFFFu) L[pos++] = ent[s];
   if (threadIdx.x == 0) ucount[tile] = scan[kUnionThreads / 32];
 }
 
@@ -627,15 +629,15 @@ template <int MODE>
 int launch_tile(const Geometry& g, const CUtensorMap& tq, const CUtensorMap& tk,
                 const CUtensorMap& tv, const TileArgs& a, const DevCtx& ctx, cudaStream_t st) {
   switch (g.G) {
+    case 4: return launch_tile_g<4, MODE>(tq, tk, tv, a, ctx, st);
     case 8: return launch_tile_g<8, MODE>(tq, tk, tv, a, ctx, st);
     case 16: return launch_tile_g<16, MODE>(tq, tk, tv, a, ctx, st);
     default: break;
   }
-  if constexpr (MODE != kTileUnion) {  // the union lists' token masks hold 16 tokens
+  if constexpr (MODE != kTileUnion) {  // the union lists' token masks hold 32 tokens
     switch (g.G) {
       case 1: return launch_tile_g<1, MODE>(tq, tk, tv, a, ctx, st);
       case 2: return launch_tile_g<2, MODE>(tq, tk, tv, a, ctx, st);
-      case 4: return launch_tile_g<4, MODE>(tq, tk, tv, a, ctx, st);
       default: break;
     }
   }
@@ -680,14 +682,48 @@ TileArgs tile_args(const Geometry& g, void* O, float* lse) {
 
 }  // namespace
 
-bool union_supported(const Geometry& g) { return g.G >= 8; }
+bool union_supported(const Geometry& g) { return g.G >= 4; }
+
+namespace {
+int64_t union_tiles(const Geometry& g) {
+  const int TPT = 128 / g.G;
+  return static_cast<int64_t>(g.B) * g.Hkv * ((g.Tq + TPT - 1) / TPT);
+}
+size_t union_lists_bytes(const Geometry& g) {
+  const size_t b = static_cast<size_t>(union_tiles(g)) * (128 / g.G) * g.topk * sizeof(uint2);
+  return (b + 255) & ~static_cast<size_t>(255);
+}
+}  // namespace
 
 size_t union_ws_bytes(const Geometry& g) {
   if (!union_supported(g) || g.B == 0 || g.Tq == 0) return 0;
+  return union_lists_bytes(g) + static_cast<size_t>(union_tiles(g)) * sizeof(int32_t);
+}
+
+int launch_union_build(const Geometry& g, const int32_t* idx, void* ws, const uint2** ulist,
+                       const int32_t** ucount, int* stride, cudaStream_t st) {
+  if (!union_supported(g)) return INFLLMV2_ERR_UNSUPPORTED;
   const int TPT = 128 / g.G;
-  const int64_t tiles = static_cast<int64_t>(g.B) * g.Hkv * ((g.Tq + TPT - 1) / TPT);
-  const size_t lists = static_cast<size_t>(tiles) * TPT * g.topk * sizeof(uint32_t);
-  return ((lists + 255) & ~static_cast<size_t>(255)) + static_cast<size_t>(tiles) * sizeof(int32_t);
+  const int n_qt = (g.Tq + TPT - 1) / TPT;
+  const int64_t tiles = union_tiles(g);
+  const int n = TPT * g.topk;
+  const int cap = next_pow2(n);
+  if (cap > kUnionPer * kUnionThreads) return INFLLMV2_ERR_UNSUPPORTED;
+  uint2* L = static_cast<uint2*>(ws);
+  int32_t* C = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + union_lists_bytes(g));
+  const size_t ush = static_cast<size_t>(cap) * sizeof(uint32_t);
+  const unsigned grid = static_cast<unsigned>(tiles);
+  if (TPT == 8)
+    union_build_kernel<8><<<grid, kUnionThreads, ush, st>>>(idx, L, C, g.q0, g.Tq, g.topk, n_qt, cap);
+  else if (TPT == 16)
+    union_build_kernel<16><<<grid, kUnionThreads, ush, st>>>(idx, L, C, g.q0, g.Tq, g.topk, n_qt, cap);
+  else
+    union_build_kernel<32><<<grid, kUnionThreads, ush, st>>>(idx, L, C, g.q0, g.Tq, g.topk, n_qt, cap);
+  if (cudaGetLastError() != cudaSuccess) return INFLLMV2_ERR_CUDA;
+  *ulist = L;
+  *ucount = C;
+  *stride = n;
+  return INFLLMV2_OK;
 }
 
 int launch_dense_tile(const Geometry& g, const void* Q, const void* K, const void* V, void* O,
@@ -704,33 +740,12 @@ int launch_union_tile(const Geometry& g, const void* Q, const void* K, const voi
                       const int32_t* idx, void* O, float* lse, void* ws, const DevCtx& ctx,
                       cudaStream_t st) {
   if (g.B == 0 || g.Tq == 0) return INFLLMV2_OK;
-  if (!union_supported(g)) return INFLLMV2_ERR_UNSUPPORTED;
-  const int TPT = 128 / g.G;
-  const int n_qt = (g.Tq + TPT - 1) / TPT;
-  const int64_t tiles = static_cast<int64_t>(g.B) * g.Hkv * n_qt;
-  const int n = TPT * g.topk;
-  const int cap = next_pow2(n);
-  if (cap > 16 * kUnionThreads) return INFLLMV2_ERR_UNSUPPORTED;
-  uint32_t* ulist = static_cast<uint32_t*>(ws);
-  const size_t lists = static_cast<size_t>(tiles) * n * sizeof(uint32_t);
-  int32_t* ucount = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) +
-                                               ((lists + 255) & ~static_cast<size_t>(255)));
-  const size_t ush = static_cast<size_t>(cap) * sizeof(uint32_t);
-  if (TPT == 8)
-    union_build_kernel<8><<<static_cast<unsigned>(tiles), kUnionThreads, ush, st>>>(
-        idx, ulist, ucount, g.Hkv, g.q0, g.Tq, g.topk, n_qt, cap);
-  else
-    union_build_kernel<16><<<static_cast<unsigned>(tiles), kUnionThreads, ush, st>>>(
-        idx, ulist, ucount, g.Hkv, g.q0, g.Tq, g.topk, n_qt, cap);
-  if (cudaGetLastError() != cudaSuccess) return INFLLMV2_ERR_CUDA;
+  TileArgs a = tile_args(g, O, lse);
+  if (int e = launch_union_build(g, idx, ws, &a.ulist, &a.ucount, &a.ustride, st)) return e;
   CUtensorMap tq, tk, tv;
   if (int e = q_map(g, Q, &tq)) return e;
   if (int e = kv_map(g, K, &tk)) return e;
   if (int e = kv_map(g, V, &tv)) return e;
-  TileArgs a = tile_args(g, O, lse);
-  a.ulist = ulist;
-  a.ucount = ucount;
-  a.ustride = n;
   return launch_tile<kTileUnion>(g, tq, tk, tv, a, ctx, st);
 }
 

@@ -193,7 +193,7 @@ def _nbytes(ws) -> int:
 
 def sparse_attn(p: Params, Q, K, V, idx, O, lse, ws=None, stream=None):
     """Block-sparse attention; ws (OP_ATTN bytes) enables the query-tile
-    schedule (groups of 8 or 16 heads) or the packed K/V gather."""
+    schedule (groups of 4, 8 or 16 heads) or the packed K/V gather."""
     _check("infllmv2_sparse_attn",
            load().infllmv2_sparse_attn(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx),
                                        _ptr(O), _ptr(lse), _ptr(ws), _nbytes(ws),
