@@ -97,6 +97,7 @@ typedef struct infllmv2_params {
 #define INFLLMV2_OP_ATTN     4  /* sparse_attn: union lists (groups of 4+ heads) or packed K/V */
 #define INFLLMV2_OP_ATTN_PER_TOKEN 5  /* sparse_attn_per_token: packed K and V */
 #define INFLLMV2_OP_FORWARD_FP32   6  /* forward_fp32: block scores (0 when dense) */
+#define INFLLMV2_OP_BACKWARD       7  /* sparse_attn_backward */
 
 /* Path reported by infllmv2_forward. */
 #define INFLLMV2_PATH_DENSE  1
@@ -171,6 +172,29 @@ int infllmv2_sparse_attn(const infllmv2_params* p, const void* Q, const void* K,
 int infllmv2_sparse_attn_per_token(const infllmv2_params* p, const void* Q, const void* K,
                                    const void* V, const int32_t* idx, void* O, float* lse,
                                    void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Gradients of infllmv2_sparse_attn with the block selection held fixed (the
+ * method is a trainable sparse attention: paper page, Abstract; the selection
+ * is a discrete choice, so training propagates through the attention over the
+ * chosen blocks).  For every query row over keys(t) as in infllmv2_sparse_attn,
+ * with P = softmax(scale q K^T) recomputed from lse and D = rowsum(dO * O):
+ *   dP = dO V^T,  dS = P * (dP - D),
+ *   dQ[row] = scale dS K,  dK += scale dS^T q,  dV += P^T dO,
+ * dK and dV summing over every row that selected a key's block.
+ *   Q, K, V, idx as given to infllmv2_sparse_attn; O, lse its outputs;
+ *   dO [B, T, Hq, d] bf16 (in);
+ *   dQ [B, T, Hq, d], dK, dV [B, T, Hkv, d] fp32 (out);
+ *   ws: at least infllmv2_workspace_bytes(p, INFLLMV2_OP_BACKWARD) bytes.
+ * Built for Hq/Hkv in {4, 8, 16} (other groups: INFLLMV2_ERR_UNSUPPORTED).
+ * dK and dV are summed in a fixed order (the rows of each block ascending),
+ * so repeated calls give identical results.  For the dense path's gradients
+ * pass an idx that lists every block (topk >= number of blocks).
+ */
+int infllmv2_sparse_attn_backward(const infllmv2_params* p, const void* Q, const void* K,
+                                  const void* V, const int32_t* idx, const void* O,
+                                  const float* lse, const void* dO, float* dQ, float* dK,
+                                  float* dV, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Exact dense causal attention (skill write-up, Architecture Overview, the

@@ -261,6 +261,8 @@ size_t infllmv2_workspace_bytes(const infllmv2_params* p, int32_t op) {
       return g.T > INFLLMV2_MAX_DECODE_T ? SIZE_MAX : decode_ws_bytes(g);
     case INFLLMV2_OP_ATTN: return attn_ws_bytes(g);
     case INFLLMV2_OP_ATTN_PER_TOKEN: return packed_kv_bytes(g);
+    case INFLLMV2_OP_BACKWARD:
+      return union_supported(g) && !check_select_size(g) ? bwd_ws_bytes(g) : SIZE_MAX;
     case INFLLMV2_OP_FORWARD_FP32:
       if (dense_fwd) return 0;
       return check_select_size(g) ? SIZE_MAX : select_ws_bytes(g);
@@ -320,6 +322,23 @@ int infllmv2_sparse_attn_per_token(const infllmv2_params* p, const void* Q, cons
   if (int e = ctx_or_error(&ctx)) return e;
   return enqueue_sparse(g, Q, K, V, idx, O, lse, ws, ws_bytes, true, ctx,
                         static_cast<cudaStream_t>(stream));
+}
+
+int infllmv2_sparse_attn_backward(const infllmv2_params* p, const void* Q, const void* K,
+                                  const void* V, const int32_t* idx, const void* O,
+                                  const float* lse, const void* dO, float* dQ, float* dK,
+                                  float* dV, void* ws, size_t ws_bytes, void* stream) {
+  Geometry g;
+  if (int e = validate(p, true, &g)) return e;
+  if (!union_supported(g)) return INFLLMV2_ERR_UNSUPPORTED;
+  if (int e = check_select_size(g)) return e;
+  if (empty(g)) return INFLLMV2_OK;
+  if (int e = check_ptrs({Q, K, V, idx, O, lse, dO, dQ, dK, dV, ws})) return e;
+  if (ws_bytes < bwd_ws_bytes(g)) return INFLLMV2_ERR_WORKSPACE;
+  DevCtx ctx;
+  if (int e = ctx_or_error(&ctx)) return e;
+  return launch_sparse_bwd(g, Q, K, V, idx, O, lse, dO, dQ, dK, dV, ws, ctx,
+                           static_cast<cudaStream_t>(stream));
 }
 
 int infllmv2_dense_attn(const infllmv2_params* p, const void* Q, const void* K, const void* V,

@@ -150,6 +150,11 @@ int launch_compressed_tile(const Geometry& g, const void* Q, const void* Kc, con
 int launch_forward_f32(const Geometry& g, const void* Q, const void* K, const void* V, void* O,
                        float* lse, float* Kc32, int32_t* idx, float* scores, bool dense,
                        cudaStream_t st);
+// Backward of the block-sparse attention with the selection fixed (attn_bwd.cu).
+size_t bwd_ws_bytes(const Geometry& g);
+int launch_sparse_bwd(const Geometry& g, const void* Q, const void* K, const void* V,
+                      const int32_t* idx, const void* O, const float* lse, const void* dO, float* dQ,
+                      float* dK, float* dV, void* ws, const DevCtx& ctx, cudaStream_t st);
 // Decode (decode.cu); g.T is the cache capacity.
 size_t decode_ws_bytes(const Geometry& g);
 int launch_decode_step(const Geometry& g, const void* q, const void* k_new, const void* v_new,

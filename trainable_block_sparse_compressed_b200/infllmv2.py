@@ -27,6 +27,7 @@ ERR_DEVICE_CHECK = -6
 STATUS_TIMEOUT = 0x1
 STATUS_SEQ_FULL = 0x2
 OP_SELECT, OP_FORWARD, OP_DECODE, OP_ATTN, OP_ATTN_PER_TOKEN, OP_FORWARD_FP32 = 1, 2, 3, 4, 5, 6
+OP_BACKWARD = 7
 PATH_DENSE, PATH_SPARSE = 1, 2
 
 # every symbol include/infllmv2.h declares
@@ -39,6 +40,7 @@ EXPORTS = (
     "infllmv2_prefill_chunk_workspace_bytes", "infllmv2_gather_peak",
     "infllmv2_sparse_attn_per_token", "infllmv2_compressed_attn", "infllmv2_forward_fp32",
     "infllmv2_prefill_varlen", "infllmv2_prefill_varlen_workspace_bytes",
+    "infllmv2_sparse_attn_backward",
 )
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
@@ -89,6 +91,7 @@ def load(path: Optional[str] = None):
         "infllmv2_sparse_attn_per_token": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "infllmv2_dense_attn": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, sz, vp]),
         "infllmv2_compressed_attn": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp]),
+        "infllmv2_sparse_attn_backward": (ctypes.c_int, [P] + [vp] * 11 + [sz, vp]),
         "infllmv2_forward": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "infllmv2_forward_fp32": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "infllmv2_decode_step": (ctypes.c_int,
@@ -207,6 +210,15 @@ def sparse_attn_per_token(p: Params, Q, K, V, idx, O, lse, ws=None, stream=None)
            load().infllmv2_sparse_attn_per_token(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V),
                                                  _ptr(idx), _ptr(O), _ptr(lse), _ptr(ws),
                                                  _nbytes(ws), _stream(stream)))
+
+
+def sparse_attn_backward(p: Params, Q, K, V, idx, O, lse, dO, dQ, dK, dV, ws, stream=None):
+    """Gradients (fp32 dQ, dK, dV) of sparse_attn with the selection idx fixed."""
+    _check("infllmv2_sparse_attn_backward",
+           load().infllmv2_sparse_attn_backward(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V),
+                                                _ptr(idx), _ptr(O), _ptr(lse), _ptr(dO), _ptr(dQ),
+                                                _ptr(dK), _ptr(dV), _ptr(ws), _nbytes(ws),
+                                                _stream(stream)))
 
 
 def compressed_attn(p: Params, Q, Kc, Vc, O, lse, stream=None):
