@@ -528,6 +528,49 @@ def run_compressed(api, wl, w, steps, warmup, flush):
     return dict(ms=sum(ms) / len(ms), attn_ms=sum(ams) / len(ams), tokens=B * T, flops=flops)
 
 
+def run_backward(api, wl, w, steps, warmup, flush):
+    """Gradients of the block-sparse attention with the selection fixed, on a
+    prefill workload: the forward (for O, lse and the selection) once, then
+    the timed backward.  Inputs and dO resident."""
+    import numpy as np
+    import torch
+    data = wl.make_prefill(w)
+    Q, K, V = (wl.to_torch_bf16(data[x]).cuda() for x in "QKV")
+    B, T, Hq, Hkv = w.B, w.T, w.Hq, w.Hkv
+    O, lse, _, idx = api.prefill(Q, K, V, topk=w.topk, n_init=w.n_init, n_local=w.n_local,
+                                 threshold=w.threshold)
+    p = api.make_params(B, T, Hq, Hkv, topk=w.topk, n_init=w.n_init, n_local=w.n_local,
+                        switch_threshold=w.threshold)
+    g = torch.Generator(device="cuda").manual_seed(7)
+    dO = torch.randn(Q.shape, generator=g, device="cuda").to(torch.bfloat16)
+    dQ = torch.empty(Q.shape, dtype=torch.float32, device="cuda")
+    dK = torch.empty(K.shape, dtype=torch.float32, device="cuda")
+    dV = torch.empty_like(dK)
+    ws = api.alloc_workspace(p, api.OP_BACKWARD)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        flush()
+        api.sparse_attn_backward(p, Q, K, V, idx, O, lse, dO, dQ, dK, dV, ws)
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(steps):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        api.sparse_attn_backward(p, Q, K, V, idx, O, lse, dO, dQ, dK, dV, ws)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    assert api.get_status() == 0
+    nkeys = attended_keys(idx.cpu().numpy(), T)
+    G = Hq // Hkv
+    # S, dP, dQ, dK, dV: five products of 2 d FLOP per (row, attended key)
+    flops = float(10 * 128 * G * nkeys.sum())
+    del Q, K, V, O, lse, idx, dO, dQ, dK, dV, ws
+    torch.cuda.empty_cache()
+    return dict(ms=sum(ms) / len(ms), tokens=B * T, flops=flops)
+
+
 def run_dense(api, wl, w, steps, warmup, flush):
     """The dense-switch workload through infllmv2_forward (T <= threshold, so
     the switch takes exact dense causal attention), inputs resident."""
@@ -754,6 +797,14 @@ def main():
             "ms_per_step": d1, "tflops": dn["flops"] / (d1 / 1e3) / 1e12,
             "tensor_frac_of_burst": dn["flops"] / (d1 / 1e3) / 1e12 / peaks["bf16_tflops"],
             "flops_per_step": dn["flops"]}
+        bw = run_backward(api, wl, wl.WORKLOADS[SIDE], args.steps, args.warmup, flush)
+        b1 = dist.max(bw["ms"])
+        extras["backward_T32768"] = {
+            "tokens_per_s": whole_job_rate(bw["tokens"], dist.world, b1), "ms_per_step": b1,
+            "useful_tflops": bw["flops"] / (b1 / 1e3) / 1e12,
+            "tensor_frac_of_burst": bw["flops"] / (b1 / 1e3) / 1e12 / peaks["bf16_tflops"],
+            "timing": "dQ, dK, dV with the forward's selection fixed (delta, dQ, index, dK/dV, "
+                      "reduce); L2 flushed"}
         cm = run_compressed(api, wl, w, args.steps, args.warmup, flush)
         c1 = dist.max(cm["ms"])
         extras["compressed_branch_T131072"] = {

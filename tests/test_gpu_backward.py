@@ -106,8 +106,11 @@ def test_sparse_backward_32k_sampled(cuda_lib):
     """The T=32768 workload with the GPU's own selection: dQ on sampled rows
     against the oracle row by row; dK and dV of the last block and of a
     middle block against the oracle over exactly the rows that selected them;
-    and two identities over all keys (the softmax rows sum to one):
-    sum_keys dV = sum_rows dO and sum_keys dK = 0, per (b, kv head)."""
+    and, over all keys, sum_keys dV = sum_rows dO per (b, kv head) (each
+    softmax row sums to one).  (The companion identity sum_keys dK = 0 holds
+    only in exact arithmetic: D is formed from the bf16 output O, and the
+    per-row residual dO . (O - bf16(O)) random-walks over the 524288 rows to
+    a few tenths, so it is not a check at this size.)"""
     import torch
     api = cuda_lib
     w = wl.WORKLOADS["sparse_prefill_T32768_Hq32_Hkv2"]
@@ -129,7 +132,6 @@ def test_sparse_backward_32k_sampled(cuda_lib):
         hs = slice(g * G, (g + 1) * G)
         sum_dO = dOf[0, :, hs].sum(axis=(0, 1))
         assert np.abs(dV[0, :, g].sum(axis=0) - sum_dO).max() <= G_RTOL * np.abs(sum_dO).max()
-        assert np.abs(dK[0, :, g].sum(axis=0)).max() <= G_RTOL * np.abs(dK[0, :, g]).max()
     # dQ on sampled rows
     for g in range(w.Hkv):
         hs = slice(g * G, (g + 1) * G)
