@@ -358,7 +358,14 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
       // the last key (or, compressed, window count) this row may see
       const int lim = MODE == kTileCompressed ? min(args.n_c, visible_windows(t)) : t + 1;
       float m = -INFINITY, l = 0.f;
+      // union stream: this half's list entry of tile i, loaded one tile ahead
+      // so that its latency overlaps the previous tile
+      const uint2* ul = args.ulist + it.list * args.ustride + hf;
+      uint2 e_next = make_uint2(0u, 0u);
+      if (MODE == kTileUnion && hf < it.n_u) e_next = __ldg(ul);
       for (int i = 0; i < it.n_kt; ++i, ++gt) {
+        uint2 e_cur = e_next;
+        if (MODE == kTileUnion && 2 * (i + 1) + hf < it.n_u) e_next = __ldg(ul + 2 * (i + 1));
         const bool s_ok =
             __all_sync(0xffffffffu, tile_wait(&sm.s_full[gt & 1], (gt >> 1) & 1, ctx, abort_flag));
         // this half's keys: [lo, lo + H) of one block (dense, union) or
@@ -366,11 +373,9 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
         int lo;
         bool sel = true;
         if (MODE == kTileUnion) {
-          const uint2 e = 2 * i + hf < it.n_u
-                              ? __ldg(args.ulist + it.list * args.ustride + 2 * i + hf)
-                              : make_uint2(0u, 0u);
-          sel = ((e.y >> tok) & 1u) != 0u;
-          lo = static_cast<int>(e.x) * kBlock;
+          if (2 * i + hf >= it.n_u) e_cur = make_uint2(0u, 0u);
+          sel = ((e_cur.y >> tok) & 1u) != 0u;
+          lo = static_cast<int>(e_cur.x) * kBlock;
         } else {
           lo = i * KT + hf * H;
         }
