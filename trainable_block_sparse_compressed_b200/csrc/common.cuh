@@ -111,28 +111,6 @@ inline int set_smem_limit(F* func, size_t bytes, std::atomic<uint64_t>& done) {
   return INFLLMV2_OK;
 }
 
-// Launches `kernel` on `st` with programmatic stream serialization: its
-// CTAs may be scheduled while the stream's previous kernel finishes (once
-// every CTA of that kernel has issued griddepcontrol.launch_dependents), and
-// must call grid_dep_wait() before reading anything that kernel writes.
-template <typename... KArgs, typename... Args>
-inline int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                      cudaStream_t st, Args... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) == cudaSuccess
-             ? INFLLMV2_OK
-             : INFLLMV2_ERR_CUDA;
-}
-
 // Tensor maps (tma.cpp).
 int make_tmap_bf16_4d(CUtensorMap* map, const void* base, const uint64_t dims[4],
                       const uint64_t strides_bytes[3], const uint32_t box[4]);

@@ -76,8 +76,6 @@ __global__ void __launch_bounds__(32) decode_append_kernel(
     __nv_bfloat16* __restrict__ Kc_, __nv_bfloat16* __restrict__ Vc_,
     __nv_bfloat16* __restrict__ Kcmp, const int32_t* __restrict__ seqlens,
     int32_t* __restrict__ active, int Hkv, int Lmax, int NC, int* status) {
-  grid_dep_launch();
-  grid_dep_wait();  // seqlens and the caches of the previous step
   const int b = blockIdx.x / Hkv, g = blockIdx.x % Hkv;
   const int tid = threadIdx.x;
   const int pos = seqlens[b];
@@ -189,9 +187,9 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_score_kernel(
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   DScoreSmem& sm = *reinterpret_cast<DScoreSmem*>(base + kDStages * kDStageBytes);
   __shared__ int32_t s_seq[256];
-  grid_dep_launch();
   const int warp = warp_id(), lane = lane_id();
   const int64_t n_units = static_cast<int64_t>(B) * Hkv * n_tpb;
+  for (int i = threadIdx.x; i < B && i < 256; i += blockDim.x) s_seq[i] = seqlens[i];
   const int32_t* seq = B <= 256 ? s_seq : seqlens;
 
   // query rows past G stay zero (padding columns of the product)
@@ -216,8 +214,6 @@ __global__ void __launch_bounds__(kDThreads, 1) decode_score_kernel(
     tmem_alloc(&sm.tmem_base, kDAcc * 16);
     tmem_relinquish();
   }
-  grid_dep_wait();  // the appended compressed keys and positions
-  for (int i = threadIdx.x; i < B && i < 256; i += blockDim.x) s_seq[i] = seqlens[i];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -394,8 +390,6 @@ __global__ void __launch_bounds__(256) decode_pool_kernel(
   constexpr int kWin = 4 * kPoolBlocks + 4;  // windows 4*blk0-1 .. 4*blk1+3 (clipped)
   __shared__ float S[kWin];
   __shared__ float lse2[G];
-  grid_dep_launch();
-  grid_dep_wait();  // the scores of this step
   const int bg = blockIdx.x / n_pool;
   const int part = blockIdx.x % n_pool;
   const int b = bg / Hkv;
@@ -472,8 +466,6 @@ template <int PER>
 __global__ void __launch_bounds__(256) decode_topk_kernel(
     const float* __restrict__ bs_all, const int32_t* __restrict__ seqlens, int32_t* __restrict__ idx,
     int Hkv, int NB, int Lmax, int topk, int n_init, int n_local) {
-  grid_dep_launch();
-  grid_dep_wait();  // the block scores of this step
   const int bg = blockIdx.x;
   const int t = seqlens[bg / Hkv];
   int32_t* orow = idx + static_cast<int64_t>(bg) * topk;
@@ -500,8 +492,6 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(
     const float* __restrict__ part, const int32_t* __restrict__ active, int32_t* seqlens,
     __nv_bfloat16* __restrict__ O, float* __restrict__ lse, int Hq, int Hkv, int n_chunks,
     int64_t n_items) {
-  grid_dep_launch();
-  grid_dep_wait();  // the attention partials of this step
   const int bg = blockIdx.x / G, h = blockIdx.x % G;
   const int b = bg / Hkv, g = bg % Hkv;
   const int d = threadIdx.x;
@@ -539,15 +529,12 @@ int launch_decode_g(const Geometry& g, const DecodeLayout& L, const void* q, con
   float* part = reinterpret_cast<float*>(ws + L.off_part);
   float* bs = reinterpret_cast<float*>(ws + L.off_bs);
   const int bgn = g.B * g.Hkv;
-  // every kernel of the step is launched with programmatic stream
-  // serialization: its launch and prologue overlap the previous kernel's tail
-  if (int e = launch_pdl(decode_append_kernel, dim3(bgn), dim3(32), 0, st,
-                         static_cast<const __nv_bfloat16*>(k_new),
-                         static_cast<const __nv_bfloat16*>(v_new),
-                         static_cast<__nv_bfloat16*>(Kc_), static_cast<__nv_bfloat16*>(Vc_),
-                         static_cast<__nv_bfloat16*>(Kcmp), static_cast<const int32_t*>(seqlens),
-                         active, g.Hkv, g.T, L.NC, ctx.status))
-    return e;
+  decode_append_kernel<<<bgn, 32, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new),
+      static_cast<__nv_bfloat16*>(Kc_), static_cast<__nv_bfloat16*>(Vc_),
+      static_cast<__nv_bfloat16*>(Kcmp), seqlens, active, g.Hkv, g.T, L.NC,
+      ctx.status);
+  if (cudaGetLastError() != cudaSuccess) return INFLLMV2_ERR_CUDA;
   if (L.NC > 0) {
     CUtensorMap tk, tq;
     {
@@ -573,22 +560,17 @@ int launch_decode_g(const Geometry& g, const DecodeLayout& L, const void* q, con
     if (int e = set_smem_limit(decode_score_kernel<G>, smem, smem_set)) return e;
     const int64_t n_units = static_cast<int64_t>(bgn) * L.n_split;
     const int grid = static_cast<int>(n_units < sm_count() ? n_units : sm_count());
-    if (int e = launch_pdl(decode_score_kernel<G>, dim3(grid), dim3(kDThreads), smem, st, tk, tq,
-                           static_cast<const int32_t*>(seqlens), x, ml, g.B, g.Hkv, L.NC, L.n_split,
-                           g.T, g.scale_log2, ctx))
-      return e;
+    decode_score_kernel<G><<<grid, kDThreads, smem, st>>>(tk, tq, seqlens, x, ml, g.B, g.Hkv, L.NC,
+                                                          L.n_split, g.T, g.scale_log2, ctx);
+    if (cudaGetLastError() != cudaSuccess) return INFLLMV2_ERR_CUDA;
   }
   const int per = select_per(L.NB);
-  if (int e = launch_pdl(decode_pool_kernel<G>, dim3(bgn * L.n_pool), dim3(256), 0, st,
-                         static_cast<const float*>(x), static_cast<const float*>(ml),
-                         static_cast<const int32_t*>(seqlens), bs, g.Hkv, L.NC, L.NB, g.T,
-                         L.n_split, L.n_pool, ctx.status))
-    return e;
-  int sel_rc = INFLLMV2_ERR_UNSUPPORTED;
+  decode_pool_kernel<G><<<bgn * L.n_pool, 256, 0, st>>>(x, ml, seqlens, bs, g.Hkv, L.NC, L.NB, g.T,
+                                                       L.n_split, L.n_pool, ctx.status);
+  if (cudaGetLastError() != cudaSuccess) return INFLLMV2_ERR_CUDA;
 #define INFLLMV2_SEL(V)                                                                     \
-  sel_rc = launch_pdl(decode_topk_kernel<V>, dim3(bgn), dim3(256), 0, st,                    \
-                      static_cast<const float*>(bs), static_cast<const int32_t*>(seqlens), idx, \
-                      g.Hkv, L.NB, g.T, g.topk, g.n_init, g.n_local)
+  decode_topk_kernel<V><<<bgn, 256, 0, st>>>(bs, seqlens, idx, g.Hkv, L.NB, g.T, g.topk, \
+                                             g.n_init, g.n_local)
   switch (per) {
     case 1: INFLLMV2_SEL(1); break;
     case 2: INFLLMV2_SEL(2); break;
@@ -596,17 +578,18 @@ int launch_decode_g(const Geometry& g, const DecodeLayout& L, const void* q, con
     case 8: INFLLMV2_SEL(8); break;
     case 16: INFLLMV2_SEL(16); break;
     case 32: INFLLMV2_SEL(32); break;
-    default: break;
+    default: return INFLLMV2_ERR_UNSUPPORTED;
   }
 #undef INFLLMV2_SEL
-  if (sel_rc) return sel_rc;
+  if (cudaGetLastError() != cudaSuccess) return INFLLMV2_ERR_CUDA;
   if (int e = launch_decode_attn(g, q, Kc_, Vc_, idx, seqlens, part, L.n_chunks, kChunkBlocks, ctx,
                                  st))
     return e;
   const int64_t n_items = static_cast<int64_t>(bgn) * L.n_chunks;
-  return launch_pdl(decode_combine_kernel<G>, dim3(bgn * G), dim3(128), 0, st,
-                    static_cast<const float*>(part), static_cast<const int32_t*>(active), seqlens,
-                    static_cast<__nv_bfloat16*>(O), lse, g.Hq, g.Hkv, L.n_chunks, n_items);
+  decode_combine_kernel<G><<<bgn * G, 128, 0, st>>>(part, active, seqlens,
+                                                static_cast<__nv_bfloat16*>(O), lse, g.Hq, g.Hkv,
+                                                L.n_chunks, n_items);
+  return cudaGetLastError() == cudaSuccess ? INFLLMV2_OK : INFLLMV2_ERR_CUDA;
 }
 
 }  // namespace

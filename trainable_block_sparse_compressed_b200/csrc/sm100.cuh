@@ -319,20 +319,6 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 }
 
 // ---------------------------------------------------------------------------
-// programmatic dependent launch
-// ---------------------------------------------------------------------------
-// Lets the next kernel of the stream, when launched with programmatic stream
-// serialization, be scheduled once every CTA of this grid has issued this.
-__device__ __forceinline__ void grid_dep_launch() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-// Waits until the grids this one depends on have completed and their
-// writes are visible (returns at once when launched without a dependency).
-__device__ __forceinline__ void grid_dep_wait() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-
-// ---------------------------------------------------------------------------
 // math helpers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float fast_exp2(float x) {

@@ -193,7 +193,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const AttnArgs args, DevCtx ctx) {
   extern __shared__ uint8_t smem_raw[];
-  grid_dep_launch();
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint8_t* sKV = base;                                   // kStages x (K 32 KB, V 32 KB)
@@ -247,9 +246,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  // launched with programmatic stream serialization (decode): nothing the
-  // previous kernel writes is read before this point
-  grid_dep_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -630,8 +626,8 @@ int launch_attn_g(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMa
   static std::atomic<uint64_t> smem_set{0};
   if (int e = set_smem_limit(sparse_attn_kernel<G>, smem, smem_set)) return e;
   const int64_t grid = n_items < sm_count() ? n_items : sm_count();
-  return launch_pdl(sparse_attn_kernel<G>, dim3(static_cast<unsigned>(grid)), dim3(kThreads), smem,
-                    st, tq, tk, tv, args, ctx);
+  sparse_attn_kernel<G><<<static_cast<unsigned>(grid), kThreads, smem, st>>>(tq, tk, tv, args, ctx);
+  return cudaGetLastError() == cudaSuccess ? INFLLMV2_OK : INFLLMV2_ERR_CUDA;
 }
 
 int launch_attn(const Geometry& g, const void* Q, int q_tokens, const void* K, const void* V,
