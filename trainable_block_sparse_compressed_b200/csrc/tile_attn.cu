@@ -29,8 +29,9 @@
 //              (K = 2 x 128), Vc its high plane.
 //
 // Warp roles: warp 0 loads Q (double-buffered) and the key tiles (K and V of
-// a tile in one ring stage) by TMA; warp 1 owns tensor memory and one thread
-// issues the MMAs; warps 2-9 are the softmax, two warpgroups on the same 128
+// a tile in one ring stage) by TMA; warp 1 owns tensor memory and one of its
+// threads issues the S products, one thread of warp 10 the P V products;
+// warps 2-9 are the softmax, two warpgroups on the same 128
 // rows (thread = TMEM lane = query row), warpgroup hf taking the tile's keys
 // hf*KT/2 .. (hf+1)*KT/2 - 1 (in the union stream: one selected block each).
 // Each row keeps a reference maximum m, common to its two halves, that moves
@@ -77,7 +78,7 @@ struct TileCfg {
   static constexpr uint32_t kOCol = 2 * KT;
   static constexpr uint32_t kPCol = kOCol + 128;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr int kThreads = 64 + 256;
+  static constexpr int kThreads = 64 + 256 + 32;  // producer, S issuer, softmax x 8, P V issuer
 };
 
 struct TileSmem {
@@ -176,7 +177,7 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
       mbar_init(&sm.kv_empty[s], 1);
     }
     mbar_init(&sm.o_free, 8);
-    mbar_init(&sm.drain, 1);
+    mbar_init(&sm.drain, 2);  // one commit from each MMA issuer
     sm.abort_flag = 0;
     fence_mbar_init();
   }
@@ -258,69 +259,84 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
       for (int64_t q = gt - 1; q >= 0 && q >= gt - C::kStages; --q)
         mbar_wait(&sm.kv_full[q % C::kStages], (q / C::kStages) & 1, ctx.wait_ns);
     }
-  } else if (warp == 1) {
-    // ----------------------------- MMA issuer -----------------------------
+  } else if (warp == 1 || warp == 10) {
+    // ---------------------------- MMA issuers ----------------------------
+    // Issuing a tcgen05.mma holds the issuing thread for about as long as the
+    // tensor core takes to read a 128-wide operand, and a barrier wait costs
+    // a few hundred cycles even when already complete, so one thread issuing
+    // both products of every tile would be the bottleneck.  Warp 1 issues the
+    // S products, warp 10 the P V products, each waiting only for what it
+    // needs:
+    //  - S(gt) needs its K tile and its TMEM buffer, last read by the softmax
+    //    for S(gt-2) before it signalled P(gt-2);
+    //  - P V(gt) needs P(gt) (signalled after S(gt) completed and was read,
+    //    so the K tile is read too: kv_empty after P V covers the whole
+    //    stage) and, first in its item, the previous item's O read out.
     if (lane == 0) {
+      const bool pv_role = warp == 10;
       constexpr uint32_t idesc_s = instr_desc_bf16(128, KT, 0, 0);
       constexpr uint32_t idesc_pv = instr_desc_bf16(128, 128, 0, 1);
       int qk = 0, ik = 0;
       int64_t gt = 0;
       bool ok = true;
-      // P V of tile q (its P written to tensor memory by the softmax);
-      // `first` starts the item's O accumulator, after the previous item's
-      // epilogue read O out
-      auto issue_pv = [&](int64_t q, bool first) -> bool {
-        if (!tile_wait(&sm.p_full[q & 1], static_cast<uint32_t>((q >> 1) & 1), ctx, abort_flag))
-          return false;
-        if (first && ik > 0 && !tile_wait(&sm.o_free, (ik - 1) & 1, ctx, abort_flag)) return false;
-        tc_fence_after();
-        const int s = static_cast<int>(q % C::kStages);
-        const uint32_t v_addr = smem_u32(sKV + s * C::kStageBytes + C::kKBytes);
-        const uint32_t p_tmem = tmem + C::kPCol + static_cast<uint32_t>(q & 1) * (KT / 2);
-#pragma unroll
-        for (int kk = 0; kk < KT / 16; ++kk) {
-          // A = P in tensor memory: 16 keys = 8 columns of bf16 pairs.  B = V:
-          // MN-major, 128-byte swizzle: 16 keys = 2 KB, the two 64-channel
-          // halves KT rows apart.
-          const uint64_t bd = smem_desc(v_addr + kk * 2048, KT * 128, 1024, 2);
-          umma_bf16_ts(tmem + C::kOCol, p_tmem + 8 * kk, bd, idesc_pv, (first && kk == 0) ? 0u : 1u);
-        }
-        umma_commit(&sm.kv_empty[s]);
-        umma_commit(&sm.pv_done[q & 1]);
-        return true;
-      };
       for (int64_t k = blockIdx.x; ok && k < n_items; k += gridDim.x) {
         const TileItem it = tile_item<G, MODE>(k, args, n_qt);
         if (it.n_kt == 0) continue;
-        const int qb = qk & 1;
-        if (!(ok = tile_wait(&sm.q_full[qb], (qk >> 1) & 1, ctx, abort_flag))) break;
-        const uint32_t q_addr = smem_u32(sQ + qb * C::kQBytes);
-        for (int i = 0; ok && i < it.n_kt; ++i, ++gt) {
-          const int s = static_cast<int>(gt % C::kStages);
-          if (!(ok = tile_wait(&sm.kv_full[s], (gt / C::kStages) & 1, ctx, abort_flag))) break;
-          tc_fence_after();
-          // S(gt) overwrites the buffer of S(gt-2), read by the softmax
-          // before it signalled P(gt-2), which P V(gt-2) waited for
-          const uint32_t k_addr = smem_u32(sKV + s * C::kStageBytes);
+        if (pv_role) {
+          for (int i = 0; ok && i < it.n_kt; ++i, ++gt) {
+            if (!(ok = tile_wait(&sm.p_full[gt & 1], static_cast<uint32_t>((gt >> 1) & 1), ctx,
+                                 abort_flag)))
+              break;
+            if (i == 0 && ik > 0 && !(ok = tile_wait(&sm.o_free, (ik - 1) & 1, ctx, abort_flag)))
+              break;
+            tc_fence_after();
+            const int s = static_cast<int>(gt % C::kStages);
+            const uint32_t v_addr = smem_u32(sKV + s * C::kStageBytes + C::kKBytes);
+            const uint32_t p_tmem = tmem + C::kPCol + static_cast<uint32_t>(gt & 1) * (KT / 2);
 #pragma unroll
-          for (int kk = 0; kk < 8 * C::KP; ++kk) {
-            // K-major, 128-byte swizzle: 16 channels = 32 B inside a
-            // 64-channel half; plane p, half h at (2p + h) * KT rows
-            const uint32_t off = ((kk >> 2) & 1) * (KT * 128) + (kk & 3) * 32;
-            const uint64_t qd = smem_desc(q_addr + ((kk >> 2) & 1) * (C::kQBytes / 2) + (kk & 3) * 32,
-                                          16, 1024, 2);
-            const uint64_t kd = smem_desc(k_addr + (kk >> 3) * (2 * KT * 128) + off, 16, 1024, 2);
-            umma_bf16(tmem + static_cast<uint32_t>(gt & 1) * KT, qd, kd, idesc_s, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < KT / 16; ++kk) {
+              // A = P in tensor memory: 16 keys = 8 columns of bf16 pairs.
+              // B = V: MN-major, 128-byte swizzle: 16 keys = 2 KB, the two
+              // 64-channel halves KT rows apart.
+              const uint64_t bd = smem_desc(v_addr + kk * 2048, KT * 128, 1024, 2);
+              umma_bf16_ts(tmem + C::kOCol, p_tmem + 8 * kk, bd, idesc_pv,
+                           (i == 0 && kk == 0) ? 0u : 1u);
+            }
+            umma_commit(&sm.kv_empty[s]);
+            umma_commit(&sm.pv_done[gt & 1]);
           }
-          umma_commit(&sm.s_full[gt & 1]);
-          if (i == it.n_kt - 1) umma_commit(&sm.q_empty[qb]);
-          if (i > 0) ok = issue_pv(gt - 1, i == 1);
+        } else {
+          const int qb = qk & 1;
+          if (!(ok = tile_wait(&sm.q_full[qb], (qk >> 1) & 1, ctx, abort_flag))) break;
+          const uint32_t q_addr = smem_u32(sQ + qb * C::kQBytes);
+          for (int i = 0; ok && i < it.n_kt; ++i, ++gt) {
+            const int s = static_cast<int>(gt % C::kStages);
+            if (!(ok = tile_wait(&sm.kv_full[s], (gt / C::kStages) & 1, ctx, abort_flag))) break;
+            if (gt >= 2 && !(ok = tile_wait(&sm.p_full[gt & 1],
+                                            static_cast<uint32_t>(((gt >> 1) & 1) ^ 1), ctx,
+                                            abort_flag)))
+              break;
+            tc_fence_after();
+            const uint32_t k_addr = smem_u32(sKV + s * C::kStageBytes);
+#pragma unroll
+            for (int kk = 0; kk < 8 * C::KP; ++kk) {
+              // K-major, 128-byte swizzle: 16 channels = 32 B inside a
+              // 64-channel half; plane p, half h at (2p + h) * KT rows
+              const uint32_t off = ((kk >> 2) & 1) * (KT * 128) + (kk & 3) * 32;
+              const uint64_t qd = smem_desc(
+                  q_addr + ((kk >> 2) & 1) * (C::kQBytes / 2) + (kk & 3) * 32, 16, 1024, 2);
+              const uint64_t kd = smem_desc(k_addr + (kk >> 3) * (2 * KT * 128) + off, 16, 1024, 2);
+              umma_bf16(tmem + static_cast<uint32_t>(gt & 1) * KT, qd, kd, idesc_s,
+                        kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&sm.s_full[gt & 1]);
+            if (i == it.n_kt - 1) umma_commit(&sm.q_empty[qb]);
+          }
+          ++qk;
         }
-        if (ok) ok = issue_pv(gt - 1, it.n_kt == 1);
-        ++qk;
         ++ik;
       }
-      // drain: every MMA of this CTA completes before TMEM is released
+      // drain: every MMA of this thread completes before TMEM is released
       umma_commit(&sm.drain);
       mbar_wait(&sm.drain, 0, ctx.wait_ns);
     }
