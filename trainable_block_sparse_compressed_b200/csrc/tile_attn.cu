@@ -66,7 +66,11 @@ template <int MODE>
 struct TileCfg {
   static constexpr int KT = MODE == kTileCompressed ? 64 : 128;  // keys per tile
   static constexpr int KP = MODE == kTileCompressed ? 2 : 1;     // bf16 planes of K
-  static constexpr int kStages = MODE == kTileCompressed ? 3 : 2;
+  // K/V ring depth and query buffers: the 64 KB key tiles of the dense and
+  // union streams take three stages and a single query buffer (a 227 KB
+  // budget); the compressed stream's 48 KB tiles leave room for two
+  static constexpr int kStages = 3;
+  static constexpr int kQBufs = MODE == kTileCompressed ? 2 : 1;
   static constexpr int kBox = 64 * 128;                          // 64 rows x 64 channels
   static constexpr int kKBytes = KP * KT * 256;
   static constexpr int kVBytes = KT * 256;
@@ -88,8 +92,9 @@ struct TileSmem {
   uint64_t o_free, drain;
   uint32_t tmem_base;
   int abort_flag;
-  float xch[2][2][128];  // per tile parity and warpgroup: a row's half maximum
-  float xl[2][128];      // per warpgroup: a row's half sum, at the item's end
+  // per tile parity and warpgroup: a row's half maximum; at an item's end
+  // the parity after its last tile holds the rows' half sums
+  float xch[2][2][128];
 };
 
 constexpr float kTileSlack = 8.0f;   // log2 units
@@ -146,9 +151,15 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
   constexpr int KT = C::KT;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
+  // 128-byte swizzled tiles need 1024-byte alignment; dynamic shared memory
+  // starts on a 1 KB boundary (the launch leaves no slack for more)
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t* sQ = base;                                   // 2 x 32 KB
-  uint8_t* sKV = sQ + 2 * C::kQBytes;                   // stages: K planes, then V
+  if (base != smem_raw) {
+    if (threadIdx.x == 0) report_status(ctx.status, INFLLMV2_STATUS_CHECK);
+    return;
+  }
+  uint8_t* sQ = base;                                   // kQBufs x 32 KB
+  uint8_t* sKV = sQ + C::kQBufs * C::kQBytes;           // stages: K planes, then V
   TileSmem& sm = *reinterpret_cast<TileSmem*>(sKV + C::kStages * C::kStageBytes);
 
   const int warp = warp_id(), lane = lane_id();
@@ -203,8 +214,9 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
       for (int64_t k = blockIdx.x; ok && k < n_items; k += gridDim.x) {
         const TileItem it = tile_item<G, MODE>(k, args, n_qt);
         if (it.n_kt == 0) continue;
-        const int qb = qk & 1;
-        if (qk >= 2 && !(ok = tile_wait(&sm.q_empty[qb], ((qk >> 1) & 1) ^ 1, ctx, abort_flag)))
+        const int qb = qk % C::kQBufs;
+        if (qk >= C::kQBufs &&
+            !(ok = tile_wait(&sm.q_empty[qb], ((qk / C::kQBufs) & 1) ^ 1, ctx, abort_flag)))
           break;
         mbar_arrive_expect_tx(&sm.q_full[qb], C::kQBytes);
         uint8_t* q = sQ + qb * C::kQBytes;
@@ -254,8 +266,8 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
         }
       }
       // drain: never leave with copies of this CTA in flight
-      for (int x = 0; x < 2 && x < qk; ++x)
-        mbar_wait(&sm.q_full[(qk - 1 - x) & 1], ((qk - 1 - x) >> 1) & 1, ctx.wait_ns);
+      for (int x = 0; x < C::kQBufs && x < qk; ++x)
+        mbar_wait(&sm.q_full[(qk - 1 - x) % C::kQBufs], ((qk - 1 - x) / C::kQBufs) & 1, ctx.wait_ns);
       for (int64_t q = gt - 1; q >= 0 && q >= gt - C::kStages; --q)
         mbar_wait(&sm.kv_full[q % C::kStages], (q / C::kStages) & 1, ctx.wait_ns);
     }
@@ -306,8 +318,8 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
             umma_commit(&sm.pv_done[gt & 1]);
           }
         } else {
-          const int qb = qk & 1;
-          if (!(ok = tile_wait(&sm.q_full[qb], (qk >> 1) & 1, ctx, abort_flag))) break;
+          const int qb = qk % C::kQBufs;
+          if (!(ok = tile_wait(&sm.q_full[qb], (qk / C::kQBufs) & 1, ctx, abort_flag))) break;
           const uint32_t q_addr = smem_u32(sQ + qb * C::kQBytes);
           for (int i = 0; ok && i < it.n_kt; ++i, ++gt) {
             const int s = static_cast<int>(gt % C::kStages);
@@ -488,12 +500,12 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
                                    tile_wait(&sm.pv_done[(gt - 1) & 1],
                                              static_cast<uint32_t>(((gt - 1) >> 1) & 1), ctx,
                                              abort_flag));
-      sm.xl[hf][r] = l;
+      sm.xch[gt & 1][hf][r] = l;  // the parity no tile of this item still reads
       if (named_bar_or(bar_or, kSm, !e_ok || *abort_flag != 0)) {
         ok = false;
         break;
       }
-      const float L = sm.xl[0][r] + sm.xl[1][r];
+      const float L = sm.xch[gt & 1][0][r] + sm.xch[gt & 1][1][r];
       const float inv = L > 0.f ? 1.f / L : 0.f;
       tc_fence_after();
 #pragma unroll
@@ -636,7 +648,7 @@ int launch_tile_g(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMa
                   const TileArgs& a, const DevCtx& ctx, cudaStream_t st) {
   using C = TileCfg<MODE>;
   constexpr int TPT = 128 / G;
-  const size_t smem = 1024 + 2 * C::kQBytes + C::kStages * C::kStageBytes + sizeof(TileSmem);
+  const size_t smem = C::kQBufs * C::kQBytes + C::kStages * C::kStageBytes + sizeof(TileSmem);
   static std::atomic<uint64_t> smem_set{0};
   if (int e = set_smem_limit(tile_attn_kernel<G, MODE>, smem, smem_set)) return e;
   const int64_t n_items = static_cast<int64_t>(a.B) * a.Hkv * ((a.Tq + TPT - 1) / TPT);
