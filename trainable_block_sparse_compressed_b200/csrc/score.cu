@@ -48,7 +48,9 @@ constexpr int kStages = 2;
 constexpr int kHalfBytes = kRows * 64 * 2; // one 64-channel half of a 128-row tile
 constexpr int kTileBytes = 2 * kHalfBytes; // 32 KB: the query tile
 constexpr int kKcBytes = 4 * kHalfBytes;   // 64 KB: hi and lo planes of 128 compressed keys
-constexpr int kEpiThreads = 256;          // two epilogue warpgroups, 64 columns each
+constexpr int kEpiWG = 4;                  // epilogue warpgroups
+constexpr int kCW = 128 / kEpiWG;          // accumulator columns per warpgroup
+constexpr int kEpiThreads = 128 * kEpiWG;
 constexpr int kThreads = 64 + kEpiThreads;
 constexpr uint32_t kTmemCols = 256;
 
@@ -62,7 +64,7 @@ struct ScoreSmem {
   uint32_t tmem_base;
   int abort_flag;
   float lse2[kRows];                 // per query row: log2-domain LSE
-  float part_m[kRows], part_l[kRows];  // pass 1: the upper column half's running max / sum
+  float part_m[kEpiWG][kRows], part_l[kEpiWG][kRows];  // pass 1: each column group's max / sum
   float carry[3][4][kRows];          // S of the window just before each 32-lane quadrant
 };
 
@@ -192,23 +194,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&sm.drain, 0, ctx.wait_ns);
     }
   } else {
-    // ---------------- epilogue: 8 warps, thread <-> TMEM lane ----------------
-    // Two warpgroups split the accumulator's 128 columns: warpgroup hf reads
-    // columns 64 hf .. 64 hf + 63 of its lanes.  Pass 1: each keeps a partial
-    // running max / sum of its row over its half, merged at the end of the
-    // pass.  Pass 2: the columns are (token, head) pairs, so warpgroup hf owns
-    // tokens hf TPT/2 .. (hf+1) TPT/2 - 1.  Two warps per scheduler keep the
-    // exp2 / shuffle chains of the epilogue overlapped.
-    constexpr int TPH = TPT / 2;     // tokens per warpgroup in pass 2 (G <= 64)
+    // -------------- epilogue: 16 warps, thread <-> TMEM lane --------------
+    // Four warpgroups split the accumulator's 128 columns: warpgroup hf reads
+    // columns kCW hf .. kCW hf + kCW - 1 of its lanes.  Pass 1: each keeps a
+    // partial running max / sum of its row over its columns, merged at the
+    // end of the pass.  Pass 2: the columns are (token, head) pairs, so
+    // warpgroup hf owns tokens hf TPH .. (hf+1) TPH - 1.  Four warps per
+    // scheduler keep the exp2 / shuffle chains of the epilogue overlapped.
+    constexpr int TPH = TPT / kEpiWG;  // tokens per warpgroup in pass 2 (G <= 32)
     const int hf = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;  // TMEM lane this thread reads
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + hf * 64;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + hf * kCW;
     // the queries' rows of the causally packed workspace, from row q0 on
     const int64_t row0 = score_row_offset(q0);
     const int64_t slab = score_row_offset(q_end) - row0;
     float* srow_base = scores + (static_cast<int64_t>(b) * Hkv + g) * slab;
-    constexpr uint32_t bar_sync_all = 1, bar_or_all = 2;  // 256 threads
+    constexpr uint32_t bar_sync_all = 1, bar_or_all = 2;  // every epilogue thread
     const uint32_t bar_sync_half = 3 + hf;                // the 128 threads of this warpgroup
 
     // pass-1 row identity
@@ -219,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     for (int it = 0; it < n_it; ++it) {
       const int a = it & 1;
-      // all 256 threads take the same decision, so the named barriers below
+      // all epilogue threads take the same decision, so the named barriers below
       // are always reached by every thread that waits at them
       const bool ok = !*abort_flag && mbar_wait(&sm.acc_full[a], (it >> 1) & 1, ctx.wait_ns);
       if (named_bar_or(bar_or_all, kEpiThreads, !ok)) {
@@ -228,9 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      float x[64];
+      float x[kCW];
       tmem_ld32(lane_addr + a * 128, *reinterpret_cast<float(*)[32]>(x));
-      tmem_ld32(lane_addr + a * 128 + 32, *reinterpret_cast<float(*)[32]>(x + 32));
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
@@ -238,36 +239,43 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       if (it < n_t) {
         // ---- pass 1: running max / sum of row r over its visible windows ----
-        const int j0 = it * kKcTile + hf * 64;
-        const int nv = min(64, my_v - j0);  // valid columns of this half (may be <= 0)
-        float tmax = -INFINITY;
+        const int j0 = it * kKcTile + hf * kCW;
+        const int nv = min(kCW, my_v - j0);  // valid columns of this group (may be <= 0)
+        float tm4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c < nv) tmax = fmaxf(tmax, x[c]);
+        for (int c = 0; c < kCW; ++c)
+          if (c < nv) tm4[c & 3] = fmaxf(tm4[c & 3], x[c]);
+        const float tmax = fmaxf(fmaxf(tm4[0], tm4[1]), fmaxf(tm4[2], tm4[3]));
         const float m_new = fmaxf(m_run, tmax);
         if (m_new > -INFINITY) {
           const float mb = m_new * scale_log2;
-          float acc = 0.f;
+          float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (c < nv) acc += fast_exp2(fmaf(x[c], scale_log2, -mb));
-          l_run = l_run * fast_exp2((m_run - m_new) * scale_log2) + acc;
+          for (int c = 0; c < kCW; ++c)
+            if (c < nv) a4[c & 3] += fast_exp2(fmaf(x[c], scale_log2, -mb));
+          l_run = l_run * fast_exp2((m_run - m_new) * scale_log2) + ((a4[0] + a4[1]) + (a4[2] + a4[3]));
           m_run = m_new;
         }
         if (it == n_t - 1) {
-          // merge the two halves of row r
-          if (hf == 1) {
-            sm.part_m[r] = m_run;
-            sm.part_l[r] = l_run;
+          // merge the column groups of row r
+          if (hf > 0) {
+            sm.part_m[hf][r] = m_run;
+            sm.part_l[hf][r] = l_run;
           }
           named_bar_sync(bar_sync_all, kEpiThreads);
           if (hf == 0) {
-            const float m2 = sm.part_m[r], l2 = sm.part_l[r];
-            const float mm = fmaxf(m_run, m2);
+            float mm = m_run;
+#pragma unroll
+            for (int w = 1; w < kEpiWG; ++w) mm = fmaxf(mm, sm.part_m[w][r]);
             float ll = 0.f;
-            if (mm > -INFINITY)
-              ll = (m_run > -INFINITY ? l_run * fast_exp2((m_run - mm) * scale_log2) : 0.f) +
-                   (m2 > -INFINITY ? l2 * fast_exp2((m2 - mm) * scale_log2) : 0.f);
+            if (mm > -INFINITY) {
+              ll = m_run > -INFINITY ? l_run * fast_exp2((m_run - mm) * scale_log2) : 0.f;
+#pragma unroll
+              for (int w = 1; w < kEpiWG; ++w) {
+                const float m2 = sm.part_m[w][r];
+                if (m2 > -INFINITY) ll += sm.part_l[w][r] * fast_exp2((m2 - mm) * scale_log2);
+              }
+            }
             sm.lse2[r] = my_v > 0 ? mm * scale_log2 + __log2f(ll) : INFINITY;
           }
           named_bar_sync(bar_sync_all, kEpiThreads);
@@ -282,11 +290,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int tok = hf * TPH + tl;
           const int t = t0 + tok;
           const int v = t < q_end ? min(n_c, visible_windows(t)) : 0;
-          float acc = 0.f;
+          float a2[2] = {0.f, 0.f};
 #pragma unroll
           for (int h = 0; h < G; ++h)
-            acc += fast_exp2(fmaf(x[tl * G + h], scale_log2, -sm.lse2[tok * G + h]));
-          S[tl] = j < v ? acc : -INFINITY;
+            a2[h & 1] += fast_exp2(fmaf(x[tl * G + h], scale_log2, -sm.lse2[tok * G + h]));
+          S[tl] = j < v ? a2[0] + a2[1] : -INFINITY;
         }
         const int cb = i % 3;
         if (lane == 31) {
@@ -299,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               sm.carry[(i + 1) % 3][0][tok] = S[tl];
           }
         }
-        named_bar_sync(bar_sync_half, kEpiThreads / 2);
+        named_bar_sync(bar_sync_half, 128);
         const int blk = i * (kKcTile / 4) + quad * 8 + (lane >> 2);
 #pragma unroll
         for (int tl = 0; tl < TPH; ++tl) {
