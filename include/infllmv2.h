@@ -151,7 +151,8 @@ int infllmv2_select_blocks(const infllmv2_params* p, const void* Q, const void* 
  * rows (128/G tokens x G heads) run over the union of their tokens' selected
  * blocks, each row masked to its own token's blocks, so a block that several
  * tokens of a tile selected is loaded and multiplied once (ws holds the
- * union lists; contents on return unspecified).  Otherwise (smaller groups, or
+ * union lists and K and V repacked into 16 KB block tiles, each block then
+ * gathered by one bulk copy; contents on return unspecified).  Otherwise (smaller groups, or
  * ws NULL / too small) the call runs infllmv2_sparse_attn_per_token's
  * schedule.  Results agree within rounding.
  */

@@ -56,13 +56,16 @@ def test_host_helpers(lib):
         assert lib.infllmv2_strerror(code)
 
 
-def _union_bytes(B, T, Hkv, G, topk):
-    """Union lists of the query-tile schedule: per tile of 128/G tokens, room
-    for every token's topk (block, token mask) entries of 8 bytes (256-byte
-    aligned), then one count per tile."""
+def _union_bytes(B, Tq, Hkv, G, topk, T=None):
+    """Workspace of the query-tile schedule: per tile of 128/G query tokens,
+    room for every token's topk (block, token mask) entries of 8 bytes, then
+    one count per tile (each part 256-byte aligned), then K and V of all T
+    keys repacked into 16 KB block tiles."""
+    T = Tq if T is None else T
     tpt = 128 // G
-    tiles = B * Hkv * (-(-T // tpt))
-    return (-(-(tiles * tpt * topk * 8) // 256) * 256) + tiles * 4
+    tiles = B * Hkv * (-(-Tq // tpt))
+    up = lambda x: -(-x // 256) * 256  # noqa: E731
+    return up(tiles * tpt * topk * 8) + up(tiles * 4) + _packed_bytes(B, T, Hkv)
 
 
 def _packed_bytes(B, T, Hkv):
@@ -173,12 +176,13 @@ def test_prefill_chunk_workspace_sizes(lib):
     p = api.make_params(1, 131072, 32, 2, topk=64, switch_threshold=8192)
     # the whole sequence as one chunk needs what forward needs
     assert api.prefill_chunk_workspace_bytes(p, 0, 131072) == api.workspace_bytes(p, api.OP_FORWARD)
-    # a tail chunk: the block scores of its rows only, then the union lists of its tiles
+    # a tail chunk: the block scores of its rows only, then the union lists of
+    # its tiles and the packed K/V of every key
     q0, n = 131072 - 4096, 4096
     rows = sum(t // 64 + 1 for t in range(q0, q0 + n))
     sel = 2 * rows * 4
     assert api.prefill_chunk_workspace_bytes(p, q0, n) == \
-        (-(-sel // 256) * 256) + _union_bytes(1, n, 2, 16, 64)
+        (-(-sel // 256) * 256) + _union_bytes(1, n, 2, 16, 64, T=131072)
     d = api.make_params(1, 4096, 32, 2, switch_threshold=8192)
     assert api.prefill_chunk_workspace_bytes(d, 1000, 3096) == 0
 

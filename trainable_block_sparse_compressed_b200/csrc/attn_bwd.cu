@@ -66,7 +66,7 @@ BwdLayout bwd_layout(const Geometry& g) {
   L.off_D = o;
   o = up(o + static_cast<size_t>(g.B) * g.Hq * g.Tq * sizeof(float));
   L.off_union = o;
-  o = up(o + union_ws_bytes(g));
+  o = up(o + union_lists_ws_bytes(g));
   L.off_H = o;
   o = up(o + bg * L.n_ch * L.nb * sizeof(int32_t));
   L.off_cnt = o;

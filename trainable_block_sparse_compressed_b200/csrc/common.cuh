@@ -133,7 +133,8 @@ int launch_sparse_attn(const Geometry& g, const void* Q, const void* K, const vo
 // Query-tile attention (tile_attn.cu): dense causal, the union of the tile's
 // selected blocks, or the compressed windows.
 bool union_supported(const Geometry& g);
-size_t union_ws_bytes(const Geometry& g);
+size_t union_lists_ws_bytes(const Geometry& g);  // the union lists and their counts
+size_t union_ws_bytes(const Geometry& g);        // the lists, then packed K/V tiles
 // Union lists of the query tiles of g (in ws, union_ws_bytes(g) bytes):
 // per tile, `stride` slots of (block, token mask) ascending, and the counts.
 int launch_union_build(const Geometry& g, const int32_t* idx, void* ws, const uint2** ulist,

@@ -55,6 +55,9 @@ struct TileArgs {
   const uint2* ulist;       // union: per query tile, its blocks ascending
   const int32_t* ucount;    // union: entries per query tile
   int ustride;              // union: list capacity per query tile
+  const uint8_t* Kp;        // union: K and V repacked into 16 KB block tiles (pack.cu)
+  const uint8_t* Vp;
+  int nb;                   // union: blocks per (batch, kv head) of the tiles
   int B, Hq, Hkv, q0, Tq;   // queries are tokens q0 .. q0+Tq-1
   int n_c;                  // compressed: windows in Kc / Vc
   float scale_log2;
@@ -223,6 +226,12 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
         tma_load_4d(q, &tmQ, &sm.q_full[qb], 0, it.g * G, it.qtok0, it.b);
         tma_load_4d(q + C::kQBytes / 2, &tmQ, &sm.q_full[qb], 64, it.g * G, it.qtok0, it.b);
         ++qk;
+        uint2 ent[2] = {make_uint2(0u, 0u), make_uint2(0u, 0u)};  // union entries of tile i
+        if (MODE == kTileUnion) {
+          const uint2* L = args.ulist + it.list * args.ustride;
+          ent[0] = __ldg(L);
+          if (it.n_u > 1) ent[1] = __ldg(L + 1);
+        }
         for (int i = 0; i < it.n_kt; ++i, ++gt) {
           const int s = static_cast<int>(gt % C::kStages);
           if (gt >= C::kStages &&
@@ -247,19 +256,30 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
               blk[1] = 2 * i + 1;
               nblk = blk[1] * kBlock <= it.t_last ? 2 : 1;
             } else {
-              const uint2* L = args.ulist + it.list * args.ustride;
-              blk[0] = static_cast<int>(__ldg(L + 2 * i).x);
+              blk[0] = static_cast<int>(ent[0].x);
               nblk = 2 * i + 1 < it.n_u ? 2 : 1;
-              blk[1] = nblk == 2 ? static_cast<int>(__ldg(L + 2 * i + 1).x) : 0;
+              blk[1] = nblk == 2 ? static_cast<int>(ent[1].x) : 0;
+              // the next tile's entries, loaded while this tile's copies fly
+              const uint2* L = args.ulist + it.list * args.ustride;
+              if (2 * i + 2 < it.n_u) ent[0] = __ldg(L + 2 * i + 2);
+              if (2 * i + 3 < it.n_u) ent[1] = __ldg(L + 2 * i + 3);
             }
             mbar_arrive_expect_tx(full, nblk * 4 * C::kBox);
             for (int e = 0; e < nblk; ++e) {
-              // half h of block e at h * (KT rows) + e * 64 rows
-              for (int h = 0; h < 2; ++h) {
-                tma_load_4d(stK + h * KT * 128 + e * C::kBox, &tmK, full, 64 * h, it.g,
-                            blk[e] * kBlock, it.b);
-                tma_load_4d(stV + h * KT * 128 + e * C::kBox, &tmV, full, 64 * h, it.g,
-                            blk[e] * kBlock, it.b);
+              if (MODE == kTileUnion) {
+                // one 16 KB bulk copy per block and tensor from the packed
+                // tiles (no-swizzle canonical image; block e at e * 16 KB)
+                const int64_t tile = (static_cast<int64_t>(it.b) * args.Hkv + it.g) * args.nb + blk[e];
+                bulk_load(stK + e * 16384, args.Kp + tile * 16384, 16384, full);
+                bulk_load(stV + e * 16384, args.Vp + tile * 16384, 16384, full);
+              } else {
+                // 128-byte swizzled boxes: half h of block e at h * (KT rows) + e * 64 rows
+                for (int h = 0; h < 2; ++h) {
+                  tma_load_4d(stK + h * KT * 128 + e * C::kBox, &tmK, full, 64 * h, it.g,
+                              blk[e] * kBlock, it.b);
+                  tma_load_4d(stV + h * KT * 128 + e * C::kBox, &tmV, full, 64 * h, it.g,
+                              blk[e] * kBlock, it.b);
+                }
               }
             }
           }
@@ -310,7 +330,11 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
               // A = P in tensor memory: 16 keys = 8 columns of bf16 pairs.
               // B = V: MN-major, 128-byte swizzle: 16 keys = 2 KB, the two
               // 64-channel halves KT rows apart.
-              const uint64_t bd = smem_desc(v_addr + kk * 2048, KT * 128, 1024, 2);
+              // (union: packed tiles, MN-major no swizzle: 8-key groups 2 KB
+              // apart, 8-channel groups 128 B apart, 16 keys = 4 KB)
+              const uint64_t bd = MODE == kTileUnion
+                                      ? smem_desc(v_addr + kk * 4096, 2048, 128, 0)
+                                      : smem_desc(v_addr + kk * 2048, KT * 128, 1024, 2);
               umma_bf16_ts(tmem + C::kOCol, p_tmem + 8 * kk, bd, idesc_pv,
                            (i == 0 && kk == 0) ? 0u : 1u);
             }
@@ -337,7 +361,12 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
               const uint32_t off = ((kk >> 2) & 1) * (KT * 128) + (kk & 3) * 32;
               const uint64_t qd = smem_desc(
                   q_addr + ((kk >> 2) & 1) * (C::kQBytes / 2) + (kk & 3) * 32, 16, 1024, 2);
-              const uint64_t kd = smem_desc(k_addr + (kk >> 3) * (2 * KT * 128) + off, 16, 1024, 2);
+              // (union: packed tiles, K-major no swizzle: 8-channel core
+              // matrices 128 B apart, 8-key groups 2 KB apart)
+              const uint64_t kd =
+                  MODE == kTileUnion
+                      ? smem_desc(k_addr + kk * 256, 128, 2048, 0)
+                      : smem_desc(k_addr + (kk >> 3) * (2 * KT * 128) + off, 16, 1024, 2);
               umma_bf16(tmem + static_cast<uint32_t>(gt & 1) * KT, qd, kd, idesc_s,
                         kk > 0 ? 1u : 0u);
             }
@@ -728,9 +757,17 @@ size_t union_lists_bytes(const Geometry& g) {
 }
 }  // namespace
 
-size_t union_ws_bytes(const Geometry& g) {
+size_t union_lists_ws_bytes(const Geometry& g) {
   if (!union_supported(g) || g.B == 0 || g.Tq == 0) return 0;
-  return union_lists_bytes(g) + static_cast<size_t>(union_tiles(g)) * sizeof(int32_t);
+  const size_t counts = static_cast<size_t>(union_tiles(g)) * sizeof(int32_t);
+  return union_lists_bytes(g) + ((counts + 255) & ~static_cast<size_t>(255));
+}
+
+// The query-tile schedule's workspace: the union lists, then K and V
+// repacked into block tiles.
+size_t union_ws_bytes(const Geometry& g) {
+  const size_t lists = union_lists_ws_bytes(g);
+  return lists ? lists + packed_kv_bytes(g) : 0;
 }
 
 int launch_union_build(const Geometry& g, const int32_t* idx, void* ws, const uint2** ulist,
@@ -775,6 +812,11 @@ int launch_union_tile(const Geometry& g, const void* Q, const void* K, const voi
   if (g.B == 0 || g.Tq == 0) return INFLLMV2_OK;
   TileArgs a = tile_args(g, O, lse);
   if (int e = launch_union_build(g, idx, ws, &a.ulist, &a.ucount, &a.ustride, st)) return e;
+  uint8_t* packed = static_cast<uint8_t*>(ws) + union_lists_ws_bytes(g);
+  if (int e = launch_pack_kv(g, K, V, packed, st)) return e;
+  a.Kp = packed;
+  a.Vp = packed + packed_kv_bytes(g) / 2;
+  a.nb = (g.T + kBlock - 1) / kBlock;
   CUtensorMap tq, tk, tv;
   if (int e = q_map(g, Q, &tq)) return e;
   if (int e = kv_map(g, K, &tk)) return e;
