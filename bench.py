@@ -926,7 +926,8 @@ def main():
     sustained = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     if dom == "sparse_attn":
         achieved = main_r["useful_attn_flops"] / (kern[dom] / 1e3) / 1e12
-        kfile = "sparse_attn.cu"
+        # G >= 4 runs the query-tile kernel over the union of the tile's blocks
+        kfile = "tile_attn.cu" if w.Hq // w.Hkv >= 4 else "sparse_attn.cu"
     else:
         achieved = main_r["useful_score_flops"] / (kern[dom] / 1e3) / 1e12
         kfile = "score.cu"
