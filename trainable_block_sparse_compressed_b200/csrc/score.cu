@@ -63,7 +63,7 @@ struct ScoreSmem {
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
-  float lse2[kRows];                 // per query row: log2-domain LSE
+  float nlse2[kRows];                // per query row: minus the log2-domain LSE
   float part_m[kEpiWG][kRows], part_l[kEpiWG][kRows];  // pass 1: each column group's max / sum
   float carry[3][4][kRows];          // S of the window just before each 32-lane quadrant
 };
@@ -241,19 +241,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---- pass 1: running max / sum of row r over its visible windows ----
         const int j0 = it * kKcTile + hf * kCW;
         const int nv = min(kCW, my_v - j0);  // valid columns of this group (may be <= 0)
-        float tm4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int c = 0; c < kCW; ++c)
-          if (c < nv) tm4[c & 3] = fmaxf(tm4[c & 3], x[c]);
-        const float tmax = fmaxf(fmaxf(tm4[0], tm4[1]), fmaxf(tm4[2], tm4[3]));
-        const float m_new = fmaxf(m_run, tmax);
-        if (m_new > -INFINITY) {
-          const float mb = m_new * scale_log2;
-          float a4[4] = {0.f, 0.f, 0.f, 0.f};
+        // windows the row may not see yet weigh exp2(-inf) = 0; only tiles
+        // where a lane of the warp has some pay for the masking
+        if (!__all_sync(0xffffffffu, nv >= kCW)) {
 #pragma unroll
           for (int c = 0; c < kCW; ++c)
-            if (c < nv) a4[c & 3] += fast_exp2(fmaf(x[c], scale_log2, -mb));
-          l_run = l_run * fast_exp2((m_run - m_new) * scale_log2) + ((a4[0] + a4[1]) + (a4[2] + a4[3]));
+            if (c >= nv) x[c] = -INFINITY;
+        }
+        float tm2[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < kCW; c += 4) {
+          tm2[0] = fmax3(tm2[0], x[c], x[c + 1]);
+          tm2[1] = fmax3(tm2[1], x[c + 2], x[c + 3]);
+        }
+        const float m_new = fmaxf(m_run, fmaxf(tm2[0], tm2[1]));
+        if (m_new > -INFINITY) {
+          const float2 sl2x2 = make_float2(scale_log2, scale_log2);
+          const float2 nmb = make_float2(-m_new * scale_log2, -m_new * scale_log2);
+          float2 a2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+          for (int c = 0; c < kCW; c += 2) {
+            const float2 e = fma2(make_float2(x[c], x[c + 1]), sl2x2, nmb);
+            a2[(c >> 1) & 1] = add2(a2[(c >> 1) & 1], make_float2(fast_exp2(e.x), fast_exp2(e.y)));
+          }
+          l_run = l_run * fast_exp2((m_run - m_new) * scale_log2) +
+                  ((a2[0].x + a2[0].y) + (a2[1].x + a2[1].y));
           m_run = m_new;
         }
         if (it == n_t - 1) {
@@ -276,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (m2 > -INFINITY) ll += sm.part_l[w][r] * fast_exp2((m2 - mm) * scale_log2);
               }
             }
-            sm.lse2[r] = my_v > 0 ? mm * scale_log2 + __log2f(ll) : INFINITY;
+            sm.nlse2[r] = my_v > 0 ? -(mm * scale_log2 + __log2f(ll)) : -INFINITY;
           }
           named_bar_sync(bar_sync_all, kEpiThreads);
         }
@@ -290,11 +302,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int tok = hf * TPH + tl;
           const int t = t0 + tok;
           const int v = t < q_end ? min(n_c, visible_windows(t)) : 0;
-          float a2[2] = {0.f, 0.f};
+          float sum;
+          if constexpr (G >= 2) {
+            // head pairs: one packed FMA for both arguments, one packed add
+            const float2 sl2x2 = make_float2(scale_log2, scale_log2);
+            const float2* nl = reinterpret_cast<const float2*>(sm.nlse2 + tok * G);
+            float2 a2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-          for (int h = 0; h < G; ++h)
-            a2[h & 1] += fast_exp2(fmaf(x[tl * G + h], scale_log2, -sm.lse2[tok * G + h]));
-          S[tl] = j < v ? a2[0] + a2[1] : -INFINITY;
+            for (int h = 0; h < G; h += 2) {
+              const float2 e = fma2(make_float2(x[tl * G + h], x[tl * G + h + 1]), sl2x2, nl[h / 2]);
+              a2[(h >> 1) & 1] = add2(a2[(h >> 1) & 1], make_float2(fast_exp2(e.x), fast_exp2(e.y)));
+            }
+            sum = (a2[0].x + a2[0].y) + (a2[1].x + a2[1].y);
+          } else {
+            sum = fast_exp2(fmaf(x[tl], scale_log2, sm.nlse2[tok]));
+          }
+          S[tl] = j < v ? sum : -INFINITY;
         }
         const int cb = i % 3;
         if (lane == 31) {

@@ -170,13 +170,12 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
   const int64_t n_items = static_cast<int64_t>(args.B) * args.Hkv * n_qt;
 
   // A key tile may fill only its first block (dense past the last token,
-  // union with an odd count): the stale rows of the other block are masked
-  // in S, and their V rows meet P = 0, so V must hold finite values: zero
-  // every stage's V area once.
-  for (int i = threadIdx.x; i < C::kStages * C::kVBytes / 16; i += blockDim.x) {
-    const int st = i / (C::kVBytes / 16), k = i % (C::kVBytes / 16);
-    reinterpret_cast<uint4*>(sKV + st * C::kStageBytes + C::kKBytes)[k] = make_uint4(0, 0, 0, 0);
-  }
+  // union with an odd count).  The softmax gives the other block's keys the
+  // weight exp2(s - inf) = 0, which needs finite scores s, and their V rows
+  // meet P = 0, which needs finite V: zero every stage once, so that a block
+  // never loaded holds zeros and one loaded before holds finite data.
+  for (int i = threadIdx.x; i < C::kStages * C::kStageBytes / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(sKV)[i] = make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -441,22 +440,31 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
         const bool full = !none && lo + H <= lim;
         float x[H];
         float mx = -INFINITY;
-        if (s_ok && __any_sync(0xffffffffu, !none)) {
+        // a warp none of whose rows sees a key of this half reads no score
+        // (x stays unset) and writes P = 0
+        const bool warp_any = s_ok && __any_sync(0xffffffffu, !none);
+        if (warp_any) {
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < H / 32; ++c)
             tmem_ld32(lane_addr + static_cast<uint32_t>(gt & 1) * KT + hf * H + 32 * c,
                       *reinterpret_cast<float(*)[32]>(x + 32 * c));
           tmem_ld_wait();
-          if (!full) {
+          // keys past the row's last visible one: only where a lane of the
+          // warp is on its causal diagonal (rows without any visible key are
+          // handled per row below, not per key)
+          if (__any_sync(0xffffffffu, !none && !full)) {
 #pragma unroll
             for (int c = 0; c < H; ++c)
-              if (none || lo + c >= lim) x[c] = -INFINITY;
+              if (lo + c >= lim) x[c] = -INFINITY;
           }
-          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          float m2[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-          for (int c = 0; c < H; ++c) m4[c & 3] = fmaxf(m4[c & 3], x[c]);
-          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+          for (int c = 0; c < H; c += 4) {
+            m2[0] = fmax3(m2[0], x[c], x[c + 1]);
+            m2[1] = fmax3(m2[1], x[c + 2], x[c + 3]);
+          }
+          mx = none ? -INFINITY : fmaxf(m2[0], m2[1]) * sl2;
         }
         // the row's reference maximum, common to both halves
         float alpha = 1.f;
@@ -483,22 +491,35 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
         // P = exp2(s - m) as bf16 pairs into tensor memory, 32 keys at a time
         const uint32_t pcol = lane_addr + C::kPCol + static_cast<uint32_t>(gt & 1) * (KT / 2) +
                               hf * (H / 2);
-        const bool zero = none || m == -INFINITY;
-        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+        float2 s2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        if (warp_any) {
+          // a row with no visible key here takes offset -inf, so that every
+          // exp2 of it is 0 (its scores are finite: every K row in shared
+          // memory is); otherwise m is finite
+          const float mo = none ? -INFINITY : -m;
+          const float2 sl2x2 = make_float2(sl2, sl2), mo2 = make_float2(mo, mo);
 #pragma unroll
-        for (int q = 0; q < H / 32; ++q) {
+          for (int q = 0; q < H / 32; ++q) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const float2 a =
+                  fma2(make_float2(x[32 * q + 2 * c], x[32 * q + 2 * c + 1]), sl2x2, mo2);
+              const float2 p = make_float2(fast_exp2(a.x), fast_exp2(a.y));
+              s2[c & 1] = add2(s2[c & 1], p);  // masked keys: exp2(-inf) = 0
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(p.x, p.y);
+              pk[c] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+            if (w_ok) tmem_st16(pcol + 16 * q, pk);
+          }
+        } else if (w_ok) {
           uint32_t pk[16];
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float p0 = zero ? 0.f : fast_exp2(fmaf(x[32 * q + 2 * c], sl2, -m));
-            const float p1 = zero ? 0.f : fast_exp2(fmaf(x[32 * q + 2 * c + 1], sl2, -m));
-            s4[c & 3] += p0 + p1;  // masked keys: exp2(-inf) = 0
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-            pk[c] = *reinterpret_cast<uint32_t*>(&b2);
-          }
-          if (w_ok) tmem_st16(pcol + 16 * q, pk);
+          for (int c = 0; c < 16; ++c) pk[c] = 0u;
+#pragma unroll
+          for (int q = 0; q < H / 32; ++q) tmem_st16(pcol + 16 * q, pk);
         }
-        l = l * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+        l = l * alpha + ((s2[0].x + s2[0].y) + (s2[1].x + s2[1].y));
         // move the O accumulator (this half's 64 channels) to the new
         // reference, once P V of the previous tile has added into it
         if (w_ok && i > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
