@@ -85,12 +85,13 @@ struct TileCfg {
   static constexpr uint32_t kOCol = 2 * KT;
   static constexpr uint32_t kPCol = kOCol + 128;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr int kThreads = 64 + 256 + 32;  // producer, S issuer, softmax x 8, P V issuer
+  // warps: Q/K producer, S issuer, softmax x 8, P V issuer, V producer
+  static constexpr int kThreads = 64 + 256 + 64;
 };
 
 struct TileSmem {
   uint64_t q_full[2], q_empty[2];
-  uint64_t kv_full[3], kv_empty[3];
+  uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
   uint64_t s_full[2], p_full[2], pv_done[2];
   uint64_t o_free, drain;
   uint32_t tmem_base;
@@ -186,8 +187,10 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
       mbar_init(&sm.pv_done[i], 1);
     }
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&sm.kv_full[s], 1);
-      mbar_init(&sm.kv_empty[s], 1);
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.v_empty[s], 1);
     }
     mbar_init(&sm.o_free, 8);
     mbar_init(&sm.drain, 2);  // one commit from each MMA issuer
@@ -204,27 +207,39 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort_flag = &sm.abort_flag;
 
-  if (warp == 0) {
-    // ------------------------------ producer ------------------------------
+  if (warp == 0 || warp == 11) {
+    // ------------------------------ producers -----------------------------
+    // Warp 0 loads the query tiles and the K tiles, warp 11 the V tiles.  A
+    // K stage is released once S has read it and a V stage once P V has, so
+    // the K loads of the next tiles need not wait for the softmax and the
+    // P V product of the tile that held the stage.
+    const bool v_role = warp == 11;
     if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
+      if (v_role) {
+        tma_prefetch_desc(&tmV);
+      } else {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+      }
+      const CUtensorMap* tm = v_role ? &tmV : &tmK;
+      const uint8_t* packed = v_role ? args.Vp : args.Kp;
       int qk = 0;
       int64_t gt = 0;
       bool ok = true;
       for (int64_t k = blockIdx.x; ok && k < n_items; k += gridDim.x) {
         const TileItem it = tile_item<G, MODE>(k, args, n_qt);
         if (it.n_kt == 0) continue;
-        const int qb = qk % C::kQBufs;
-        if (qk >= C::kQBufs &&
-            !(ok = tile_wait(&sm.q_empty[qb], ((qk / C::kQBufs) & 1) ^ 1, ctx, abort_flag)))
-          break;
-        mbar_arrive_expect_tx(&sm.q_full[qb], C::kQBytes);
-        uint8_t* q = sQ + qb * C::kQBytes;
-        tma_load_4d(q, &tmQ, &sm.q_full[qb], 0, it.g * G, it.qtok0, it.b);
-        tma_load_4d(q + C::kQBytes / 2, &tmQ, &sm.q_full[qb], 64, it.g * G, it.qtok0, it.b);
-        ++qk;
+        if (!v_role) {
+          const int qb = qk % C::kQBufs;
+          if (qk >= C::kQBufs &&
+              !(ok = tile_wait(&sm.q_empty[qb], ((qk / C::kQBufs) & 1) ^ 1, ctx, abort_flag)))
+            break;
+          mbar_arrive_expect_tx(&sm.q_full[qb], C::kQBytes);
+          uint8_t* q = sQ + qb * C::kQBytes;
+          tma_load_4d(q, &tmQ, &sm.q_full[qb], 0, it.g * G, it.qtok0, it.b);
+          tma_load_4d(q + C::kQBytes / 2, &tmQ, &sm.q_full[qb], 64, it.g * G, it.qtok0, it.b);
+          ++qk;
+        }
         uint2 ent[2] = {make_uint2(0u, 0u), make_uint2(0u, 0u)};  // union entries of tile i
         if (MODE == kTileUnion) {
           const uint2* L = args.ulist + it.list * args.ustride;
@@ -233,20 +248,18 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
         }
         for (int i = 0; i < it.n_kt; ++i, ++gt) {
           const int s = static_cast<int>(gt % C::kStages);
+          uint64_t* empty = v_role ? &sm.v_empty[s] : &sm.k_empty[s];
+          uint64_t* full = v_role ? &sm.v_full[s] : &sm.k_full[s];
           if (gt >= C::kStages &&
-              !(ok = tile_wait(&sm.kv_empty[s], ((gt / C::kStages) & 1) ^ 1, ctx, abort_flag)))
+              !(ok = tile_wait(empty, ((gt / C::kStages) & 1) ^ 1, ctx, abort_flag)))
             break;
-          uint8_t* stK = sKV + s * C::kStageBytes;
-          uint8_t* stV = stK + C::kKBytes;
-          uint64_t* full = &sm.kv_full[s];
+          uint8_t* dst = sKV + s * C::kStageBytes + (v_role ? C::kKBytes : 0);
           if (MODE == kTileCompressed) {
-            // 64 windows: K hi / lo planes x 2 channel halves, V hi x 2 halves
-            mbar_arrive_expect_tx(full, C::kStageBytes);
-            const int j0 = i * KT;
-            for (int x = 0; x < 4; ++x)
-              tma_load_4d(stK + x * C::kBox, &tmK, full, 64 * x, it.g, j0, it.b);
-            for (int x = 0; x < 2; ++x)
-              tma_load_4d(stV + x * C::kBox, &tmV, full, 64 * x, it.g, j0, it.b);
+            // 64 windows: K hi / lo planes x 2 channel halves, or V hi x 2 halves
+            const int nbox = v_role ? 2 : 4;
+            mbar_arrive_expect_tx(full, nbox * C::kBox);
+            for (int x = 0; x < nbox; ++x)
+              tma_load_4d(dst + x * C::kBox, tm, full, 64 * x, it.g, i * KT, it.b);
           } else {
             int blk[2];
             int nblk;
@@ -263,32 +276,31 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
               if (2 * i + 2 < it.n_u) ent[0] = __ldg(L + 2 * i + 2);
               if (2 * i + 3 < it.n_u) ent[1] = __ldg(L + 2 * i + 3);
             }
-            mbar_arrive_expect_tx(full, nblk * 4 * C::kBox);
+            mbar_arrive_expect_tx(full, nblk * 2 * C::kBox);
             for (int e = 0; e < nblk; ++e) {
               if (MODE == kTileUnion) {
-                // one 16 KB bulk copy per block and tensor from the packed
-                // tiles (no-swizzle canonical image; block e at e * 16 KB)
+                // one 16 KB bulk copy per block from the packed tiles
+                // (no-swizzle canonical image; block e at e * 16 KB)
                 const int64_t tile = (static_cast<int64_t>(it.b) * args.Hkv + it.g) * args.nb + blk[e];
-                bulk_load(stK + e * 16384, args.Kp + tile * 16384, 16384, full);
-                bulk_load(stV + e * 16384, args.Vp + tile * 16384, 16384, full);
+                bulk_load(dst + e * 16384, packed + tile * 16384, 16384, full);
               } else {
                 // 128-byte swizzled boxes: half h of block e at h * (KT rows) + e * 64 rows
-                for (int h = 0; h < 2; ++h) {
-                  tma_load_4d(stK + h * KT * 128 + e * C::kBox, &tmK, full, 64 * h, it.g,
+                for (int h = 0; h < 2; ++h)
+                  tma_load_4d(dst + h * KT * 128 + e * C::kBox, tm, full, 64 * h, it.g,
                               blk[e] * kBlock, it.b);
-                  tma_load_4d(stV + h * KT * 128 + e * C::kBox, &tmV, full, 64 * h, it.g,
-                              blk[e] * kBlock, it.b);
-                }
               }
             }
           }
         }
       }
       // drain: never leave with copies of this CTA in flight
-      for (int x = 0; x < C::kQBufs && x < qk; ++x)
-        mbar_wait(&sm.q_full[(qk - 1 - x) % C::kQBufs], ((qk - 1 - x) / C::kQBufs) & 1, ctx.wait_ns);
+      if (!v_role)
+        for (int x = 0; x < C::kQBufs && x < qk; ++x)
+          mbar_wait(&sm.q_full[(qk - 1 - x) % C::kQBufs], ((qk - 1 - x) / C::kQBufs) & 1,
+                    ctx.wait_ns);
       for (int64_t q = gt - 1; q >= 0 && q >= gt - C::kStages; --q)
-        mbar_wait(&sm.kv_full[q % C::kStages], (q / C::kStages) & 1, ctx.wait_ns);
+        mbar_wait(v_role ? &sm.v_full[q % C::kStages] : &sm.k_full[q % C::kStages],
+                  (q / C::kStages) & 1, ctx.wait_ns);
     }
   } else if (warp == 1 || warp == 10) {
     // ---------------------------- MMA issuers ----------------------------
@@ -299,10 +311,10 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
     // S products, warp 10 the P V products, each waiting only for what it
     // needs:
     //  - S(gt) needs its K tile and its TMEM buffer, last read by the softmax
-    //    for S(gt-2) before it signalled P(gt-2);
-    //  - P V(gt) needs P(gt) (signalled after S(gt) completed and was read,
-    //    so the K tile is read too: kv_empty after P V covers the whole
-    //    stage) and, first in its item, the previous item's O read out.
+    //    for S(gt-2) before it signalled P(gt-2); its completion releases
+    //    the K tile;
+    //  - P V(gt) needs P(gt), its V tile and, first in its item, the previous
+    //    item's O read out; its completion releases the V tile.
     if (lane == 0) {
       const bool pv_role = warp == 10;
       constexpr uint32_t idesc_s = instr_desc_bf16(128, KT, 0, 0);
@@ -320,8 +332,9 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
               break;
             if (i == 0 && ik > 0 && !(ok = tile_wait(&sm.o_free, (ik - 1) & 1, ctx, abort_flag)))
               break;
-            tc_fence_after();
             const int s = static_cast<int>(gt % C::kStages);
+            if (!(ok = tile_wait(&sm.v_full[s], (gt / C::kStages) & 1, ctx, abort_flag))) break;
+            tc_fence_after();
             const uint32_t v_addr = smem_u32(sKV + s * C::kStageBytes + C::kKBytes);
             const uint32_t p_tmem = tmem + C::kPCol + static_cast<uint32_t>(gt & 1) * (KT / 2);
 #pragma unroll
@@ -337,7 +350,7 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
               umma_bf16_ts(tmem + C::kOCol, p_tmem + 8 * kk, bd, idesc_pv,
                            (i == 0 && kk == 0) ? 0u : 1u);
             }
-            umma_commit(&sm.kv_empty[s]);
+            umma_commit(&sm.v_empty[s]);
             umma_commit(&sm.pv_done[gt & 1]);
           }
         } else {
@@ -346,7 +359,7 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
           const uint32_t q_addr = smem_u32(sQ + qb * C::kQBytes);
           for (int i = 0; ok && i < it.n_kt; ++i, ++gt) {
             const int s = static_cast<int>(gt % C::kStages);
-            if (!(ok = tile_wait(&sm.kv_full[s], (gt / C::kStages) & 1, ctx, abort_flag))) break;
+            if (!(ok = tile_wait(&sm.k_full[s], (gt / C::kStages) & 1, ctx, abort_flag))) break;
             if (gt >= 2 && !(ok = tile_wait(&sm.p_full[gt & 1],
                                             static_cast<uint32_t>(((gt >> 1) & 1) ^ 1), ctx,
                                             abort_flag)))
@@ -369,6 +382,7 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
               umma_bf16(tmem + static_cast<uint32_t>(gt & 1) * KT, qd, kd, idesc_s,
                         kk > 0 ? 1u : 0u);
             }
+            umma_commit(&sm.k_empty[s]);
             umma_commit(&sm.s_full[gt & 1]);
             if (i == it.n_kt - 1) umma_commit(&sm.q_empty[qb]);
           }
