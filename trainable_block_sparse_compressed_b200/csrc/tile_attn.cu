@@ -9,8 +9,9 @@
 //   S[128 rows x KT keys] = Q (K-major, 128-byte swizzle) x K_tile^T
 //   O[128 rows x 128 d ] += P (tensor memory)            x V_tile (MN-major)
 //
-// with S and P double-buffered and O accumulated in tensor memory (P is the
-// A operand straight from tensor memory, so it never touches shared memory).
+// with S double-buffered in tensor memory, P written over its S (the A
+// operand straight from tensor memory, so it never touches shared memory) and
+// O accumulated in tensor memory, one accumulator per softmax warpgroup.
 // Three key streams share the kernel:
 //
 //   dense      every key 0 .. t: exact dense causal attention (InfLLM-V2 skill
@@ -28,17 +29,21 @@
 //              windows; q . Kc takes both bf16 planes of the compressed key
 //              (K = 2 x 128), Vc its high plane.
 //
-// Warp roles: warp 0 loads Q (double-buffered) and the key tiles (K and V of
-// a tile in one ring stage) by TMA; warp 1 owns tensor memory and one of its
-// threads issues the S products, one thread of warp 10 the P V products;
-// warps 2-9 are the softmax, two warpgroups on the same 128
-// rows (thread = TMEM lane = query row), warpgroup hf taking the tile's keys
-// hf*KT/2 .. (hf+1)*KT/2 - 1 (in the union stream: one selected block each).
-// Each row keeps a reference maximum m, common to its two halves, that moves
-// only when a score exceeds it by more than 8 (log2 units): P = exp2(s - m)
-// <= 256 is exact enough in bf16, the halves exchange maxima only on those
-// (rare) moves, and only then is the O accumulator rescaled in tensor memory.
-// A half whose keys no row of its warp may see skips its exponentials.
+// Warp roles: warp 0 loads Q and the K tiles by TMA (or bulk copies), warp
+// 11 the V tiles, each into its own ring (a K stage is released once S has
+// read it, a V stage once P V has); warp 1 owns tensor memory and one of its
+// threads issues the S products, one thread of warp 10 the P V products.
+// Warps 2-9 are the softmax: two warpgroups on the same 128 rows (thread =
+// TMEM lane = query row), warpgroup w taking the keys w*KT/2 .. (w+1)*KT/2 - 1
+// of every tile (in the union stream: one selected block each), with its own
+// running maximum m_w and sum l_w per row and its own O accumulator O_w in
+// tensor memory; it writes P_w over its half of S.  The two never wait for
+// each other inside an item; at the item's end they merge
+// O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / (l_0 2^(m_0 - M) + l_1 2^(m_1 - M)).
+// A row's reference maximum moves only when a score exceeds it by more than
+// 8 (log2 units): P = exp2(s - m) <= 256 is exact enough in bf16, and O_w is
+// rescaled in tensor memory only on those (rare) moves.  A half whose keys no
+// row of its warp may see skips its exponentials.
 // Persistent CTAs, one per SM, take the query tiles heaviest first.
 #include "common.cuh"
 #include "sm100.cuh"
@@ -80,10 +85,9 @@ struct TileCfg {
   static constexpr int kStageBytes = kKBytes + kVBytes;
   static constexpr int kQBytes = 128 * 256;
   static constexpr int H = KT / 2;                               // keys per softmax warpgroup
-  // tensor memory: S0, S1 (KT fp32 columns each), O (128), P0, P1 (KT/2
-  // columns of packed bf16 pairs each)
+  // tensor memory: S0, S1 (KT fp32 columns each; P(gt), KT/2 columns of
+  // packed bf16 pairs, is written over S(gt)), then O0, O1 (128 each)
   static constexpr uint32_t kOCol = 2 * KT;
-  static constexpr uint32_t kPCol = kOCol + 128;
   static constexpr uint32_t kTmemCols = 512;
   // warps: Q/K producer, S issuer, softmax x 8, P V issuer, V producer
   static constexpr int kThreads = 64 + 256 + 64;
@@ -92,7 +96,7 @@ struct TileCfg {
 struct TileSmem {
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
-  uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t s_full[2][2], p_full[2][2], pv_done[2][2];  // [TMEM buffer][warpgroup]
   uint64_t o_free, drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -182,9 +186,12 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.q_full[i], 1);
       mbar_init(&sm.q_empty[i], 1);
-      mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.p_full[i], 8);  // one arrival per softmax warp
-      mbar_init(&sm.pv_done[i], 1);
+      mbar_init(&sm.s_full[i][0], 1);
+      mbar_init(&sm.s_full[i][1], 1);
+      mbar_init(&sm.p_full[i][0], 4);  // one arrival per warp of the warpgroup
+      mbar_init(&sm.p_full[i][1], 4);
+      mbar_init(&sm.pv_done[i][0], 1);
+      mbar_init(&sm.pv_done[i][1], 1);
     }
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&sm.k_full[s], 1);
@@ -310,14 +317,16 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
     // both products of every tile would be the bottleneck.  Warp 1 issues the
     // S products, warp 10 the P V products, each waiting only for what it
     // needs:
-    //  - S(gt) needs its K tile and its TMEM buffer, last read by the softmax
-    //    for S(gt-2) before it signalled P(gt-2); its completion releases
-    //    the K tile;
-    //  - P V(gt) needs P(gt), its V tile and, first in its item, the previous
-    //    item's O read out; its completion releases the V tile.
+    //  - S_w(gt), warpgroup w's half, needs the K tile and its half of the
+    //    TMEM buffer, which holds P_w(gt-2) until P V_w(gt-2) has completed;
+    //    completion of both halves releases the K tile;
+    //  - P V(gt) needs its V tile, first in its item both O accumulators
+    //    read out by the previous item's merge, and per warpgroup w its
+    //    P_w(gt), which it multiplies into O_w; its completion releases the
+    //    V tile.
     if (lane == 0) {
       const bool pv_role = warp == 10;
-      constexpr uint32_t idesc_s = instr_desc_bf16(128, KT, 0, 0);
+      constexpr uint32_t idesc_s = instr_desc_bf16(128, C::H, 0, 0);
       constexpr uint32_t idesc_pv = instr_desc_bf16(128, 128, 0, 1);
       int qk = 0, ik = 0;
       int64_t gt = 0;
@@ -327,31 +336,37 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
         if (it.n_kt == 0) continue;
         if (pv_role) {
           for (int i = 0; ok && i < it.n_kt; ++i, ++gt) {
-            if (!(ok = tile_wait(&sm.p_full[gt & 1], static_cast<uint32_t>((gt >> 1) & 1), ctx,
-                                 abort_flag)))
-              break;
             if (i == 0 && ik > 0 && !(ok = tile_wait(&sm.o_free, (ik - 1) & 1, ctx, abort_flag)))
               break;
             const int s = static_cast<int>(gt % C::kStages);
             if (!(ok = tile_wait(&sm.v_full[s], (gt / C::kStages) & 1, ctx, abort_flag))) break;
-            tc_fence_after();
             const uint32_t v_addr = smem_u32(sKV + s * C::kStageBytes + C::kKBytes);
-            const uint32_t p_tmem = tmem + C::kPCol + static_cast<uint32_t>(gt & 1) * (KT / 2);
+            for (int w = 0; ok && w < 2; ++w) {
+              // warpgroup w's P (over its S segment) times the V rows of its keys
+              if (!(ok = tile_wait(&sm.p_full[gt & 1][w], static_cast<uint32_t>((gt >> 1) & 1),
+                                   ctx, abort_flag)))
+                break;
+              tc_fence_after();
+              const uint32_t p_tmem = tmem + static_cast<uint32_t>(gt & 1) * KT + w * C::H;
+              const uint32_t o_tmem = tmem + C::kOCol + static_cast<uint32_t>(w) * 128;
 #pragma unroll
-            for (int kk = 0; kk < KT / 16; ++kk) {
-              // A = P in tensor memory: 16 keys = 8 columns of bf16 pairs.
-              // B = V: MN-major, 128-byte swizzle: 16 keys = 2 KB, the two
-              // 64-channel halves KT rows apart.
-              // (union: packed tiles, MN-major no swizzle: 8-key groups 2 KB
-              // apart, 8-channel groups 128 B apart, 16 keys = 4 KB)
-              const uint64_t bd = MODE == kTileUnion
-                                      ? smem_desc(v_addr + kk * 4096, 2048, 128, 0)
-                                      : smem_desc(v_addr + kk * 2048, KT * 128, 1024, 2);
-              umma_bf16_ts(tmem + C::kOCol, p_tmem + 8 * kk, bd, idesc_pv,
-                           (i == 0 && kk == 0) ? 0u : 1u);
+              for (int kk = 0; kk < C::H / 16; ++kk) {
+                // A = P in tensor memory: 16 keys = 8 columns of bf16 pairs.
+                // B = V: MN-major, 128-byte swizzle: 16 keys = 2 KB, the two
+                // 64-channel halves KT rows apart.
+                // (union: packed tiles, MN-major no swizzle: 8-key groups 2 KB
+                // apart, 8-channel groups 128 B apart, 16 keys = 4 KB)
+                const int kv = w * (C::H / 16) + kk;  // 16-key step within the tile
+                const uint64_t bd = MODE == kTileUnion
+                                        ? smem_desc(v_addr + kv * 4096, 2048, 128, 0)
+                                        : smem_desc(v_addr + kv * 2048, KT * 128, 1024, 2);
+                // the item's first tile starts the accumulator
+                umma_bf16_ts(o_tmem, p_tmem + 8 * kk, bd, idesc_pv, (i == 0 && kk == 0) ? 0u : 1u);
+              }
+              umma_commit(&sm.pv_done[gt & 1][w]);
             }
+            if (!ok) break;
             umma_commit(&sm.v_empty[s]);
-            umma_commit(&sm.pv_done[gt & 1]);
           }
         } else {
           const int qb = qk % C::kQBufs;
@@ -360,30 +375,38 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
           for (int i = 0; ok && i < it.n_kt; ++i, ++gt) {
             const int s = static_cast<int>(gt % C::kStages);
             if (!(ok = tile_wait(&sm.k_full[s], (gt / C::kStages) & 1, ctx, abort_flag))) break;
-            if (gt >= 2 && !(ok = tile_wait(&sm.p_full[gt & 1],
-                                            static_cast<uint32_t>(((gt >> 1) & 1) ^ 1), ctx,
-                                            abort_flag)))
-              break;
-            tc_fence_after();
             const uint32_t k_addr = smem_u32(sKV + s * C::kStageBytes);
+            for (int w = 0; ok && w < 2; ++w) {
+              // S_w(gt), the half of warpgroup w (N = KT/2 keys), needs its
+              // half of the TMEM buffer: P_w(gt-2) until P V_w(gt-2) completed
+              if (gt >= 2 && !(ok = tile_wait(&sm.pv_done[gt & 1][w],
+                                              static_cast<uint32_t>(((gt >> 1) & 1) ^ 1), ctx,
+                                              abort_flag)))
+                break;
+              tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 8 * C::KP; ++kk) {
-              // K-major, 128-byte swizzle: 16 channels = 32 B inside a
-              // 64-channel half; plane p, half h at (2p + h) * KT rows
-              const uint32_t off = ((kk >> 2) & 1) * (KT * 128) + (kk & 3) * 32;
-              const uint64_t qd = smem_desc(
-                  q_addr + ((kk >> 2) & 1) * (C::kQBytes / 2) + (kk & 3) * 32, 16, 1024, 2);
-              // (union: packed tiles, K-major no swizzle: 8-channel core
-              // matrices 128 B apart, 8-key groups 2 KB apart)
-              const uint64_t kd =
-                  MODE == kTileUnion
-                      ? smem_desc(k_addr + kk * 256, 128, 2048, 0)
-                      : smem_desc(k_addr + (kk >> 3) * (2 * KT * 128) + off, 16, 1024, 2);
-              umma_bf16(tmem + static_cast<uint32_t>(gt & 1) * KT, qd, kd, idesc_s,
-                        kk > 0 ? 1u : 0u);
+              for (int kk = 0; kk < 8 * C::KP; ++kk) {
+                // K-major, 128-byte swizzle: 16 channels = 32 B inside a
+                // 64-channel half; plane p, half h at (2p + h) * KT rows, the
+                // warpgroup's keys w * KT/2 rows further
+                const uint32_t off =
+                    ((kk >> 2) & 1) * (KT * 128) + (kk & 3) * 32 + w * (C::H * 128);
+                const uint64_t qd = smem_desc(
+                    q_addr + ((kk >> 2) & 1) * (C::kQBytes / 2) + (kk & 3) * 32, 16, 1024, 2);
+                // (union: packed tiles, block w at w * 16 KB, K-major no
+                // swizzle: 8-channel core matrices 128 B apart, 8-key groups
+                // 2 KB apart)
+                const uint64_t kd =
+                    MODE == kTileUnion
+                        ? smem_desc(k_addr + w * 16384 + kk * 256, 128, 2048, 0)
+                        : smem_desc(k_addr + (kk >> 3) * (2 * KT * 128) + off, 16, 1024, 2);
+                umma_bf16(tmem + static_cast<uint32_t>(gt & 1) * KT + w * C::H, qd, kd, idesc_s,
+                          kk > 0 ? 1u : 0u);
+              }
+              umma_commit(&sm.s_full[gt & 1][w]);
             }
+            if (!ok) break;
             umma_commit(&sm.k_empty[s]);
-            umma_commit(&sm.s_full[gt & 1]);
             if (i == it.n_kt - 1) umma_commit(&sm.q_empty[qb]);
           }
           ++qk;
@@ -396,16 +419,23 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
     }
   } else {
     // ------------------------------ softmax ------------------------------
-    constexpr int H = C::H;               // keys of this warpgroup per tile
-    const int hf = (warp - 2) >> 2;       // warpgroup: keys hf*H .. hf*H+H-1 of a tile
+    // Warpgroup w (warps 2-5, 6-9) takes segment w of every key tile (keys
+    // w*H .. w*H+H-1: one 64-key block, or 32 windows) for all 128 rows,
+    // with its own running maximum and sum per row and its own accumulator
+    // O_w, so the two never wait for each other inside an item; P_w is
+    // written over the segment's S.  At the item's end the two partial
+    // results are merged, each warpgroup writing 64 of the 128 channels.
+    constexpr int H = C::H;               // keys per segment
+    const int w = (warp - 2) >> 2;
     const int quad = warp & 3;            // TMEM lane quadrant of this warp
     const int r = quad * 32 + lane;       // query row of the tile
     const int tok = r / G, h = r % G;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    const uint32_t o_addr = lane_addr + C::kOCol;
     const float sl2 = args.scale_log2;
-    // named barriers over the 256 softmax threads: every decision taken at
-    // one is the same for both warpgroups, so neither leaves a loop while the
-    // other waits at a later barrier
+    const float2 sl2x2 = make_float2(sl2, sl2);
+    // named barriers over the 256 softmax threads, met once per item by both
+    // warpgroups, so neither leaves the item loop while the other waits
     constexpr uint32_t bar_sync = 1, bar_or = 2, kSm = 256;
     int64_t gt = 0;
     bool ok = true;
@@ -419,55 +449,59 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
       if (it.n_kt == 0) {
         // no visible key for any row of the tile (compressed, t < 31)
         if (row_ok) {
-          uint4* o = reinterpret_cast<uint4*>(args.O + orow * kHeadDim + 64 * hf);
+          uint4* o = reinterpret_cast<uint4*>(args.O + orow * kHeadDim + 64 * w);
           for (int c = 0; c < 8; ++c) o[c] = make_uint4(0, 0, 0, 0);
-          if (hf == 0) args.lse[lrow] = -INFINITY;
+          if (w == 0) args.lse[lrow] = -INFINITY;
         }
         continue;
       }
       // the last key (or, compressed, window count) this row may see
       const int lim = MODE == kTileCompressed ? min(args.n_c, visible_windows(t)) : t + 1;
       float m = -INFINITY, l = 0.f;
-      // union stream: this half's list entry of tile i, loaded one tile ahead
-      // so that its latency overlaps the previous tile
-      const uint2* ul = args.ulist + it.list * args.ustride + hf;
+      const int64_t gt0 = gt;
+      // union stream: this segment's list entry of tile i, loaded one tile
+      // ahead so that its latency overlaps the previous tile
+      const uint2* ul = args.ulist + it.list * args.ustride + w;
       uint2 e_next = make_uint2(0u, 0u);
-      if (MODE == kTileUnion && hf < it.n_u) e_next = __ldg(ul);
-      for (int i = 0; i < it.n_kt; ++i, ++gt) {
-        uint2 e_cur = e_next;
-        if (MODE == kTileUnion && 2 * (i + 1) + hf < it.n_u) e_next = __ldg(ul + 2 * (i + 1));
-        const bool s_ok =
-            __all_sync(0xffffffffu, tile_wait(&sm.s_full[gt & 1], (gt >> 1) & 1, ctx, abort_flag));
-        // this half's keys: [lo, lo + H) of one block (dense, union) or
-        // window range (compressed); sel: the row's token selected them
+      if (MODE == kTileUnion && w < it.n_u) e_next = __ldg(ul);
+      bool t_ok = true;
+      for (int i = 0; t_ok && i < it.n_kt; ++i) {
+        const int64_t g = gt0 + i;
+        const uint2 e_cur = e_next;  // an absent second block: entry 0, mask 0
+        if (MODE == kTileUnion)
+          e_next = 2 * (i + 1) + w < it.n_u ? __ldg(ul + 2 * (i + 1)) : make_uint2(0u, 0u);
+        const uint32_t s_addr = lane_addr + static_cast<uint32_t>(g & 1) * KT + w * H;
+        const bool s_ok = __all_sync(
+            0xffffffffu,
+            tile_wait(&sm.s_full[g & 1][w], static_cast<uint32_t>((g >> 1) & 1), ctx, abort_flag));
+        // this segment's keys: [lo, lo + H) of a block (dense, union) or
+        // window range (compressed); sel: the row's token selected the block
         int lo;
         bool sel = true;
         if (MODE == kTileUnion) {
-          if (2 * i + hf >= it.n_u) e_cur = make_uint2(0u, 0u);
           sel = ((e_cur.y >> tok) & 1u) != 0u;
           lo = static_cast<int>(e_cur.x) * kBlock;
         } else {
-          lo = i * KT + hf * H;
+          lo = i * KT + w * H;
         }
-        // none: no key of the half visible to the row; full: every key is
+        // none: no key of the segment visible to the row; full: every key is
         const bool none = !(row_ok && sel && lo < lim) || !s_ok;
         const bool full = !none && lo + H <= lim;
-        float x[H];
+        const bool any = __any_sync(0xffffffffu, !none);
+        const bool diag = __any_sync(0xffffffffu, !none && !full);
+        // pass 1: the row's maximum over the segment
         float mx = -INFINITY;
-        // a warp none of whose rows sees a key of this half reads no score
-        // (x stays unset) and writes P = 0
-        const bool warp_any = s_ok && __any_sync(0xffffffffu, !none);
-        if (warp_any) {
+        if (any) {
+          float x[H];
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < H / 32; ++c)
-            tmem_ld32(lane_addr + static_cast<uint32_t>(gt & 1) * KT + hf * H + 32 * c,
-                      *reinterpret_cast<float(*)[32]>(x + 32 * c));
+            tmem_ld32(s_addr + 32 * c, *reinterpret_cast<float(*)[32]>(x + 32 * c));
           tmem_ld_wait();
           // keys past the row's last visible one: only where a lane of the
-          // warp is on its causal diagonal (rows without any visible key are
-          // handled per row below, not per key)
-          if (__any_sync(0xffffffffu, !none && !full)) {
+          // warp is on its causal diagonal (rows without a visible key in
+          // the segment are handled per row, not per key)
+          if (diag) {
 #pragma unroll
             for (int c = 0; c < H; ++c)
               if (lo + c >= lim) x[c] = -INFINITY;
@@ -478,121 +512,133 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
             m2[0] = fmax3(m2[0], x[c], x[c + 1]);
             m2[1] = fmax3(m2[1], x[c + 2], x[c + 3]);
           }
-          mx = none ? -INFINITY : fmaxf(m2[0], m2[1]) * sl2;
+          if (!none) mx = fmaxf(m2[0], m2[1]) * sl2;
         }
-        // the row's reference maximum, common to both halves
+        // the reference maximum moves only when a score exceeds it by more
+        // than the slack (P <= 2^slack stays exact in bf16 and fp32)
         float alpha = 1.f;
-        const bool ab = !s_ok || *abort_flag != 0;
-        if (named_bar_or(bar_or, kSm, mx > m + kTileSlack || ab)) {
-          if (named_bar_or(bar_or, kSm, ab)) {
-            ok = false;
-            break;
-          }
-          sm.xch[gt & 1][hf][r] = mx;
-          named_bar_sync(bar_sync, kSm);
-          const float rm = fmaxf(mx, sm.xch[gt & 1][hf ^ 1][r]);
-          if (rm > m + kTileSlack) {
-            alpha = fast_exp2(m - rm);  // 0 while the row had no key
-            m = rm;
+        if (mx > m + kTileSlack) {
+          alpha = fast_exp2(m - mx);  // 0 while the row had no key
+          m = mx;
+        }
+        // move O_w to the new reference once P V of the previous tile has
+        // added into it (the item's first tile overwrites O_w)
+        if (i > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          t_ok = __all_sync(0xffffffffu,
+                            tile_wait(&sm.pv_done[(g - 1) & 1][w],
+                                      static_cast<uint32_t>(((g - 1) >> 1) & 1), ctx, abort_flag));
+          if (!t_ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float o[32];
+            tmem_ld32(o_addr + 128 * w + 32 * c, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              const float2 v = mul2(make_float2(o[j], o[j + 1]), make_float2(alpha, alpha));
+              o[j] = v.x;
+              o[j + 1] = v.y;
+            }
+            tmem_st32(o_addr + 128 * w + 32 * c, o);
           }
         }
-        // P(gt) reuses the buffer of P(gt-2): P V(gt-2) must have read it
-        bool w_ok = true;
-        if (gt >= 2)
-          w_ok = __all_sync(0xffffffffu, tile_wait(&sm.pv_done[gt & 1],
-                                                   static_cast<uint32_t>(((gt >> 1) & 1) ^ 1), ctx,
-                                                   abort_flag));
-        // P = exp2(s - m) as bf16 pairs into tensor memory, 32 keys at a time
-        const uint32_t pcol = lane_addr + C::kPCol + static_cast<uint32_t>(gt & 1) * (KT / 2) +
-                              hf * (H / 2);
+        // pass 2: P = exp2(s - m) as bf16 pairs written over the segment's S
+        // (keys 2c, 2c + 1 -> column c; the segment is read first), 32 keys
+        // at a time
         float2 s2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        if (warp_any) {
-          // a row with no visible key here takes offset -inf, so that every
-          // exp2 of it is 0 (its scores are finite: every K row in shared
-          // memory is); otherwise m is finite
+        if (any) {
+          float x[H];
+#pragma unroll
+          for (int c = 0; c < H / 32; ++c)
+            tmem_ld32(s_addr + 32 * c, *reinterpret_cast<float(*)[32]>(x + 32 * c));
+          tmem_ld_wait();
+          if (diag) {
+#pragma unroll
+            for (int c = 0; c < H; ++c)
+              if (lo + c >= lim) x[c] = -INFINITY;
+          }
+          // a row without a visible key in the segment takes offset -inf, so
+          // that every exp2 of it is 0 (its scores are finite: every K row in
+          // shared memory is); otherwise m is finite
           const float mo = none ? -INFINITY : -m;
-          const float2 sl2x2 = make_float2(sl2, sl2), mo2 = make_float2(mo, mo);
+          const float2 mo2 = make_float2(mo, mo);
 #pragma unroll
           for (int q = 0; q < H / 32; ++q) {
             uint32_t pk[16];
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
-              const float2 a =
-                  fma2(make_float2(x[32 * q + 2 * c], x[32 * q + 2 * c + 1]), sl2x2, mo2);
-              const float2 p = make_float2(fast_exp2(a.x), fast_exp2(a.y));
-              s2[c & 1] = add2(s2[c & 1], p);  // masked keys: exp2(-inf) = 0
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(p.x, p.y);
+              const float2 a = fma2(make_float2(x[32 * q + 2 * c], x[32 * q + 2 * c + 1]), sl2x2, mo2);
+              const float2 pp = make_float2(fast_exp2(a.x), fast_exp2(a.y));
+              s2[c & 1] = add2(s2[c & 1], pp);  // masked keys: exp2(-inf) = 0
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(pp.x, pp.y);
               pk[c] = *reinterpret_cast<uint32_t*>(&b2);
             }
-            if (w_ok) tmem_st16(pcol + 16 * q, pk);
+            tmem_st16(s_addr + 16 * q, pk);
           }
-        } else if (w_ok) {
+        } else {
           uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) pk[c] = 0u;
 #pragma unroll
-          for (int q = 0; q < H / 32; ++q) tmem_st16(pcol + 16 * q, pk);
+          for (int q = 0; q < H / 32; ++q) tmem_st16(s_addr + 16 * q, pk);
         }
         l = l * alpha + ((s2[0].x + s2[0].y) + (s2[1].x + s2[1].y));
-        // move the O accumulator (this half's 64 channels) to the new
-        // reference, once P V of the previous tile has added into it
-        if (w_ok && i > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-          w_ok = __all_sync(0xffffffffu,
-                            tile_wait(&sm.pv_done[(gt - 1) & 1],
-                                      static_cast<uint32_t>(((gt - 1) >> 1) & 1), ctx, abort_flag));
-          if (w_ok) {
-            tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              float o[32];
-              tmem_ld32(lane_addr + C::kOCol + 64 * hf + 32 * c, o);
-              tmem_ld_wait();
-#pragma unroll
-              for (int j = 0; j < 32; ++j) o[j] *= alpha;
-              tmem_st32(lane_addr + C::kOCol + 64 * hf + 32 * c, o);
-            }
-          }
-        }
-        if (w_ok) tmem_st_wait();
+        tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0 && w_ok) mbar_arrive(&sm.p_full[gt & 1]);
+        if (lane == 0 && s_ok) mbar_arrive(&sm.p_full[g & 1][w]);
+        t_ok = s_ok;
       }
-      if (!ok) break;
-      // ---- epilogue: O / l and the row's log-sum-exp ----
-      const bool e_ok = __all_sync(0xffffffffu,
-                                   tile_wait(&sm.pv_done[(gt - 1) & 1],
-                                             static_cast<uint32_t>(((gt - 1) >> 1) & 1), ctx,
-                                             abort_flag));
-      sm.xch[gt & 1][hf][r] = l;  // the parity no tile of this item still reads
+      gt = gt0 + it.n_kt;
+      // ---- merge: O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / L, and the LSE ----
+      // P V_1 of the item's last tile completes after all the others (the
+      // item's first tile overwrote both accumulators)
+      const int64_t gl = gt - 1;
+      const bool e_ok = t_ok && __all_sync(0xffffffffu,
+                                           tile_wait(&sm.pv_done[gl & 1][1],
+                                                     static_cast<uint32_t>((gl >> 1) & 1), ctx,
+                                                     abort_flag));
+      sm.xch[0][w][r] = m;
+      sm.xch[1][w][r] = l;
       if (named_bar_or(bar_or, kSm, !e_ok || *abort_flag != 0)) {
         ok = false;
         break;
       }
-      const float L = sm.xch[gt & 1][0][r] + sm.xch[gt & 1][1][r];
+      const float m0 = sm.xch[0][0][r], m1 = sm.xch[0][1][r];
+      const float M = fmaxf(m0, m1);
+      const float c0 = m0 > -INFINITY ? fast_exp2(m0 - M) : 0.f;
+      const float c1 = m1 > -INFINITY ? fast_exp2(m1 - M) : 0.f;
+      const float L = sm.xch[1][0][r] * c0 + sm.xch[1][1][r] * c1;
       const float inv = L > 0.f ? 1.f / L : 0.f;
+      const float2 f0 = make_float2(c0 * inv, c0 * inv), f1 = make_float2(c1 * inv, c1 * inv);
+      named_bar_sync(bar_sync, kSm);  // the exchange slots are free for the next item
       tc_fence_after();
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        float o[32];
-        tmem_ld32(lane_addr + C::kOCol + 64 * hf + 32 * c, o);
+        float o0[32], o1[32];
+        tmem_ld32(o_addr + 64 * w + 32 * c, o0);
+        tmem_ld32(o_addr + 128 + 64 * w + 32 * c, o1);
         tmem_ld_wait();
         if (row_ok && INFLLMV2_CHECK(ctx.status, it.b < args.B && it.g < args.Hkv)) {
-          uint4* dst = reinterpret_cast<uint4*>(args.O + orow * kHeadDim + 64 * hf + 32 * c);
+          uint4* dst = reinterpret_cast<uint4*>(args.O + orow * kHeadDim + 64 * w + 32 * c);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            uint32_t w[4];
+            uint32_t wd[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              __nv_bfloat162 b2 = __floats2bfloat162_rn(o[8 * j + 2 * e] * inv,
-                                                        o[8 * j + 2 * e + 1] * inv);
-              w[e] = *reinterpret_cast<uint32_t*>(&b2);
+              const int n = 8 * j + 2 * e;
+              // a half no key of which the row saw has c = 0 (and O = 0)
+              const float2 v = fma2(make_float2(o1[n], o1[n + 1]), f1,
+                                    mul2(make_float2(o0[n], o0[n + 1]), f0));
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(v.x, v.y);
+              wd[e] = *reinterpret_cast<uint32_t*>(&b2);
             }
-            dst[j] = make_uint4(w[0], w[1], w[2], w[3]);
+            dst[j] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
           }
         }
       }
-      if (row_ok && hf == 0) args.lse[lrow] = L > 0.f ? (m + __log2f(L)) * kLn2f : -INFINITY;
+      if (row_ok && w == 0) args.lse[lrow] = L > 0.f ? (M + __log2f(L)) * kLn2f : -INFINITY;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.o_free);
