@@ -65,7 +65,6 @@ struct ScoreSmem {
   int abort_flag;
   float nlse2[kRows];                // per query row: minus the log2-domain LSE
   float part_m[kEpiWG][kRows], part_l[kEpiWG][kRows];  // pass 1: each column group's max / sum
-  float carry[3][4][kRows];          // S of the window just before each 32-lane quadrant
 };
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, const DevCtx& ctx,
@@ -124,7 +123,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  for (int i = threadIdx.x; i < 3 * 4 * kRows; i += blockDim.x) (&sm.carry[0][0][0])[i] = -INFINITY;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -210,8 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t row0 = score_row_offset(q0);
     const int64_t slab = score_row_offset(q_end) - row0;
     float* srow_base = scores + (static_cast<int64_t>(b) * Hkv + g) * slab;
-    constexpr uint32_t bar_sync_all = 1, bar_or_all = 2;  // every epilogue thread
-    const uint32_t bar_sync_half = 3 + hf;                // the 128 threads of this warpgroup
+    constexpr uint32_t bar_sync_all = 1;  // every epilogue thread
 
     // pass-1 row identity
     const int my_tok = r / G;
@@ -221,13 +218,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     for (int it = 0; it < n_it; ++it) {
       const int a = it & 1;
-      // all epilogue threads take the same decision, so the named barriers below
-      // are always reached by every thread that waits at them
-      const bool ok = !*abort_flag && mbar_wait(&sm.acc_full[a], (it >> 1) & 1, ctx.wait_ns);
-      if (named_bar_or(bar_or_all, kEpiThreads, !ok)) {
-        if (!ok) report_status(ctx.status, INFLLMV2_STATUS_TIMEOUT);
+      // A wait that gives up sets the abort flag, after which no thread waits
+      // again; every epilogue thread still runs all n_it iterations (on
+      // whatever the accumulator holds), so the named barriers below are
+      // always met by all of them, without a vote per iteration.
+      if (!*abort_flag && !mbar_wait(&sm.acc_full[a], (it >> 1) & 1, ctx.wait_ns)) {
+        report_status(ctx.status, INFLLMV2_STATUS_TIMEOUT);
         *abort_flag = 1;
-        break;
       }
       tc_fence_after();
       float x[kCW];
@@ -290,6 +287,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             sm.nlse2[r] = my_v > 0 ? -(mm * scale_log2 + __log2f(ll)) : -INFINITY;
           }
+          // Blocks 8k start a 32-lane quadrant of pass 2: their windows come
+          // from two warps (the first one is the previous quadrant's last
+          // lane), which combine them by atomic max on the score's bits
+          // (scores are >= 0 or -inf, so integer order is float order).
+          // Start them at -inf.
+          for (int e = threadIdx.x - 64; e < TPT * (t_last / (8 * kBlock) + 1); e += kEpiThreads) {
+            const int tok = e % TPT, k8 = 8 * (e / TPT);
+            const int t = t0 + tok;
+            if (t < q_end && k8 <= t / kBlock &&
+                INFLLMV2_CHECK(ctx.status, score_row_offset(t) - row0 + k8 < slab))
+              srow_base[score_row_offset(t) - row0 + k8] = -INFINITY;
+          }
           named_bar_sync(bar_sync_all, kEpiThreads);
         }
       } else {
@@ -319,44 +328,45 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           S[tl] = j < v ? sum : -INFINITY;
         }
-        const int cb = i % 3;
-        if (lane == 31) {
-#pragma unroll
-          for (int tl = 0; tl < TPH; ++tl) {
-            const int tok = hf * TPH + tl;
-            if (quad < 3)
-              sm.carry[cb][quad + 1][tok] = S[tl];
-            else
-              sm.carry[(i + 1) % 3][0][tok] = S[tl];
-          }
-        }
-        named_bar_sync(bar_sync_half, 128);
         const int blk = i * (kKcTile / 4) + quad * 8 + (lane >> 2);
 #pragma unroll
         for (int tl = 0; tl < TPH; ++tl) {
           const int tok = hf * TPH + tl;
           float m4 = fmaxf(S[tl], __shfl_xor_sync(0xffffffffu, S[tl], 1));
           m4 = fmaxf(m4, __shfl_xor_sync(0xffffffffu, m4, 2));
-          float prev = __shfl_up_sync(0xffffffffu, S[tl], 1);
-          if (lane == 0) prev = sm.carry[cb][quad][tok];
+          const float prev = __shfl_up_sync(0xffffffffu, S[tl], 1);
           const int t = t0 + tok;
-          if ((lane & 3) == 0 && t < q_end && blk <= t / kBlock &&
-              INFLLMV2_CHECK(ctx.status, blk >= 0 && score_row_offset(t) - row0 + blk < slab))
-            srow_base[score_row_offset(t) - row0 + blk] = fmaxf(m4, prev);
+          if (t < q_end) {
+            const int cur = t / kBlock;
+            float* srow = srow_base + score_row_offset(t) - row0;
+            // block blk = max over windows 4 blk - 1 .. 4 blk + 3
+            if ((lane & 3) == 0 && blk <= cur &&
+                INFLLMV2_CHECK(ctx.status, blk >= 0 && score_row_offset(t) - row0 + blk < slab)) {
+              if (lane == 0)  // window 4 blk - 1 is the previous quadrant's
+                atomicMax(reinterpret_cast<int*>(srow + blk), __float_as_int(m4));
+              else
+                srow[blk] = fmaxf(m4, prev);
+            }
+            // this lane's window is the first of block blk + 1, which starts
+            // the next quadrant (or tile)
+            if (lane == 31 && blk + 1 <= cur &&
+                INFLLMV2_CHECK(ctx.status, score_row_offset(t) - row0 + blk + 1 < slab))
+              atomicMax(reinterpret_cast<int*>(srow + blk + 1), __float_as_int(S[tl]));
+          }
         }
       }
     }
-    // blocks past the last compressed-key tile: at most block 32*n_t, whose
-    // only visible window can be the last one of the final tile.
+    // blocks past the last compressed-key tile have no visible window, except
+    // block 32 n_t (a quadrant start, combined above), whose window before it
+    // is the final tile's last
     if (!*abort_flag) {
       for (int tok = hf * TPH + r; tok < (hf + 1) * TPH; tok += 128) {
         const int t = t0 + tok;
         if (t >= q_end) continue;
         const int cur = t / kBlock;
-        for (int blk = n_t * (kKcTile / 4); blk <= cur; ++blk)
+        for (int blk = n_t > 0 ? n_t * (kKcTile / 4) + 1 : 0; blk <= cur; ++blk)
           if (INFLLMV2_CHECK(ctx.status, score_row_offset(t) - row0 + blk < slab))
-            srow_base[score_row_offset(t) - row0 + blk] =
-              blk == n_t * (kKcTile / 4) ? sm.carry[n_t % 3][0][tok] : -INFINITY;
+            srow_base[score_row_offset(t) - row0 + blk] = -INFINITY;
       }
     }
   }

@@ -656,70 +656,42 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
 // ---------------------------------------------------------------------------
 // union lists: for every query tile (b, g, qt), the blocks its TPT tokens
 // selected, ascending, each with the mask of the tokens that selected it.
-// One CTA per tile: the (block, token) keys of the tile's index rows are
-// sorted (bitonic, in shared memory), equal blocks merged.
+// One CTA per tile: a token mask per block the tile's tokens may see (in
+// shared memory) takes one bit per (token, selected block); the non-empty
+// masks are then compacted in block order.
 // ---------------------------------------------------------------------------
 constexpr int kUnionThreads = 256;
-constexpr int kUnionPer = 32;  // sorted keys per thread when merging (cap <= 8192)
 
 template <int TPT>
 __global__ void __launch_bounds__(kUnionThreads) union_build_kernel(
     const int32_t* __restrict__ idx, uint2* __restrict__ ulist, int32_t* __restrict__ ucount,
-    int q0, int Tq, int topk, int n_qt, int cap) {
-  extern __shared__ uint32_t keys[];  // cap entries (a power of two)
+    int q0, int Tq, int topk, int n_qt) {
+  extern __shared__ uint32_t mask[];  // per block 0 .. nbt-1: the tokens that selected it
   __shared__ int scan[kUnionThreads / 32 + 1];
   const int64_t tile = blockIdx.x;
   const int64_t bg = tile / n_qt;
   const int qt = static_cast<int>(tile % n_qt);
+  const int t_last = q0 + min((qt + 1) * TPT, Tq) - 1;
+  const int nbt = t_last / kBlock + 1;  // blocks the tile's tokens may see
+  for (int b = threadIdx.x; b < nbt; b += blockDim.x) mask[b] = 0u;
+  __syncthreads();
   const int n = TPT * topk;
-  for (int e = threadIdx.x; e < cap; e += blockDim.x) {
-    uint32_t key = 0xFFFFFFFFu;
-    if (e < n) {
-      const int tk = e / topk, j = e % topk;
-      const int qtok = qt * TPT + tk;
-      if (qtok < Tq) {
-        const int v = __ldg(idx + ((bg * Tq + qtok) * topk + j));
-        const int t = q0 + qtok;
-        if (v >= 0 && v <= t / kBlock)
-          key = (static_cast<uint32_t>(v) << 5) | static_cast<uint32_t>(tk);
-      }
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    const int tk = e / topk, j = e % topk;
+    const int qtok = qt * TPT + tk;
+    if (qtok < Tq) {
+      const int v = __ldg(idx + ((bg * Tq + qtok) * topk + j));
+      const int t = q0 + qtok;
+      if (v >= 0 && v <= t / kBlock) atomicOr(&mask[v], 1u << tk);
     }
-    keys[e] = key;
   }
   __syncthreads();
-  for (int size = 2; size <= cap; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = threadIdx.x; i < cap / 2; i += blockDim.x) {
-        const int lo = 2 * i - (i & (stride - 1));
-        const int hi = lo + stride;
-        const bool up = (lo & size) == 0;
-        const uint32_t a = keys[lo], b = keys[hi];
-        if ((a > b) == up) {
-          keys[lo] = b;
-          keys[hi] = a;
-        }
-      }
-      __syncthreads();
-    }
-  }
-  // merge equal blocks: the first key of each block emits (block, token mask)
-  const int base = threadIdx.x * kUnionPer;
-  uint2 ent[kUnionPer];
+  // compaction in block order: thread i takes blocks [i per, (i+1) per)
+  const int per = (nbt + kUnionThreads - 1) / kUnionThreads;
+  const int b0 = threadIdx.x * per, b1 = min(b0 + per, nbt);
   int nh = 0;
-#pragma unroll
-  for (int s = 0; s < kUnionPer; ++s) {
-    const int p = base + s;
-    ent[s] = make_uint2(0xFFFFFFFFu, 0u);
-    if (p < cap && keys[p] != 0xFFFFFFFFu && (p == 0 || (keys[p] >> 5) != (keys[p - 1] >> 5))) {
-      const uint32_t blk = keys[p] >> 5;
-      uint32_t mask = 0u;
-      for (int q = p; q < cap && keys[q] != 0xFFFFFFFFu && (keys[q] >> 5) == blk; ++q)
-        mask |= 1u << (keys[q] & 31u);
-      ent[s] = make_uint2(blk, mask);
-      ++nh;
-    }
-  }
-  // exclusive scan of the head counts over threads
+  for (int b = b0; b < b1; ++b) nh += mask[b] != 0u;
+  // exclusive scan of the counts over threads
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   int x = nh;
 #pragma unroll
@@ -741,16 +713,11 @@ __global__ void __launch_bounds__(kUnionThreads) union_build_kernel(
   __syncthreads();
   int pos = scan[wid] + x - nh;
   uint2* L = ulist + tile * static_cast<int64_t>(n);
-#pragma unroll
-  for (int s = 0; s < kUnionPer; ++s)
-    if (ent[s].x != 0xFFFFFFFFu) L[pos++] = ent[s];
+  for (int b = b0; b < b1; ++b) {
+    const uint32_t m = mask[b];
+    if (m != 0u) L[pos++] = make_uint2(static_cast<uint32_t>(b), m);
+  }
   if (threadIdx.x == 0) ucount[tile] = scan[kUnionThreads / 32];
-}
-
-int next_pow2(int x) {
-  int p = 1;
-  while (p < x) p <<= 1;
-  return p;
 }
 
 template <int G, int MODE>
@@ -858,18 +825,19 @@ int launch_union_build(const Geometry& g, const int32_t* idx, void* ws, const ui
   const int n_qt = (g.Tq + TPT - 1) / TPT;
   const int64_t tiles = union_tiles(g);
   const int n = TPT * g.topk;
-  const int cap = next_pow2(n);
-  if (cap > kUnionPer * kUnionThreads) return INFLLMV2_ERR_UNSUPPORTED;
   uint2* L = static_cast<uint2*>(ws);
   int32_t* C = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + union_lists_bytes(g));
-  const size_t ush = static_cast<size_t>(cap) * sizeof(uint32_t);
+  // one token mask per block the last query token may see (<= 16 KB within
+  // the selection size limit)
+  const size_t ush = static_cast<size_t>((g.q0 + g.Tq - 1) / kBlock + 1) * sizeof(uint32_t);
+  if (ush > 48 * 1024) return INFLLMV2_ERR_UNSUPPORTED;
   const unsigned grid = static_cast<unsigned>(tiles);
   if (TPT == 8)
-    union_build_kernel<8><<<grid, kUnionThreads, ush, st>>>(idx, L, C, g.q0, g.Tq, g.topk, n_qt, cap);
+    union_build_kernel<8><<<grid, kUnionThreads, ush, st>>>(idx, L, C, g.q0, g.Tq, g.topk, n_qt);
   else if (TPT == 16)
-    union_build_kernel<16><<<grid, kUnionThreads, ush, st>>>(idx, L, C, g.q0, g.Tq, g.topk, n_qt, cap);
+    union_build_kernel<16><<<grid, kUnionThreads, ush, st>>>(idx, L, C, g.q0, g.Tq, g.topk, n_qt);
   else
-    union_build_kernel<32><<<grid, kUnionThreads, ush, st>>>(idx, L, C, g.q0, g.Tq, g.topk, n_qt, cap);
+    union_build_kernel<32><<<grid, kUnionThreads, ush, st>>>(idx, L, C, g.q0, g.Tq, g.topk, n_qt);
   if (cudaGetLastError() != cudaSuccess) return INFLLMV2_ERR_CUDA;
   *ulist = L;
   *ucount = C;
