@@ -10,49 +10,60 @@
 // each head's log-sum-exp over all visible windows before any probability can
 // be summed, so the kernel makes two passes over the compressed keys.
 //
-// One CTA owns a 128-row query tile: 128/G consecutive tokens x the G heads
-// of one group, rows ordered (token, head) -- exactly the box a single TMA
-// load of the BSHD query tensor produces.  Compressed-key tiles of 128 rows
-// stream through a 2-stage TMA ring.  Both passes run tcgen05.mma (M = N =
-// 128, bf16 in, fp32 accumulate in tensor memory).  Pass 2 runs over K =
-// 2 x 128: each compressed key is the bf16 pair hi + lo, so q . Kc = q . hi +
-// q . lo is accumulated in one tile (a single bf16 rounding of the keys would move
-// block scores by up to ~1e-2 relative).  Pass 1 only needs each row's
-// log-sum-exp, which scales all of that head's probabilities by one common
-// factor; the hi plane alone keeps that factor within ~2e-4 of exact (a fp64
-// emulation over the T=2048 and T=32768 workloads stays inside the selection
-// band on every row), so pass 1 reads and multiplies the hi plane only:
+// A query tile is 128 rows: 128/G consecutive tokens x the G heads of one
+// group, rows ordered (token, head) -- exactly the box a single TMA load of
+// the BSHD query tensor produces.  One CTA owns two consecutive query tiles,
+// so that every compressed-key tile it streams from L2 (the kernel's bound:
+// each CTA reads all the windows its tokens see) serves 256 rows.
+// Compressed-key tiles of 128 rows stream through a 2-stage TMA ring.  Both
+// passes run tcgen05.mma (bf16 in, fp32 accumulate in tensor memory).  Pass
+// 2 runs over K = 2 x 128: each compressed key is the bf16 pair hi + lo, so
+// q . Kc = q . hi + q . lo is accumulated in one tile (a single bf16 rounding
+// of the keys would move block scores by up to ~1e-2 relative).  Pass 1 only
+// needs each row's log-sum-exp, which scales all of that head's
+// probabilities by one common factor; the hi plane alone keeps that factor
+// within ~2e-4 of exact (a fp64 emulation over the T=2048 and T=32768
+// workloads stays inside the selection band on every row), so pass 1 reads
+// and multiplies the hi plane only:
 //
-//   pass 1  D = Q  x Kc^T : a TMEM lane is a query row; each thread keeps the
-//           running max / sum of its row -> per-row LSE, no cross-lane work;
-//   pass 2  D = Kc x Q^T  : operands swapped, a TMEM lane is a compressed key
-//           j and the thread holds all (token, head) scores of that key, so
-//           the group sum over heads is a register sum, and the max-pool over
-//           windows 4b-1 .. 4b+3 is two xor-shuffles plus one shuffle-up
-//           across neighbouring lanes (neighbouring windows).
+//   pass 1  D_i = Q_i x Kc^T (M = N = 128, one per query tile): a TMEM lane
+//           is a query row; each thread keeps the running max / sum of its
+//           row -> per-row LSE, no cross-lane work;
+//   pass 2  D = Kc x [Q_0; Q_1]^T (M = 128, N = 256): operands swapped, a
+//           TMEM lane is a compressed key j and the thread holds all (token,
+//           head) scores of that key, so the group sum over heads is a
+//           register sum, and the max-pool over windows 4b-1 .. 4b+3 is two
+//           xor-shuffles plus one shuffle-up across neighbouring lanes
+//           (neighbouring windows); a block that starts a 32-lane quadrant
+//           takes its first window from the previous quadrant's warp by an
+//           atomic max in global memory.
 //
 // Warp roles: warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs, warps
-// 2-5 (128 threads = 128 TMEM lanes) run the softmax / pooling epilogue.  The
-// accumulator is double-buffered in TMEM (2 x 128 columns) so the MMA of tile
-// i+1 overlaps the epilogue of tile i.  Block scores go to a causally packed
-// fp32 workspace (row t holds t/64 + 1 scores) for the top-k kernel.
+// 2-17 (four warpgroups, two per query tile) run the softmax / pooling
+// epilogue.  The accumulator (256 columns) is double-buffered in TMEM so the
+// MMAs of tile i+1 overlap the epilogue of tile i.  Block scores go to a
+// causally packed fp32 workspace (row t holds t/64 + 1 scores) for the top-k
+// kernel.
 #include "common.cuh"
 #include "sm100.cuh"
 
 namespace infllmv2 {
 namespace {
 
-constexpr int kRows = 128;                 // query rows per tile (M of pass 1)
+constexpr int kRows = 128;                 // query rows per query tile (M of pass 1)
+constexpr int kQT = 2;                     // query tiles per CTA (pass 2: N = 256)
 constexpr int kKcTile = 128;               // compressed keys per tile
 constexpr int kStages = 2;
 constexpr int kHalfBytes = kRows * 64 * 2; // one 64-channel half of a 128-row tile
-constexpr int kTileBytes = 2 * kHalfBytes; // 32 KB: the query tile
+constexpr int kTileBytes = 2 * kHalfBytes; // 32 KB: one query tile, or one plane of a key tile
+constexpr int kQBytes = kQT * kTileBytes;  // both query tiles: [half][tile][row]
 constexpr int kKcBytes = 4 * kHalfBytes;   // 64 KB: hi and lo planes of 128 compressed keys
-constexpr int kEpiWG = 4;                  // epilogue warpgroups
-constexpr int kCW = 128 / kEpiWG;          // accumulator columns per warpgroup
+constexpr int kEpiWG = 4;                  // epilogue warpgroups: two per query tile
+constexpr int kCW = kQT * 128 / kEpiWG;    // accumulator columns per warpgroup (two chunks of 32)
 constexpr int kEpiThreads = 128 * kEpiWG;
 constexpr int kThreads = 64 + kEpiThreads;
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kAccCols = kQT * 128;   // one accumulator: both query tiles
+constexpr uint32_t kTmemCols = 2 * kAccCols;
 
 struct ScoreSmem {
   uint64_t q_full;
@@ -63,8 +74,8 @@ struct ScoreSmem {
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
-  float nlse2[kRows];                // per query row: minus the log2-domain LSE
-  float part_m[kEpiWG][kRows], part_l[kEpiWG][kRows];  // pass 1: each column group's max / sum
+  float nlse2[kQT * kRows];          // per query row: minus the log2-domain LSE
+  float part_m[kEpiWG][kRows], part_l[kEpiWG][kRows];  // pass 1: each column half's max / sum
 };
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, const DevCtx& ctx,
@@ -82,24 +93,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tmKc, float* __restrict__ scores,
                         int B, int q0, int Tq, int Hkv, int n_c, float scale_log2,
                         DevCtx ctx) {
-  constexpr int TPT = kRows / G;  // tokens per tile
+  constexpr int TPT = kRows / G;  // tokens per query tile
+  constexpr int TPC = 32 / G;     // tokens per 32-column chunk in pass 2 (G <= 32)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint8_t* sQ = base;
-  uint8_t* sKc = base + kTileBytes;
-  ScoreSmem& sm = *reinterpret_cast<ScoreSmem*>(base + kTileBytes + kKcBytes * kStages);
+  uint8_t* sKc = base + kQBytes;
+  ScoreSmem& sm = *reinterpret_cast<ScoreSmem*>(base + kQBytes + kKcBytes * kStages);
 
-  // heaviest (latest) query tiles first
-  // queries are tokens q0 .. q0+Tq-1 (a whole prefill: q0 = 0); keys and
-  // compressed keys cover tokens 0 .. q0+Tq-1
+  // A CTA takes the query tiles 2p and 2p+1 of one (b, g), heaviest (latest)
+  // pairs first.  Queries are tokens q0 .. q0+Tq-1 (a whole prefill: q0 = 0);
+  // keys and compressed keys cover tokens 0 .. q0+Tq-1.
   const int q_end = q0 + Tq;
   const int n_qt = (Tq + TPT - 1) / TPT;
+  const int n_pair = (n_qt + kQT - 1) / kQT;
   const int bg = blockIdx.x % (B * Hkv);
-  const int qt = n_qt - 1 - static_cast<int>(blockIdx.x / (B * Hkv));
+  const int pair = n_pair - 1 - static_cast<int>(blockIdx.x / (B * Hkv));
   const int b = bg / Hkv, g = bg % Hkv;
-  const int t0 = q0 + qt * TPT;
-  const int t_last = min(t0 + TPT - 1, q_end - 1);
+  const int t0 = q0 + pair * kQT * TPT;  // first token of the CTA
+  const int t_last = min(t0 + kQT * TPT - 1, q_end - 1);
   const int v_max = min(n_c, visible_windows(t_last));
   const int n_t = (v_max + kKcTile - 1) / kKcTile;
   const int n_it = 2 * n_t;
@@ -134,9 +147,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && n_t > 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmKc);
-      mbar_arrive_expect_tx(&sm.q_full, kTileBytes);
-      tma_load_4d(sQ, &tmQ, &sm.q_full, 0, g * G, t0 - q0, b);
-      tma_load_4d(sQ + kHalfBytes, &tmQ, &sm.q_full, 64, g * G, t0 - q0, b);
+      // query tile i, channel half h at h * 64 KB + i * 32 KB (a tile past
+      // the last query token is filled with zeros)
+      mbar_arrive_expect_tx(&sm.q_full, kQBytes);
+      for (int i = 0; i < kQT; ++i)
+        for (int h = 0; h < 2; ++h)
+          tma_load_4d(sQ + h * kQT * kHalfBytes + i * kHalfBytes, &tmQ, &sm.q_full, 64 * h, g * G,
+                      t0 - q0 + i * TPT, b);
       int issued = 0;
       for (int it = 0; it < n_it; ++it) {
         const int s = it % kStages;
@@ -163,7 +180,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0 && n_t > 0) {
-      constexpr uint32_t idesc = instr_desc_bf16(128, 128, 0, 0);
+      constexpr uint32_t idesc1 = instr_desc_bf16(128, 128, 0, 0);
+      constexpr uint32_t idesc2 = instr_desc_bf16(128, kQT * 128, 0, 0);
       bool ok = wait_or_abort(&sm.q_full, 0, ctx, abort_flag);
       const uint32_t q_addr = smem_u32(sQ);
       for (int it = 0; ok && it < n_it; ++it) {
@@ -173,16 +191,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         tc_fence_after();
         const uint32_t kc_addr = smem_u32(sKc + s * kKcBytes);
-        const bool pass1 = it < n_t;
-        // pass 2: q . Kc = q . hi + q . lo, K = 2 x 128 with the query tile
-        // used twice; pass 1: q . hi, K = 128
+        const uint32_t d = tmem + a * kAccCols;
+        if (it < n_t) {
+          // pass 1: S_i = Q_i x hi^T (K = 128) into columns i * 128 of the
+          // accumulator, for both query tiles
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          if (pass1 && k >= 8) break;
-          const uint32_t off = ((k >> 2) & 1) * kHalfBytes + (k & 3) * 32;
-          const uint64_t qd = smem_desc(q_addr + off, 16, 1024, 2);
-          const uint64_t kd = smem_desc(kc_addr + (k >> 3) * kTileBytes + off, 16, 1024, 2);
-          umma_bf16(tmem + a * 128, pass1 ? qd : kd, pass1 ? kd : qd, idesc, k > 0 ? 1u : 0u);
+          for (int i = 0; i < kQT; ++i)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const uint32_t off = ((k >> 2) & 1) * kHalfBytes + (k & 3) * 32;
+              const uint64_t qd = smem_desc(
+                  q_addr + ((k >> 2) & 1) * kQT * kHalfBytes + i * kHalfBytes + (k & 3) * 32, 16,
+                  1024, 2);
+              const uint64_t kd = smem_desc(kc_addr + off, 16, 1024, 2);
+              umma_bf16(d + i * 128, qd, kd, idesc1, k > 0 ? 1u : 0u);
+            }
+        } else {
+          // pass 2: D = Kc x [Q_0; Q_1]^T (M = 128 keys, N = 256 query rows,
+          // K = 2 x 128: q . Kc = q . hi + q . lo); the 256 rows of a channel
+          // half are contiguous, so one descriptor spans both tiles
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const uint32_t off = ((k >> 2) & 1) * kHalfBytes + (k & 3) * 32;
+            const uint64_t qd =
+                smem_desc(q_addr + ((k >> 2) & 1) * kQT * kHalfBytes + (k & 3) * 32, 16, 1024, 2);
+            const uint64_t kd = smem_desc(kc_addr + (k >> 3) * kTileBytes + off, 16, 1024, 2);
+            umma_bf16(d, kd, qd, idesc2, k > 0 ? 1u : 0u);
+          }
         }
         umma_commit(&sm.kc_empty[s]);
         umma_commit(&sm.acc_full[a]);
@@ -193,14 +228,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // -------------- epilogue: 16 warps, thread <-> TMEM lane --------------
-    // Four warpgroups split the accumulator's 128 columns: warpgroup hf reads
-    // columns kCW hf .. kCW hf + kCW - 1 of its lanes.  Pass 1: each keeps a
-    // partial running max / sum of its row over its columns, merged at the
-    // end of the pass.  Pass 2: the columns are (token, head) pairs, so
-    // warpgroup hf owns tokens hf TPH .. (hf+1) TPH - 1.  Four warps per
-    // scheduler keep the exp2 / shuffle chains of the epilogue overlapped.
-    constexpr int TPH = TPT / kEpiWG;  // tokens per warpgroup in pass 2 (G <= 32)
+    // Warpgroup hf reads accumulator columns kCW hf .. kCW hf + kCW - 1 of its
+    // lanes, two chunks of 32: in pass 1 half (hf & 1) of the key columns of
+    // query tile hf / 2 (a lane is a query row of that tile); in pass 2 the
+    // (token, head) columns of tokens (hf & 1) TPT/2 .. of tile hf / 2 (a
+    // lane is a compressed key).  Pass 1 keeps a partial running max / sum
+    // per row, merged at the end of the pass.
     const int hf = (warp - 2) >> 2;
+    const int qi = hf >> 1;          // the warpgroup's query tile
     const int quad = warp & 3;
     const int r = quad * 32 + lane;  // TMEM lane this thread reads
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + hf * kCW;
@@ -209,10 +244,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t slab = score_row_offset(q_end) - row0;
     float* srow_base = scores + (static_cast<int64_t>(b) * Hkv + g) * slab;
     constexpr uint32_t bar_sync_all = 1;  // every epilogue thread
+    const int tq0 = t0 + qi * TPT;        // first token of the warpgroup's query tile
 
     // pass-1 row identity
-    const int my_tok = r / G;
-    const int my_t = t0 + my_tok;
+    const int my_t = tq0 + r / G;
     const int my_v = my_t < q_end ? min(n_c, visible_windows(my_t)) : 0;
     float m_run = -INFINITY, l_run = 0.f;
 
@@ -226,141 +261,142 @@ __global__ void __launch_bounds__(kThreads, 1)
         report_status(ctx.status, INFLLMV2_STATUS_TIMEOUT);
         *abort_flag = 1;
       }
-      tc_fence_after();
-      float x[kCW];
-      tmem_ld32(lane_addr + a * 128, *reinterpret_cast<float(*)[32]>(x));
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.acc_empty[a]);
-
-      if (it < n_t) {
-        // ---- pass 1: running max / sum of row r over its visible windows ----
-        const int j0 = it * kKcTile + hf * kCW;
-        const int nv = min(kCW, my_v - j0);  // valid columns of this group (may be <= 0)
-        // windows the row may not see yet weigh exp2(-inf) = 0; only tiles
-        // where a lane of the warp has some pay for the masking
-        if (!__all_sync(0xffffffffu, nv >= kCW)) {
 #pragma unroll
-          for (int c = 0; c < kCW; ++c)
-            if (c >= nv) x[c] = -INFINITY;
+      for (int c = 0; c < kCW / 32; ++c) {
+        tc_fence_after();
+        float x[32];
+        tmem_ld32(lane_addr + a * kAccCols + 32 * c, x);
+        tmem_ld_wait();
+        if (c == kCW / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.acc_empty[a]);
         }
-        float tm2[2] = {-INFINITY, -INFINITY};
+        if (it < n_t) {
+          // ---- pass 1: running max / sum of row r over its visible windows ----
+          const int j0 = it * kKcTile + (hf & 1) * kCW + 32 * c;
+          const int nv = min(32, my_v - j0);  // valid columns of this chunk (may be <= 0)
+          // windows the row may not see yet weigh exp2(-inf) = 0; only chunks
+          // where a lane of the warp has some pay for the masking
+          if (!__all_sync(0xffffffffu, nv >= 32)) {
 #pragma unroll
-        for (int c = 0; c < kCW; c += 4) {
-          tm2[0] = fmax3(tm2[0], x[c], x[c + 1]);
-          tm2[1] = fmax3(tm2[1], x[c + 2], x[c + 3]);
-        }
-        const float m_new = fmaxf(m_run, fmaxf(tm2[0], tm2[1]));
-        if (m_new > -INFINITY) {
-          const float2 sl2x2 = make_float2(scale_log2, scale_log2);
-          const float2 nmb = make_float2(-m_new * scale_log2, -m_new * scale_log2);
-          float2 a2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-          for (int c = 0; c < kCW; c += 2) {
-            const float2 e = fma2(make_float2(x[c], x[c + 1]), sl2x2, nmb);
-            a2[(c >> 1) & 1] = add2(a2[(c >> 1) & 1], make_float2(fast_exp2(e.x), fast_exp2(e.y)));
+            for (int j = 0; j < 32; ++j)
+              if (j >= nv) x[j] = -INFINITY;
           }
-          l_run = l_run * fast_exp2((m_run - m_new) * scale_log2) +
-                  ((a2[0].x + a2[0].y) + (a2[1].x + a2[1].y));
-          m_run = m_new;
-        }
-        if (it == n_t - 1) {
-          // merge the column groups of row r
-          if (hf > 0) {
-            sm.part_m[hf][r] = m_run;
-            sm.part_l[hf][r] = l_run;
-          }
-          named_bar_sync(bar_sync_all, kEpiThreads);
-          if (hf == 0) {
-            float mm = m_run;
+          float tm2[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-            for (int w = 1; w < kEpiWG; ++w) mm = fmaxf(mm, sm.part_m[w][r]);
-            float ll = 0.f;
-            if (mm > -INFINITY) {
-              ll = m_run > -INFINITY ? l_run * fast_exp2((m_run - mm) * scale_log2) : 0.f;
-#pragma unroll
-              for (int w = 1; w < kEpiWG; ++w) {
-                const float m2 = sm.part_m[w][r];
-                if (m2 > -INFINITY) ll += sm.part_l[w][r] * fast_exp2((m2 - mm) * scale_log2);
-              }
-            }
-            sm.nlse2[r] = my_v > 0 ? -(mm * scale_log2 + __log2f(ll)) : -INFINITY;
+          for (int j = 0; j < 32; j += 4) {
+            tm2[0] = fmax3(tm2[0], x[j], x[j + 1]);
+            tm2[1] = fmax3(tm2[1], x[j + 2], x[j + 3]);
           }
-          // Blocks 8k start a 32-lane quadrant of pass 2: their windows come
-          // from two warps (the first one is the previous quadrant's last
-          // lane), which combine them by atomic max on the score's bits
-          // (scores are >= 0 or -inf, so integer order is float order).
-          // Start them at -inf.
-          for (int e = threadIdx.x - 64; e < TPT * (t_last / (8 * kBlock) + 1); e += kEpiThreads) {
-            const int tok = e % TPT, k8 = 8 * (e / TPT);
-            const int t = t0 + tok;
-            if (t < q_end && k8 <= t / kBlock &&
-                INFLLMV2_CHECK(ctx.status, score_row_offset(t) - row0 + k8 < slab))
-              srow_base[score_row_offset(t) - row0 + k8] = -INFINITY;
-          }
-          named_bar_sync(bar_sync_all, kEpiThreads);
-        }
-      } else {
-        // ---- pass 2: lane r is compressed key j; columns are (token, head) rows ----
-        const int i = it - n_t;
-        const int j = i * kKcTile + r;
-        float S[TPH];
-#pragma unroll
-        for (int tl = 0; tl < TPH; ++tl) {
-          const int tok = hf * TPH + tl;
-          const int t = t0 + tok;
-          const int v = t < q_end ? min(n_c, visible_windows(t)) : 0;
-          float sum;
-          if constexpr (G >= 2) {
-            // head pairs: one packed FMA for both arguments, one packed add
+          const float m_new = fmaxf(m_run, fmaxf(tm2[0], tm2[1]));
+          if (m_new > -INFINITY) {
             const float2 sl2x2 = make_float2(scale_log2, scale_log2);
-            const float2* nl = reinterpret_cast<const float2*>(sm.nlse2 + tok * G);
+            const float2 nmb = make_float2(-m_new * scale_log2, -m_new * scale_log2);
             float2 a2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-            for (int h = 0; h < G; h += 2) {
-              const float2 e = fma2(make_float2(x[tl * G + h], x[tl * G + h + 1]), sl2x2, nl[h / 2]);
-              a2[(h >> 1) & 1] = add2(a2[(h >> 1) & 1], make_float2(fast_exp2(e.x), fast_exp2(e.y)));
+            for (int j = 0; j < 32; j += 2) {
+              const float2 e = fma2(make_float2(x[j], x[j + 1]), sl2x2, nmb);
+              a2[(j >> 1) & 1] = add2(a2[(j >> 1) & 1], make_float2(fast_exp2(e.x), fast_exp2(e.y)));
             }
-            sum = (a2[0].x + a2[0].y) + (a2[1].x + a2[1].y);
-          } else {
-            sum = fast_exp2(fmaf(x[tl], scale_log2, sm.nlse2[tok]));
+            l_run = l_run * fast_exp2((m_run - m_new) * scale_log2) +
+                    ((a2[0].x + a2[0].y) + (a2[1].x + a2[1].y));
+            m_run = m_new;
           }
-          S[tl] = j < v ? sum : -INFINITY;
-        }
-        const int blk = i * (kKcTile / 4) + quad * 8 + (lane >> 2);
+        } else {
+          // ---- pass 2: lane r is compressed key j; columns are (token, head) pairs ----
+          const int i = it - n_t;
+          const int j = i * kKcTile + r;
+          const int tc0 = ((hf & 1) * kCW + 32 * c) / G;  // first token of the chunk in its tile
+          float S[TPC];
 #pragma unroll
-        for (int tl = 0; tl < TPH; ++tl) {
-          const int tok = hf * TPH + tl;
-          float m4 = fmaxf(S[tl], __shfl_xor_sync(0xffffffffu, S[tl], 1));
-          m4 = fmaxf(m4, __shfl_xor_sync(0xffffffffu, m4, 2));
-          const float prev = __shfl_up_sync(0xffffffffu, S[tl], 1);
-          const int t = t0 + tok;
-          if (t < q_end) {
-            const int cur = t / kBlock;
-            float* srow = srow_base + score_row_offset(t) - row0;
-            // block blk = max over windows 4 blk - 1 .. 4 blk + 3
-            if ((lane & 3) == 0 && blk <= cur &&
-                INFLLMV2_CHECK(ctx.status, blk >= 0 && score_row_offset(t) - row0 + blk < slab)) {
-              if (lane == 0)  // window 4 blk - 1 is the previous quadrant's
-                atomicMax(reinterpret_cast<int*>(srow + blk), __float_as_int(m4));
-              else
-                srow[blk] = fmaxf(m4, prev);
+          for (int tl = 0; tl < TPC; ++tl) {
+            const int tok = tc0 + tl;
+            const int t = tq0 + tok;
+            const int v = t < q_end ? min(n_c, visible_windows(t)) : 0;
+            float sum;
+            if constexpr (G >= 2) {
+              // head pairs: one packed FMA for both arguments, one packed add
+              const float2 sl2x2 = make_float2(scale_log2, scale_log2);
+              const float2* nl = reinterpret_cast<const float2*>(sm.nlse2 + qi * kRows + tok * G);
+              float2 a2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+              for (int h = 0; h < G; h += 2) {
+                const float2 e = fma2(make_float2(x[tl * G + h], x[tl * G + h + 1]), sl2x2, nl[h / 2]);
+                a2[(h >> 1) & 1] = add2(a2[(h >> 1) & 1], make_float2(fast_exp2(e.x), fast_exp2(e.y)));
+              }
+              sum = (a2[0].x + a2[0].y) + (a2[1].x + a2[1].y);
+            } else {
+              sum = fast_exp2(fmaf(x[tl], scale_log2, sm.nlse2[qi * kRows + tok]));
             }
-            // this lane's window is the first of block blk + 1, which starts
-            // the next quadrant (or tile)
-            if (lane == 31 && blk + 1 <= cur &&
-                INFLLMV2_CHECK(ctx.status, score_row_offset(t) - row0 + blk + 1 < slab))
-              atomicMax(reinterpret_cast<int*>(srow + blk + 1), __float_as_int(S[tl]));
+            S[tl] = j < v ? sum : -INFINITY;
+          }
+          const int blk = i * (kKcTile / 4) + quad * 8 + (lane >> 2);
+#pragma unroll
+          for (int tl = 0; tl < TPC; ++tl) {
+            float m4 = fmaxf(S[tl], __shfl_xor_sync(0xffffffffu, S[tl], 1));
+            m4 = fmaxf(m4, __shfl_xor_sync(0xffffffffu, m4, 2));
+            const float prev = __shfl_up_sync(0xffffffffu, S[tl], 1);
+            const int t = tq0 + tc0 + tl;
+            if (t < q_end) {
+              const int cur = t / kBlock;
+              float* srow = srow_base + score_row_offset(t) - row0;
+              // block blk = max over windows 4 blk - 1 .. 4 blk + 3
+              if ((lane & 3) == 0 && blk <= cur &&
+                  INFLLMV2_CHECK(ctx.status, blk >= 0 && score_row_offset(t) - row0 + blk < slab)) {
+                if (lane == 0)  // window 4 blk - 1 is the previous quadrant's
+                  atomicMax(reinterpret_cast<int*>(srow + blk), __float_as_int(m4));
+                else
+                  srow[blk] = fmaxf(m4, prev);
+              }
+              // this lane's window is the first of block blk + 1, which starts
+              // the next quadrant (or tile)
+              if (lane == 31 && blk + 1 <= cur &&
+                  INFLLMV2_CHECK(ctx.status, score_row_offset(t) - row0 + blk + 1 < slab))
+                atomicMax(reinterpret_cast<int*>(srow + blk + 1), __float_as_int(S[tl]));
+            }
           }
         }
+      }
+      if (it == n_t - 1) {
+        // merge the two column halves of row r of query tile qi
+        if (hf & 1) {
+          sm.part_m[hf][r] = m_run;
+          sm.part_l[hf][r] = l_run;
+        }
+        named_bar_sync(bar_sync_all, kEpiThreads);
+        if (!(hf & 1)) {
+          const float m2 = sm.part_m[hf + 1][r];
+          const float mm = fmaxf(m_run, m2);
+          float ll = 0.f;
+          if (mm > -INFINITY) {
+            if (m_run > -INFINITY) ll += l_run * fast_exp2((m_run - mm) * scale_log2);
+            if (m2 > -INFINITY) ll += sm.part_l[hf + 1][r] * fast_exp2((m2 - mm) * scale_log2);
+          }
+          sm.nlse2[qi * kRows + r] = my_v > 0 ? -(mm * scale_log2 + __log2f(ll)) : -INFINITY;
+        }
+        // Blocks 8k start a 32-lane quadrant of pass 2: their windows come
+        // from two warps (the first one is the previous quadrant's last
+        // lane), which combine them by atomic max on the score's bits
+        // (scores are >= 0 or -inf, so integer order is float order).
+        // Start them at -inf.
+        for (int e = threadIdx.x - 64; e < kQT * TPT * (t_last / (8 * kBlock) + 1);
+             e += kEpiThreads) {
+          const int tok = e % (kQT * TPT), k8 = 8 * (e / (kQT * TPT));
+          const int t = t0 + tok;
+          if (t < q_end && k8 <= t / kBlock &&
+              INFLLMV2_CHECK(ctx.status, score_row_offset(t) - row0 + k8 < slab))
+            srow_base[score_row_offset(t) - row0 + k8] = -INFINITY;
+        }
+        named_bar_sync(bar_sync_all, kEpiThreads);
       }
     }
     // blocks past the last compressed-key tile have no visible window, except
     // block 32 n_t (a quadrant start, combined above), whose window before it
     // is the final tile's last
     if (!*abort_flag) {
-      for (int tok = hf * TPH + r; tok < (hf + 1) * TPH; tok += 128) {
+      for (int tok = hf * (kQT * TPT / kEpiWG) + r; tok < (hf + 1) * (kQT * TPT / kEpiWG);
+           tok += 128) {
         const int t = t0 + tok;
         if (t >= q_end) continue;
         const int cur = t / kBlock;
@@ -383,11 +419,13 @@ template <int G>
 int launch_score_g(const Geometry& g, const CUtensorMap& tq, const CUtensorMap& tk, float* scores,
                    const DevCtx& ctx, cudaStream_t st) {
   constexpr int TPT = kRows / G;
-  const size_t smem = 1024 + kTileBytes + kKcBytes * kStages + sizeof(ScoreSmem);
+  const size_t smem = 1024 + kQBytes + kKcBytes * kStages + sizeof(ScoreSmem);
+  static_assert(1024 + kQBytes + kKcBytes * kStages + sizeof(ScoreSmem) <= 227 * 1024,
+                "scoring tiles exceed the shared memory of a CTA");
   static std::atomic<uint64_t> smem_set{0};
   if (int e = set_smem_limit(score_blocks_kernel<G>, smem, smem_set)) return e;
   const int n_qt = (g.Tq + TPT - 1) / TPT;
-  const unsigned grid = static_cast<unsigned>(n_qt) * g.B * g.Hkv;
+  const unsigned grid = static_cast<unsigned>((n_qt + kQT - 1) / kQT) * g.B * g.Hkv;
   score_blocks_kernel<G><<<grid, kThreads, smem, st>>>(tq, tk, scores, g.B, g.q0, g.Tq, g.Hkv, g.n_c,
                                                        g.scale_log2, ctx);
   return cudaGetLastError() == cudaSuccess ? INFLLMV2_OK : INFLLMV2_ERR_CUDA;
