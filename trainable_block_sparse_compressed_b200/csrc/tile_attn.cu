@@ -326,7 +326,8 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
     //    V tile.
     if (lane == 0) {
       const bool pv_role = warp == 10;
-      constexpr uint32_t idesc_s = instr_desc_bf16(128, C::H, 0, 0);
+      constexpr uint32_t idesc_s =
+          instr_desc_bf16(128, MODE == kTileCompressed ? KT : C::H, 0, 0);
       constexpr uint32_t idesc_pv = instr_desc_bf16(128, 128, 0, 1);
       int qk = 0, ik = 0;
       int64_t gt = 0;
@@ -378,11 +379,15 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
             const uint32_t k_addr = smem_u32(sKV + s * C::kStageBytes);
             for (int w = 0; ok && w < 2; ++w) {
               // S_w(gt), the half of warpgroup w (N = KT/2 keys), needs its
-              // half of the TMEM buffer: P_w(gt-2) until P V_w(gt-2) completed
+              // half of the TMEM buffer: P_w(gt-2) until P V_w(gt-2) completed.
+              // (Compressed stream: N = KT/2 = 32 would leave the tensor core
+              // waiting on issue, so S is one N = KT product after both.)
               if (gt >= 2 && !(ok = tile_wait(&sm.pv_done[gt & 1][w],
                                               static_cast<uint32_t>(((gt >> 1) & 1) ^ 1), ctx,
                                               abort_flag)))
                 break;
+              if (MODE == kTileCompressed && w == 0) continue;
+              const int w0 = MODE == kTileCompressed ? 0 : w;  // first half of the product
               tc_fence_after();
 #pragma unroll
               for (int kk = 0; kk < 8 * C::KP; ++kk) {
@@ -390,7 +395,7 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
                 // 64-channel half; plane p, half h at (2p + h) * KT rows, the
                 // warpgroup's keys w * KT/2 rows further
                 const uint32_t off =
-                    ((kk >> 2) & 1) * (KT * 128) + (kk & 3) * 32 + w * (C::H * 128);
+                    ((kk >> 2) & 1) * (KT * 128) + (kk & 3) * 32 + w0 * (C::H * 128);
                 const uint64_t qd = smem_desc(
                     q_addr + ((kk >> 2) & 1) * (C::kQBytes / 2) + (kk & 3) * 32, 16, 1024, 2);
                 // (union: packed tiles, block w at w * 16 KB, K-major no
@@ -400,9 +405,10 @@ __global__ void __launch_bounds__(TileCfg<MODE>::kThreads, 1)
                     MODE == kTileUnion
                         ? smem_desc(k_addr + w * 16384 + kk * 256, 128, 2048, 0)
                         : smem_desc(k_addr + (kk >> 3) * (2 * KT * 128) + off, 16, 1024, 2);
-                umma_bf16(tmem + static_cast<uint32_t>(gt & 1) * KT + w * C::H, qd, kd, idesc_s,
+                umma_bf16(tmem + static_cast<uint32_t>(gt & 1) * KT + w0 * C::H, qd, kd, idesc_s,
                           kk > 0 ? 1u : 0u);
               }
+              if (MODE == kTileCompressed) umma_commit(&sm.s_full[gt & 1][0]);
               umma_commit(&sm.s_full[gt & 1][w]);
             }
             if (!ok) break;
