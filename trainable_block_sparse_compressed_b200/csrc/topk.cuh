@@ -12,7 +12,8 @@
 // Scores become order-preserving 32-bit keys (non-candidates get key 0), each
 // lane holds VPL keys in registers (block i at lane i % 32, slot i / 32), and
 // the warp finds the exact free-th largest key tau by a most-significant-bit-
-// first search: 32 rounds of "count keys >= candidate".  Blocks with key > tau
+// first search: up to 32 rounds of "count keys >= candidate", stopping early
+// once exactly the free slots hold keys >= the candidate.  Blocks with key > tau
 // are kept; among keys == tau the lowest indices fill the remaining slots,
 // ranked with ballots in index order.
 #pragma once
@@ -58,6 +59,9 @@ __device__ __forceinline__ void warp_select_row(const float* srow, int cur, int 
       for (int s = 0; s < VPL; ++s) cnt += key[s] >= c ? 1 : 0;
       cnt = __reduce_add_sync(0xffffffffu, cnt);
       if (cnt >= free_slots) tau = c;
+      // exactly free_slots keys are >= c: they are the free_slots largest,
+      // with no tie at the boundary, so the remaining bits change nothing
+      if (cnt == free_slots) break;
     }
     int gt = 0;
 #pragma unroll
@@ -167,7 +171,12 @@ __device__ __forceinline__ void cta_select_row(const float* srow, int cur, int t
       int n = 0;
 #pragma unroll
       for (int s = 0; s < PER; ++s) n += key[s] >= c ? 1 : 0;
-      if (cta_count<NT>(n, cnt_buf, round) >= free_slots) tau = c;
+      const int tot = cta_count<NT>(n, cnt_buf, round);
+      if (tot >= free_slots) tau = c;
+      if (tot == free_slots) {  // the free_slots largest keys are exactly those >= c
+        ++round;                // the next count uses the other buffer
+        break;
+      }
     }
     int n = 0;
 #pragma unroll
