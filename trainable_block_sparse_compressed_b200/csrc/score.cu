@@ -74,7 +74,7 @@ struct ScoreSmem {
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
-  float nlse2[kQT * kRows];          // per query row: minus the log2-domain LSE
+  alignas(16) float nlse2[kQT * kRows];  // per query row: minus the log2-domain LSE
   float part_m[kEpiWG][kRows], part_l[kEpiWG][kRows];  // pass 1: each column half's max / sum
 };
 
@@ -315,17 +315,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int t = tq0 + tok;
             const int v = t < q_end ? min(n_c, visible_windows(t)) : 0;
             float sum;
-            if constexpr (G >= 2) {
-              // head pairs: one packed FMA for both arguments, one packed add
+            if constexpr (G >= 4) {
+              // head pairs: one packed FMA for both arguments, one packed add;
+              // the heads' -LSE four at a time (one 128-bit shared load)
               const float2 sl2x2 = make_float2(scale_log2, scale_log2);
-              const float2* nl = reinterpret_cast<const float2*>(sm.nlse2 + qi * kRows + tok * G);
+              const float4* nl = reinterpret_cast<const float4*>(sm.nlse2 + qi * kRows + tok * G);
               float2 a2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-              for (int h = 0; h < G; h += 2) {
-                const float2 e = fma2(make_float2(x[tl * G + h], x[tl * G + h + 1]), sl2x2, nl[h / 2]);
-                a2[(h >> 1) & 1] = add2(a2[(h >> 1) & 1], make_float2(fast_exp2(e.x), fast_exp2(e.y)));
+              for (int h = 0; h < G; h += 4) {
+                const float4 n4 = nl[h / 4];
+                const float2 e0 = fma2(make_float2(x[tl * G + h], x[tl * G + h + 1]), sl2x2,
+                                       make_float2(n4.x, n4.y));
+                const float2 e1 = fma2(make_float2(x[tl * G + h + 2], x[tl * G + h + 3]), sl2x2,
+                                       make_float2(n4.z, n4.w));
+                a2[0] = add2(a2[0], make_float2(fast_exp2(e0.x), fast_exp2(e0.y)));
+                a2[1] = add2(a2[1], make_float2(fast_exp2(e1.x), fast_exp2(e1.y)));
               }
               sum = (a2[0].x + a2[0].y) + (a2[1].x + a2[1].y);
+            } else if constexpr (G == 2) {
+              const float2 e = fma2(make_float2(x[2 * tl], x[2 * tl + 1]),
+                                    make_float2(scale_log2, scale_log2),
+                                    *reinterpret_cast<const float2*>(sm.nlse2 + qi * kRows + 2 * tok));
+              sum = fast_exp2(e.x) + fast_exp2(e.y);
             } else {
               sum = fast_exp2(fmaf(x[tl], scale_log2, sm.nlse2[qi * kRows + tok]));
             }
