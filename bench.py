@@ -248,12 +248,14 @@ def run_prefill(api, wl, w, steps, warmup, dist, flush, time_e2e=True, clocks=No
     useful_score_flops = float(2 * 128 * Hq * B * v.sum())
     executed_score_flops = 0.0
     tpt = 128 // G
-    for t0 in range(0, T, tpt):
-        tl = min(t0 + tpt - 1, T - 1)
+    # a scoring CTA takes two query tiles (256 rows) and streams the windows
+    # its later tile sees; both tiles run both passes over them
+    for t0 in range(0, T, 2 * tpt):
+        tl = min(t0 + 2 * tpt - 1, T - 1)
         vt = 0 if tl < 31 else min(n_c, (tl - 31) // 16 + 1)
         nt = (vt + 127) // 128
         # pass 1 multiplies the hi plane only (K = 128), pass 2 hi and lo (K = 256)
-        executed_score_flops += (2 * 128 * 128 * 128 + 2 * 128 * 128 * 256) * nt
+        executed_score_flops += 2 * (2 * 128 * 128 * 128 + 2 * 128 * 128 * 256) * nt
     executed_score_flops *= B * Hkv
     idx_np = idx.cpu().numpy()
     cur = (np.arange(T) // 64)[None, None, :, None]
@@ -286,7 +288,9 @@ def run_prefill(api, wl, w, steps, warmup, dist, flush, time_e2e=True, clocks=No
     out = dict(ms=ms, step_ms=step_ms, kernels=kern, tokens=B * T, gather=gather,
                useful_attn_flops=useful_attn_flops, useful_score_flops=useful_score_flops,
                executed_score_flops=executed_score_flops, executed_attn_flops=executed_attn_flops,
-               clocks=clk, launches_per_step=5)
+               clocks=clk,
+               # compress, score, top-k, (union lists,) pack, attention
+               launches_per_step=6 if G >= 4 else 5)
     if chunk_len:
         out["chunk"] = time_chunk(api, p, Q, K, V, Kc, chunk_len, steps, warmup, flush)
     if time_e2e:
