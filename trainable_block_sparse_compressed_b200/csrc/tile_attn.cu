@@ -100,8 +100,8 @@ struct TileSmem {
   uint64_t o_free, drain;
   uint32_t tmem_base;
   int abort_flag;
-  // per tile parity and warpgroup: a row's half maximum; at an item's end
-  // the parity after its last tile holds the rows' half sums
+  // at an item's end, for the merge: [0] each warpgroup's reference maximum
+  // and [1] its sum, per row
   float xch[2][2][128];
 };
 
